@@ -1,0 +1,197 @@
+/*
+ * kvz.h — C ABI of libkvz, a B200 (sm_100a) implementation of the KVzip
+ * query-agnostic KV-cache compression hot path:
+ *
+ *   score   -> S_{l,h}[j], the maximum cross-attention a context key receives
+ *              while the model reconstructs the context
+ *   select  -> the kept key indices (top ratio, per head or across all heads)
+ *   compact -> the kept K/V rows gathered, in key order, into a packed cache
+ *
+ * Definitions follow "KVzip: Query-Agnostic KV Cache Compression with Context
+ * Reconstruction" (analysis report, §2.1 problem statement, §3.2 "KV importance
+ * scoring" and its equation for S_{l,h}, §4.1 "eviction structure").  The
+ * keep-count rounding m = floor(rho * n) follows the SelKV page (§3.1).
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     never allocates device memory; scratch space is passed in ("workspace")
+ *     with its size given by the matching *_workspace_size() function.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and returns after enqueueing its kernels.
+ *   - The return value reports errors the host can detect before launching:
+ *     null pointers, unsupported head dimension, bad sizes, misalignment,
+ *     aliasing, short workspace, and launch failures (KVZ_ERR_CUDA).
+ *   - `d_status` (nullable) is a device int32 the kernels write when they
+ *     detect an error on the device (first error wins; the library never
+ *     clears it).  Read it after synchronising the stream.  Codes are the
+ *     kvz_status values.
+ *   - Tensors are row-major and densely packed.  bf16 tensors are IEEE
+ *     bfloat16 bit patterns.  Every base pointer must be 16-byte aligned.
+ *   - Head index b enumerates the B = L*H KV heads of a call layer-major
+ *     (b = l*H + h), so a whole model's cache is one call.
+ *   - Results are deterministic: identical inputs give bit-identical S, idx,
+ *     counts, offsets and compacted rows, independent of scheduling.
+ */
+#ifndef KVZ_H_
+#define KVZ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvz_status {
+  KVZ_OK = 0,
+  KVZ_ERR_INVALID_ARG = 1,   /* null pointer, size out of range, bad mode/ratio/scale */
+  KVZ_ERR_UNSUPPORTED = 2,   /* head dimension d not in {64, 128} */
+  KVZ_ERR_ALIGNMENT = 3,     /* a base pointer or leading dimension is not 16-byte aligned */
+  KVZ_ERR_WORKSPACE = 4,     /* workspace missing or smaller than *_workspace_size() */
+  KVZ_ERR_CUDA = 5,          /* a CUDA runtime/driver call or kernel launch failed */
+  KVZ_ERR_INVALID_SCORE = 6, /* device: a score was NaN or negative (valid: +0 .. +inf) */
+  KVZ_ERR_TIMEOUT = 7        /* device: a bounded wait inside a kernel expired */
+} kvz_status;
+
+typedef enum kvz_mode {
+  KVZ_PER_HEAD = 0,          /* keep floor(ratio*n_c) keys in every head */
+  KVZ_GLOBAL = 1             /* keep floor(ratio*B*n_c) keys across all B heads */
+} kvz_mode;
+
+/* Library version, as 10000*major + 100*minor + patch. */
+int kvz_version(void);
+
+/* Human-readable name of a kvz_status value (static string, never NULL). */
+const char* kvz_status_string(int status);
+
+/* ------------------------------------------------------------------------ */
+/* Scoring.                                                                  */
+/*                                                                          */
+/* KVzip §3.2: for each KV head b, the repeat-prompt + context input of      */
+/* n_in = n_prompt + n_c tokens gives grouped queries Q_b (G x n_in x d) and */
+/* keys K_b = [K_ctx_b ; K_in_b] ((n_c + n_in) x d).  With                   */
+/*     A_b = Softmax(scale * Q_b K_b^T)  (per query row, causal),            */
+/* sliced to the n_c context-key columns, the score is                      */
+/*     S_b[j] = max over g < G, i < n_in of A_b[g, i, j],   j < n_c.         */
+/* Causality: input position i (0-based, prompt first) sees every context   */
+/* key and the input keys 0..i (its own position included).  The softmax    */
+/* is normalised over all visible keys (context and input) before slicing.  */
+/* The attention matrix is never materialised.                              */
+/*                                                                          */
+/* Layouts (bf16):  Q     [B][G][n_in][d]                                    */
+/*                  K_ctx [B][n_c][d]                                        */
+/*                  K_in  [B][n_in][d]                                       */
+/* Output:          S     [B][n_c] fp32, values in [0, 1] up to rounding.    */
+/*                                                                          */
+/* Work is done in row chunks of `row_chunk` input positions (0 = all rows  */
+/* in one pass; otherwise a positive multiple of 256).  Chunks merge by an   */
+/* exact max, so the result does not depend on row_chunk; only the          */
+/* workspace size does.  Limits: d in {64,128}; G >= 1; n_c, n_in >= 1;     */
+/* B*G <= 2^31-1; n_c, n_in <= 2^31-1; scale finite and > 0.                */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of workspace kvz_score needs: B*G*P*4 rounded up to 256, where P is
+ * the row count of one chunk, min(row_chunk or n_in, n_in), rounded up to a
+ * multiple of 256.  Returns 0 for invalid arguments. */
+size_t kvz_score_workspace_size(int64_t B, int G, int64_t n_in, int64_t row_chunk);
+
+/* Full scoring: zero-fills S, then for each row chunk runs pass 1 (row
+ * log-sum-exp) and pass 2 (context-key column max).  `workspace` holds the
+ * per-row base-2 log-sum-exp of the current chunk. */
+kvz_status kvz_score(const void* Q, const void* K_ctx, const void* K_in,
+                     int64_t B, int G, int64_t n_c, int64_t n_in, int d,
+                     float scale, int64_t row_chunk, float* S,
+                     void* workspace, size_t workspace_bytes,
+                     int32_t* d_status, cudaStream_t stream);
+
+/* Pass 1 alone, for input rows i in [i_begin, i_end):
+ *     lse2[(b*G + g)*ld_lse2 + (i - i_begin)] =
+ *         log2( sum over visible u of 2^(scale*log2(e) * <q_{b,g,i}, k_{b,u}>) )
+ * Entries for padding rows, i in [i_end, i_begin + roundup(i_end-i_begin,256)),
+ * are set to +inf (they then never contribute in pass 2).
+ * Requires i_begin % 256 == 0, 0 <= i_begin < i_end <= n_in,
+ * ld_lse2 >= roundup(i_end - i_begin, 256) and ld_lse2 % 4 == 0. */
+kvz_status kvz_score_lse2(const void* Q, const void* K_ctx, const void* K_in,
+                          int64_t B, int G, int64_t n_c, int64_t n_in, int d,
+                          float scale, int64_t i_begin, int64_t i_end,
+                          float* lse2, int64_t ld_lse2,
+                          int32_t* d_status, cudaStream_t stream);
+
+/* Pass 2 alone, for the rows whose lse2 pass 1 produced (same i_begin,
+ * i_end, ld_lse2):
+ *     S[b*n_c + j] = max(S[b*n_c + j],
+ *                        max over g, i of 2^(scale*log2(e)*<q_{b,g,i}, k_{b,j}> - lse2[b,g,i]))
+ * If `accumulate` is 0, S is first set to 0 (so the call computes the
+ * chunk's score alone); otherwise S must already hold values >= +0 and the
+ * result is merged by max (exact).  Context keys are visible to every input
+ * row, so this pass has no mask and never reads K_in. */
+kvz_status kvz_score_colmax(const void* Q, const void* K_ctx,
+                            int64_t B, int G, int64_t n_c, int64_t n_in, int d,
+                            float scale, int64_t i_begin, int64_t i_end,
+                            const float* lse2, int64_t ld_lse2,
+                            float* S, int accumulate,
+                            int32_t* d_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Selection.                                                                */
+/*                                                                          */
+/* KVzip §4.1 keeps the r% highest-scoring KV pairs across all heads         */
+/* (KVZ_GLOBAL); KVZ_PER_HEAD keeps r% of every head.  The keep count of a   */
+/* segment of N scores is k = floor(ratio * N) computed in IEEE double.      */
+/* The kept set is unique: the k largest scores, ties at the threshold       */
+/* going to the lower flattened index (b*n_c + j).  Equivalently, it is the  */
+/* first k entries of a stable sort by descending score.                     */
+/*                                                                          */
+/* Input:  S [B][n_c] fp32, every value in [+0, +inf] (+inf forces a key to  */
+/*         be kept; -0 counts as +0).  A NaN or negative score sets          */
+/*         KVZ_ERR_INVALID_SCORE in d_status and is treated as +0.           */
+/* Output: counts[b]   number kept in head b (int32, B entries)              */
+/*         offsets[b]  sum of counts[0..b-1] (int64, B+1 entries)            */
+/*         idx[offsets[b] + p], p < counts[b]: kept key positions j of head  */
+/*                     b, strictly ascending (int32).                        */
+/* idx_capacity must be at least B*floor(ratio*n_c) (per head) or            */
+/* floor(ratio*B*n_c) (global).  ratio must lie in [0, 1].                   */
+/* ------------------------------------------------------------------------ */
+
+/* Number kept from a segment of n scores: floor(ratio * n) in IEEE double. */
+int64_t kvz_keep_count(int64_t n, double ratio);
+
+/* Bytes of workspace kvz_select needs (0 for invalid arguments). */
+size_t kvz_select_workspace_size(int64_t B, int64_t n_c, int mode);
+
+kvz_status kvz_select(const float* S, int64_t B, int64_t n_c, double ratio,
+                      int mode, int32_t* idx, int64_t idx_capacity,
+                      int32_t* counts, int64_t* offsets,
+                      void* workspace, size_t workspace_bytes,
+                      int32_t* d_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Compaction.                                                               */
+/*                                                                          */
+/* KVzip §2.1: the pruned cache K_p is a subset of the full cache K_c that   */
+/* is reused for every later query.  For p < counts[b]:                      */
+/*     K_out[dst_b + p] = K[b*n_c + idx[offsets[b] + p]]   (rows of d bf16)  */
+/*     V_out[dst_b + p] = V[b*n_c + idx[offsets[b] + p]]                     */
+/* Key order is preserved because idx is ascending within a head.            */
+/*                                                                          */
+/* Out of place (K_out != K): dst_b = out_offsets[b] if out_offsets is not   */
+/*   NULL, else offsets[b] (a packed CSR cache).  K_out/V_out must hold every */
+/*   destination row and must not overlap K or V.                             */
+/* In place (K_out == K and V_out == V): dst_b = b*n_c, i.e. each head's     */
+/*   kept rows are packed to the front of its own region; rows at and after  */
+/*   counts[b] keep stale data.  out_offsets must be NULL.  Safe because a    */
+/*   kept row never moves to a higher position.                               */
+/* Layout: K, V [B][n_c][d] bf16; idx/counts/offsets as kvz_select writes.   */
+/* ------------------------------------------------------------------------ */
+kvz_status kvz_compact(const void* K, const void* V, int64_t B, int64_t n_c,
+                       int d, const int32_t* idx, const int32_t* counts,
+                       const int64_t* offsets, const int64_t* out_offsets,
+                       void* K_out, void* V_out,
+                       int32_t* d_status, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVZ_H_ */

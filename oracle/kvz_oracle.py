@@ -1,0 +1,209 @@
+"""Plain, slow CPU oracle of the KVzip hot path.  TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference arm may import this module.  The product path (the CUDA library and
+its Python binding) never calls it and shares no code with it.
+
+What it computes (KVzip analysis report, §3.2 "KV importance scoring"):
+for one KV head with grouped queries Q (G x n_in x d) of the repeat-prompt +
+context input and keys K = [K_ctx ; K_in] ((n_c + n_in) x d),
+
+    A = Softmax(scale * Q K^T)        per query row, over the visible keys
+    S[j] = max_{g, i} A[g, i, j]      for the n_c context keys j
+
+The pages write Softmax(Q K^T) with no scale and no mask.  Readings taken here
+(each listed with its reason in the design notes):
+  * the logits are multiplied by ``scale`` (the usual 1/sqrt(d));
+  * the reconstruction forward pass is a causal LM pass: input position i
+    (0-based, repeat prompt first, then the context) sees all n_c context keys
+    and the input keys 0..i, its own position included;
+  * each row is normalised over every key it sees (context and input), and
+    only then sliced to the context columns (§3.2 slices A, not the logits);
+  * every input row, repeat-prompt rows included, enters the max.
+
+Selection (§4.1 "eviction structure": keep the r% highest scores across all
+heads; SelKV page §3.1 sets the kept count to floor(rho * n)) and compaction
+(§2.1: the pruned cache is a subset of the full cache) are written as a stable
+sort and a fancy-index gather.
+
+Arithmetic is float64 throughout.  Inputs that are bf16 on the device are
+decoded exactly from their bit patterns (``bf16_bits_to_f64``).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "bf16_bits_to_f64",
+    "row_logits",
+    "row_lse",
+    "score",
+    "keep_count",
+    "select",
+    "compact",
+    "visible_pairs",
+]
+
+
+# ---------------------------------------------------------------------------
+# Input decoding
+# ---------------------------------------------------------------------------
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """Exact float64 value of bfloat16 bit patterns (uint16 / int16 array).
+
+    A bfloat16 is the upper half of an IEEE binary32, so shifting the 16 bits
+    into the high half of a 32-bit word gives the same number as a float32.
+    """
+    b = np.asarray(bits)
+    if b.dtype not in (np.uint16, np.int16):
+        raise TypeError("expected uint16/int16 bit patterns, got %s" % b.dtype)
+    u32 = b.view(np.uint16).astype(np.uint32) << np.uint32(16)
+    return u32.view(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Scoring (KVzip §3.2)
+# ---------------------------------------------------------------------------
+def _check_head(Q, K_ctx, K_in):
+    Q = np.asarray(Q, dtype=np.float64)
+    K_ctx = np.asarray(K_ctx, dtype=np.float64)
+    K_in = np.asarray(K_in, dtype=np.float64)
+    if Q.ndim != 3 or K_ctx.ndim != 2 or K_in.ndim != 2:
+        raise ValueError("expected Q[G,n_in,d], K_ctx[n_c,d], K_in[n_in,d]")
+    G, n_in, d = Q.shape
+    if K_in.shape != (n_in, d) or K_ctx.shape[1] != d:
+        raise ValueError("shape mismatch between Q, K_ctx and K_in")
+    return Q, K_ctx, K_in
+
+
+def row_logits(q, K_ctx, K_in, i, scale):
+    """Logits z_u = scale * <q, k_u> of input row i over the keys it sees.
+
+    The unified key index u runs over the n_c context keys, then the input
+    keys; input row i sees u < n_c + i + 1 (causal, own position included).
+    Returns a float64 vector of length n_c + i + 1.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    K_ctx = np.asarray(K_ctx, dtype=np.float64)
+    K_in = np.asarray(K_in, dtype=np.float64)
+    keys = np.concatenate([K_ctx, K_in[: i + 1]], axis=0)
+    return float(scale) * (keys @ q)
+
+
+def row_lse(q, K_ctx, K_in, i, scale):
+    """Natural log-sum-exp of row i's visible logits (stable: max + log sum)."""
+    z = row_logits(q, K_ctx, K_in, i, scale)
+    m = np.max(z)
+    return float(m + np.log(np.sum(np.exp(z - m))))
+
+
+def score(Q, K_ctx, K_in, scale, rows=None, row_block=256):
+    """S[j] = max over (g, i) of softmax-row value A[g, i, j], j < n_c.
+
+    Q: [G, n_in, d]; K_ctx: [n_c, d]; K_in: [n_in, d]; scale: the logit
+    multiplier (a float32 value on the device; promoted here, not recomputed).
+    ``rows`` = (i_begin, i_end) restricts the max to input rows in that range
+    (each row is still normalised over all keys it sees); None = all rows.
+    Rows are visited ``row_block`` at a time only to bound memory: every row's
+    softmax is computed whole, and the max over rows is exact in any order.
+    """
+    Q, K_ctx, K_in = _check_head(Q, K_ctx, K_in)
+    G, n_in, d = Q.shape
+    n_c = K_ctx.shape[0]
+    scale = float(scale)
+    i_begin, i_end = (0, n_in) if rows is None else (int(rows[0]), int(rows[1]))
+    K_all = np.concatenate([K_ctx, K_in], axis=0)  # unified key index u
+    u = np.arange(n_c + n_in)
+    S = np.zeros(n_c, dtype=np.float64)
+    for r0 in range(i_begin, i_end, row_block):
+        r1 = min(i_end, r0 + row_block)
+        i = np.arange(r0, r1)
+        Z = scale * np.einsum("gid,ud->giu", Q[:, r0:r1, :], K_all)
+        visible = u[None, :] <= (n_c + i)[:, None]          # [rows, keys]
+        Z = np.where(visible[None, :, :], Z, -np.inf)
+        m = np.max(Z, axis=2, keepdims=True)                 # finite: n_c >= 1
+        lse = m + np.log(np.sum(np.exp(Z - m), axis=2, keepdims=True))
+        A_ctx = np.exp(Z[:, :, :n_c] - lse)                  # slice after softmax
+        S = np.maximum(S, A_ctx.max(axis=(0, 1)))
+    return S
+
+
+def visible_pairs(G, n_c, n_in):
+    """Number of (query row, key) pairs the causal softmax covers for a head."""
+    return G * (n_in * n_c + n_in * (n_in + 1) // 2)
+
+
+# ---------------------------------------------------------------------------
+# Selection (KVzip §4.1; keep count floor(rho*n) from the SelKV page §3.1)
+# ---------------------------------------------------------------------------
+def keep_count(n, ratio):
+    """floor(ratio * n) with the product rounded once in IEEE double."""
+    ratio = float(ratio)
+    if not (0.0 <= ratio <= 1.0):
+        raise ValueError("ratio must lie in [0, 1]")
+    return int(math.floor(ratio * int(n)))
+
+
+def select(S, ratio, mode):
+    """Top-ratio selection with ties to the lower flattened index.
+
+    S: [B, n_c] float32 scores (>= 0).  mode: "per_head" keeps
+    floor(ratio*n_c) of every head; "global" keeps floor(ratio*B*n_c) across
+    all heads.  Returns (idx int32 concatenated per head, ascending within a
+    head; counts int32 [B]; offsets int64 [B+1]).
+    """
+    S = np.asarray(S, dtype=np.float32)
+    if S.ndim != 2:
+        raise ValueError("S must be [B, n_c]")
+    B, n_c = S.shape
+    if np.isnan(S).any() or (S < 0).any():
+        raise ValueError("scores must be non-negative and not NaN")
+    if mode == "per_head":
+        per_head = []
+        k = keep_count(n_c, ratio)
+        for b in range(B):
+            order = np.argsort(-S[b], kind="stable")  # descending, ties by index
+            per_head.append(np.sort(order[:k]))
+    elif mode == "global":
+        flat = S.reshape(-1)
+        k = keep_count(B * n_c, ratio)
+        order = np.argsort(-flat, kind="stable")
+        kept = np.sort(order[:k])
+        heads = kept // n_c
+        per_head = [kept[heads == b] - b * n_c for b in range(B)]
+    else:
+        raise ValueError("mode must be 'per_head' or 'global'")
+    counts = np.array([len(x) for x in per_head], dtype=np.int32)
+    offsets = np.zeros(B + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    idx = (np.concatenate(per_head) if B else np.zeros(0)).astype(np.int32)
+    return idx, counts, offsets
+
+
+# ---------------------------------------------------------------------------
+# Compaction (KVzip §2.1: the pruned cache is a subset of the full cache)
+# ---------------------------------------------------------------------------
+def compact(K, V, idx, counts, offsets, out_offsets=None):
+    """Gather kept rows in key order.
+
+    K, V: [B, n_c, d] arrays (any dtype; bf16 caches are passed as uint16
+    bits so the copy is exact).  Returns (K_out, V_out) as a packed
+    [sum(counts), d] pair when out_offsets is None; otherwise arrays sized to
+    the largest destination row with each head's rows at out_offsets[b].
+    """
+    K = np.asarray(K)
+    V = np.asarray(V)
+    B, n_c, d = K.shape
+    counts = np.asarray(counts, dtype=np.int64)
+    offsets = np.asarray(offsets, dtype=np.int64)
+    dst = offsets if out_offsets is None else np.asarray(out_offsets, dtype=np.int64)
+    rows = int(max([dst[b] + counts[b] for b in range(B)] + [0]))
+    K_out = np.zeros((rows, d), dtype=K.dtype)
+    V_out = np.zeros((rows, d), dtype=V.dtype)
+    for b in range(B):
+        sel = np.asarray(idx[offsets[b]: offsets[b] + counts[b]], dtype=np.int64)
+        K_out[dst[b]: dst[b] + counts[b]] = K[b][sel]
+        V_out[dst[b]: dst[b] + counts[b]] = V[b][sel]
+    return K_out, V_out

@@ -1,0 +1,282 @@
+"""Pins of the CPU oracle to facts outside itself (no GPU needed).
+
+Each test checks the oracle against something the KVzip definition or plain
+mathematics fixes: hand-worked examples, closed forms, a textbook softmax,
+50-digit brute force, invariants of the definition, exhaustive search.
+"""
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import mpmath
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from oracle import kvz_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "kvzip_hand_examples.json")
+
+
+def _rand_head(rng, G, n_c, n_in, d, scale_keys=1.0):
+    Q = rng.standard_normal((G, n_in, d))
+    K_ctx = rng.standard_normal((n_c, d)) * scale_keys
+    K_in = rng.standard_normal((n_in, d)) * scale_keys
+    return Q, K_ctx, K_in
+
+
+# --------------------------------------------------------------------------
+# Hand-worked examples (tests/golden)
+# --------------------------------------------------------------------------
+def test_hand_examples():
+    with open(GOLDEN) as f:
+        data = json.load(f)
+    for ex in data["examples"]:
+        S = orc.score(np.array(ex["Q"]), np.array(ex["K_ctx"]), np.array(ex["K_in"]),
+                      ex["scale"])
+        want = np.array([float(Fraction(s)) for s in ex["S"]])
+        np.testing.assert_allclose(S, want, rtol=1e-14, atol=0, err_msg=ex["name"])
+
+
+# --------------------------------------------------------------------------
+# Closed forms
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("G,n_c,n_in,d", [(1, 1, 1, 4), (4, 7, 12, 8), (3, 33, 40, 16),
+                                          (2, 64, 5, 8)])
+def test_identical_keys_give_uniform_rows(G, n_c, n_in, d):
+    # Every row is uniform over its n_c + i + 1 visible keys; the largest
+    # weight a context key gets is at i = 0: S[j] = 1 / (n_c + 1).
+    rng = np.random.default_rng(1)
+    v = rng.standard_normal(d)
+    Q = rng.standard_normal((G, n_in, d)) * 3.0
+    S = orc.score(Q, np.tile(v, (n_c, 1)), np.tile(v, (n_in, 1)), 0.37)
+    np.testing.assert_allclose(S, 1.0 / (n_c + 1), rtol=1e-13)
+
+
+def test_zero_queries_give_uniform_rows():
+    rng = np.random.default_rng(2)
+    n_c, n_in = 19, 23
+    _, K_ctx, K_in = _rand_head(rng, 1, n_c, n_in, 8, scale_keys=5.0)
+    S = orc.score(np.zeros((3, n_in, 8)), K_ctx, K_in, 1.0)
+    np.testing.assert_allclose(S, 1.0 / (n_c + 1), rtol=1e-13)
+
+
+def test_single_row_equals_textbook_softmax():
+    # G = 1, n_in = 1: S is the first n_c entries of one softmax row over the
+    # n_c context keys and the single input key.
+    rng = np.random.default_rng(3)
+    for n_c, d in [(1, 4), (10, 8), (100, 64)]:
+        Q, K_ctx, K_in = _rand_head(rng, 1, n_c, 1, d)
+        scale = 1.0 / math.sqrt(d)
+        z = scale * (np.concatenate([K_ctx, K_in]) @ Q[0, 0])
+        np.testing.assert_allclose(orc.score(Q, K_ctx, K_in, scale),
+                                   scipy.special.softmax(z)[:n_c], rtol=1e-13)
+
+
+def test_dominant_key_closed_form():
+    # One key aligned with the only query row: S[j*] = 1 / (1 + sum_{u != j*}
+    # exp(z_u - z_j*)), tending to 1 as the alignment grows; other keys get
+    # S[j] = exp(z_j - z_j*) * S[j*].
+    rng = np.random.default_rng(4)
+    n_c, d = 12, 8
+    Q, K_ctx, K_in = _rand_head(rng, 1, n_c, 1, d)
+    for alpha in (1.0, 4.0, 16.0):
+        K2 = K_ctx.copy()
+        K2[5] = alpha * Q[0, 0]
+        z = np.concatenate([K2, K_in]) @ Q[0, 0]
+        want5 = 1.0 / (1.0 + sum(math.exp(z[u] - z[5]) for u in range(n_c + 1) if u != 5))
+        S = orc.score(Q, K2, K_in, 1.0)
+        assert abs(S[5] - want5) <= 1e-14
+        for j in range(n_c):
+            assert abs(S[j] - math.exp(z[j] - z[5]) * want5) <= 1e-14
+    assert S[5] > 1 - 1e-12
+
+
+# --------------------------------------------------------------------------
+# Brute force at 50 digits (independent restatement of the definition)
+# --------------------------------------------------------------------------
+def _mp_score(Q, K_ctx, K_in, scale):
+    mpmath.mp.dps = 50
+    G, n_in, d = Q.shape
+    n_c = K_ctx.shape[0]
+    keys = [list(map(mpmath.mpf, k)) for k in np.concatenate([K_ctx, K_in])]
+    best = [mpmath.mpf(0)] * n_c
+    sc = mpmath.mpf(scale)
+    for g in range(G):
+        for i in range(n_in):
+            q = list(map(mpmath.mpf, Q[g, i]))
+            w = [mpmath.e ** (sc * mpmath.fsum(a * b for a, b in zip(q, keys[u])))
+                 for u in range(n_c + i + 1)]
+            tot = mpmath.fsum(w)
+            for j in range(n_c):
+                best[j] = max(best[j], w[j] / tot)
+    return np.array([float(x) for x in best])
+
+
+@pytest.mark.parametrize("seed,G,n_c,n_in,d", [(10, 1, 3, 4, 2), (11, 2, 5, 7, 4),
+                                               (12, 3, 16, 8, 8), (13, 4, 9, 2, 3)])
+def test_matches_50_digit_brute_force(seed, G, n_c, n_in, d):
+    rng = np.random.default_rng(seed)
+    Q, K_ctx, K_in = _rand_head(rng, G, n_c, n_in, d, scale_keys=2.0)
+    scale = 1.0 / math.sqrt(d)
+    np.testing.assert_allclose(orc.score(Q, K_ctx, K_in, scale),
+                               _mp_score(Q, K_ctx, K_in, scale), rtol=1e-13, atol=0)
+
+
+# --------------------------------------------------------------------------
+# Invariants of the definition
+# --------------------------------------------------------------------------
+def test_rows_normalise_and_lse_matches_textbook():
+    rng = np.random.default_rng(5)
+    G, n_c, n_in, d = 2, 20, 9, 8
+    Q, K_ctx, K_in = _rand_head(rng, G, n_c, n_in, d)
+    for g in range(G):
+        for i in range(n_in):
+            z = orc.row_logits(Q[g, i], K_ctx, K_in, i, 0.3)
+            assert z.shape == (n_c + i + 1,)
+            lse = orc.row_lse(Q[g, i], K_ctx, K_in, i, 0.3)
+            assert abs(lse - scipy.special.logsumexp(z)) <= 1e-12
+            assert abs(np.exp(z - lse).sum() - 1.0) <= 1e-12
+
+
+def test_range_permutation_duplication_shift_chunks():
+    rng = np.random.default_rng(6)
+    G, n_c, n_in, d = 3, 50, 37, 16
+    Q, K_ctx, K_in = _rand_head(rng, G, n_c, n_in, d, scale_keys=3.0)
+    sc = 0.25
+    S = orc.score(Q, K_ctx, K_in, sc)
+    assert np.all(S >= 0) and np.all(S <= 1)
+    # context keys are visible to every row: permuting them permutes S
+    perm = rng.permutation(n_c)
+    np.testing.assert_allclose(orc.score(Q, K_ctx[perm], K_in, sc), S[perm], rtol=1e-12)
+    # a duplicated query group changes nothing (max over g)
+    Q2 = np.concatenate([Q, Q[1:2]], axis=0)
+    np.testing.assert_allclose(orc.score(Q2, K_ctx, K_in, sc), S, rtol=1e-13)
+    # adding one vector to every key shifts each row's logits by a constant
+    v = rng.standard_normal(d)
+    np.testing.assert_allclose(orc.score(Q, K_ctx + v, K_in + v, sc), S, rtol=1e-9)
+    # the max over rows splits into row chunks exactly
+    parts = [orc.score(Q, K_ctx, K_in, sc, rows=(a, min(n_in, a + 16)))
+             for a in range(0, n_in, 16)]
+    np.testing.assert_array_equal(np.maximum.reduce(parts), S)
+    # row_block only bounds memory
+    np.testing.assert_allclose(orc.score(Q, K_ctx, K_in, sc, row_block=7), S, rtol=1e-15)
+
+
+def test_visible_pairs_counts_the_causal_mask():
+    G, n_c, n_in = 3, 11, 6
+    brute = sum(n_c + i + 1 for g in range(G) for i in range(n_in))
+    assert orc.visible_pairs(G, n_c, n_in) == brute
+
+
+# --------------------------------------------------------------------------
+# bf16 decoding
+# --------------------------------------------------------------------------
+def test_bf16_decoding_exact():
+    bits = np.array([0x3F80, 0xC000, 0x7F80, 0x0001, 0x3F81, 0x8000, 0xFF80], np.uint16)
+    want = [1.0, -2.0, math.inf, 2.0 ** -133, 1.0 + 2.0 ** -7, -0.0, -math.inf]
+    got = orc.bf16_bits_to_f64(bits)
+    for a, b in zip(got, want):
+        assert a == b and math.copysign(1, a) == math.copysign(1, b)
+    rnd = torch.randn(1000).to(torch.bfloat16)
+    np.testing.assert_array_equal(orc.bf16_bits_to_f64(rnd.view(torch.int16).numpy()),
+                                  rnd.to(torch.float64).numpy())
+
+
+# --------------------------------------------------------------------------
+# Selection
+# --------------------------------------------------------------------------
+def test_keep_count_is_floor_in_double():
+    assert orc.keep_count(256, 0.3) == 76
+    assert orc.keep_count(8192, 0.3) == 2457
+    assert orc.keep_count(32 * 8 * 32768, 0.3) == 2516582
+    assert orc.keep_count(131072, 0.25) == 32768
+    assert orc.keep_count(256 * 65537, 0.1) == 1677747
+    assert orc.keep_count(10, 0.7) == 7          # 0.7*10 = 7.000000000000001
+    assert orc.keep_count(3, 0.1) == 0
+    assert orc.keep_count(5, 1.0) == 5 and orc.keep_count(5, 0.0) == 0
+    with pytest.raises(ValueError):
+        orc.keep_count(5, 1.5)
+
+
+def _canonical_by_exchange(vals, k):
+    """The unique k-subset in which every kept entry beats every dropped one
+    (greater value, or equal value and lower index), found by exhaustion."""
+    n = len(vals)
+    found = []
+    for sub in itertools.combinations(range(n), k):
+        kept = set(sub)
+        ok = all((vals[a] > vals[b]) or (vals[a] == vals[b] and a < b)
+                 for a in kept for b in range(n) if b not in kept)
+        if ok:
+            found.append(sub)
+    assert len(found) == 1
+    return list(found[0])
+
+
+def test_select_matches_exhaustive_search():
+    rng = np.random.default_rng(7)
+    for trial in range(30):
+        B, n_c = int(rng.integers(1, 4)), int(rng.integers(1, 7))
+        S = rng.choice(np.array([0.0, 0.25, 0.5, 1.0, np.inf], np.float32), size=(B, n_c))
+        ratio = float(rng.choice([0.0, 0.2, 0.3, 0.5, 0.75, 1.0]))
+        for mode in ("per_head", "global"):
+            idx, counts, offsets = orc.select(S, ratio, mode)
+            if mode == "per_head":
+                k = orc.keep_count(n_c, ratio)
+                for b in range(B):
+                    got = list(idx[offsets[b]:offsets[b + 1]])
+                    assert got == _canonical_by_exchange(list(S[b]), k)
+            else:
+                k = orc.keep_count(B * n_c, ratio)
+                want = _canonical_by_exchange(list(S.reshape(-1)), k)
+                got = [b * n_c + j for b in range(B) for j in idx[offsets[b]:offsets[b + 1]]]
+                assert got == want
+            assert offsets[-1] == len(idx) == counts.sum()
+
+
+def test_select_special_cases():
+    S = np.full((3, 10), 0.5, np.float32)
+    idx, counts, offsets = orc.select(S, 0.3, "per_head")
+    assert list(counts) == [3, 3, 3] and list(idx) == [0, 1, 2] * 3
+    idx, counts, offsets = orc.select(S, 0.3, "global")          # first 9 of 30
+    assert list(counts) == [9, 0, 0] and list(idx) == list(range(9))
+    idx, counts, _ = orc.select(S, 0.0, "global")
+    assert len(idx) == 0 and list(counts) == [0, 0, 0]
+    idx, counts, _ = orc.select(S, 1.0, "per_head")
+    assert list(idx) == list(range(10)) * 3
+    S2 = np.array([[0.1, -0.0, 0.0, np.inf]], np.float32)       # -0 ties with +0
+    idx, _, _ = orc.select(S2, 0.75, "per_head")
+    assert list(idx) == [0, 1, 3]
+    with pytest.raises(ValueError):
+        orc.select(np.array([[np.nan, 1.0]], np.float32), 0.5, "global")
+
+
+# --------------------------------------------------------------------------
+# Compaction
+# --------------------------------------------------------------------------
+def test_compact_gathers_in_order():
+    rng = np.random.default_rng(8)
+    B, n_c, d = 3, 9, 4
+    K = rng.integers(0, 2 ** 16, (B, n_c, d)).astype(np.uint16)
+    V = rng.integers(0, 2 ** 16, (B, n_c, d)).astype(np.uint16)
+    idx, counts, offsets = orc.select(rng.random((B, n_c)).astype(np.float32), 1.0, "per_head")
+    K_out, V_out = orc.compact(K, V, idx, counts, offsets)
+    np.testing.assert_array_equal(K_out, K.reshape(-1, d))      # identity at ratio 1
+    np.testing.assert_array_equal(V_out, V.reshape(-1, d))
+    S = rng.random((B, n_c)).astype(np.float32)
+    idx, counts, offsets = orc.select(S, 0.4, "global")
+    K_out, V_out = orc.compact(K, V, idx, counts, offsets)
+    for b in range(B):
+        sel = idx[offsets[b]:offsets[b + 1]]
+        assert np.all(np.diff(sel) > 0)
+        np.testing.assert_array_equal(K_out[offsets[b]:offsets[b + 1]], K[b][sel])
+        np.testing.assert_array_equal(V_out[offsets[b]:offsets[b + 1]], V[b][sel])
+    out_off = np.array([b * n_c for b in range(B)])
+    K2, _ = orc.compact(K, V, idx, counts, offsets, out_offsets=out_off)
+    for b in range(B):
+        np.testing.assert_array_equal(K2[b * n_c: b * n_c + counts[b]],
+                                      K_out[offsets[b]:offsets[b + 1]])
