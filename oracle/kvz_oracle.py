@@ -120,7 +120,7 @@ def score(Q, K_ctx, K_in, scale, rows=None, row_block=256):
     for r0 in range(i_begin, i_end, row_block):
         r1 = min(i_end, r0 + row_block)
         i = np.arange(r0, r1)
-        Z = scale * np.einsum("gid,ud->giu", Q[:, r0:r1, :], K_all)
+        Z = scale * (Q[:, r0:r1, :] @ K_all.T)                 # [G, rows, keys]
         visible = u[None, :] <= (n_c + i)[:, None]          # [rows, keys]
         Z = np.where(visible[None, :, :], Z, -np.inf)
         m = np.max(Z, axis=2, keepdims=True)                 # finite: n_c >= 1

@@ -1,0 +1,248 @@
+"""KVzip query-agnostic KV-cache compression hot path on B200 (sm_100a).
+
+Thin Python binding of the C ABI declared in ``include/kvz.h``: every
+function here only checks tensor shapes, allocates outputs/workspace with
+torch and calls the same-named C entry point in ``libkvz.so``.  All arithmetic
+runs in the library's CUDA kernels; there is no CPU fallback.  If the library
+is missing, importing works but every call raises ``KvzLibraryError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "KvzError", "KvzLibraryError", "lib", "lib_path", "STATUS",
+    "kvz_version", "kvz_keep_count",
+    "kvz_score_workspace_size", "kvz_score", "kvz_score_lse2", "kvz_score_colmax",
+    "kvz_select_workspace_size", "kvz_select", "kvz_compact",
+    "PER_HEAD", "GLOBAL",
+]
+
+PER_HEAD = 0
+GLOBAL = 1
+STATUS = {
+    0: "KVZ_OK", 1: "KVZ_ERR_INVALID_ARG", 2: "KVZ_ERR_UNSUPPORTED", 3: "KVZ_ERR_ALIGNMENT",
+    4: "KVZ_ERR_WORKSPACE", 5: "KVZ_ERR_CUDA", 6: "KVZ_ERR_INVALID_SCORE", 7: "KVZ_ERR_TIMEOUT",
+}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libkvz.so")
+
+
+class KvzLibraryError(RuntimeError):
+    """libkvz.so is missing or cannot be loaded."""
+
+
+class KvzError(RuntimeError):
+    """A libkvz call returned an error status."""
+
+    def __init__(self, fn: str, code: int):
+        super().__init__("%s failed: %s (%d)" % (fn, STATUS.get(code, "?"), code))
+        self.code = code
+
+
+_lib = None
+
+_c = ctypes
+_vp, _i64, _i32, _f32, _f64, _sz = _c.c_void_p, _c.c_int64, _c.c_int, _c.c_float, _c.c_double, _c.c_size_t
+_SIGS = {
+    "kvz_version": (_i32, []),
+    "kvz_status_string": (_c.c_char_p, [_i32]),
+    "kvz_score_workspace_size": (_sz, [_i64, _i32, _i64, _i64]),
+    "kvz_score": (_i32, [_vp, _vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _i64, _vp, _vp, _sz, _vp, _vp]),
+    "kvz_score_lse2": (_i32, [_vp, _vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _i64, _i64, _vp, _i64, _vp,
+                              _vp]),
+    "kvz_score_colmax": (_i32, [_vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _i64, _i64, _vp, _i64, _vp,
+                                _i32, _vp, _vp]),
+    "kvz_keep_count": (_i64, [_i64, _f64]),
+    "kvz_select_workspace_size": (_sz, [_i64, _i64, _i32]),
+    "kvz_select": (_i32, [_vp, _i64, _i64, _f64, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "kvz_compact": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+}
+
+
+def lib():
+    """The loaded libkvz.so (ctypes), with argument types declared."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise KvzLibraryError("libkvz.so not built (%s); run "
+                                  "`python -m query_agnostic_kv_kvz_b200.build`" % lib_path)
+        try:
+            handle = ctypes.CDLL(lib_path)
+        except OSError as e:  # pragma: no cover - depends on the machine
+            raise KvzLibraryError("cannot load %s: %s" % (lib_path, e)) from e
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise KvzError(fn, code)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("kvz: tensors must live on a CUDA device")
+
+
+def kvz_version() -> int:
+    return lib().kvz_version()
+
+
+def kvz_keep_count(n: int, ratio: float) -> int:
+    return lib().kvz_keep_count(int(n), float(ratio))
+
+
+def kvz_score_workspace_size(B: int, G: int, n_in: int, row_chunk: int = 0) -> int:
+    return lib().kvz_score_workspace_size(B, G, n_in, row_chunk)
+
+
+def _score_shapes(Q, K_ctx, K_in=None):
+    if Q.dim() != 4 or K_ctx.dim() != 3:
+        raise ValueError("expected Q[B,G,n_in,d] and K_ctx[B,n_c,d]")
+    B, G, n_in, d = Q.shape
+    if K_ctx.shape[0] != B or K_ctx.shape[2] != d:
+        raise ValueError("K_ctx shape does not match Q")
+    if K_in is not None and tuple(K_in.shape) != (B, n_in, d):
+        raise ValueError("K_in must be [B, n_in, d]")
+    for t in (Q, K_ctx, K_in):
+        if t is not None and (t.dtype != torch.bfloat16 or not t.is_contiguous()):
+            raise ValueError("Q/K must be contiguous bfloat16")
+    return B, G, n_in, d, K_ctx.shape[1]
+
+
+def kvz_score(Q, K_ctx, K_in, scale: Optional[float] = None, row_chunk: int = 0, S=None, workspace=None,
+              status=None, stream=None):
+    """S[b, j] = max_{g,i} Softmax_causal(scale * Q_b K_b^T)[g, i, j] (KVzip §3.2); returns S."""
+    _need_cuda(Q, K_ctx, K_in, S, workspace, status)
+    B, G, n_in, d, n_c = _score_shapes(Q, K_ctx, K_in)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if S is None:
+        S = torch.empty((B, n_c), dtype=torch.float32, device=Q.device)
+    need = kvz_score_workspace_size(B, G, n_in, row_chunk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check("kvz_score", lib().kvz_score(_ptr(Q), _ptr(K_ctx), _ptr(K_in), B, G, n_c, n_in, d, scale, row_chunk,
+                                        _ptr(S), _ptr(workspace), nbytes, _ptr(status), _stream(stream)))
+    return S
+
+
+def kvz_score_lse2(Q, K_ctx, K_in, i_begin: int = 0, i_end: Optional[int] = None, scale: Optional[float] = None,
+                   lse2=None, ld: Optional[int] = None, status=None, stream=None):
+    """Pass 1: base-2 log-sum-exp of input rows [i_begin, i_end); returns lse2 [B, G, ld]."""
+    _need_cuda(Q, K_ctx, K_in, lse2, status)
+    B, G, n_in, d, n_c = _score_shapes(Q, K_ctx, K_in)
+    i_end = n_in if i_end is None else i_end
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rows_pad = (i_end - i_begin + 255) // 256 * 256
+    ld = rows_pad if ld is None else ld
+    if lse2 is None:
+        lse2 = torch.empty((B, G, ld), dtype=torch.float32, device=Q.device)
+    _check("kvz_score_lse2", lib().kvz_score_lse2(_ptr(Q), _ptr(K_ctx), _ptr(K_in), B, G, n_c, n_in, d, scale,
+                                                  i_begin, i_end, _ptr(lse2), ld, _ptr(status), _stream(stream)))
+    return lse2
+
+
+def kvz_score_colmax(Q, K_ctx, lse2, i_begin: int = 0, i_end: Optional[int] = None,
+                     scale: Optional[float] = None, S=None, accumulate: bool = False, status=None, stream=None):
+    """Pass 2: context-key column max given pass 1's lse2 [B, G, ld]; returns S [B, n_c]."""
+    _need_cuda(Q, K_ctx, lse2, S, status)
+    B, G, n_in, d, n_c = _score_shapes(Q, K_ctx)
+    i_end = n_in if i_end is None else i_end
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if S is None:
+        S = torch.empty((B, n_c), dtype=torch.float32, device=Q.device)
+    ld = lse2.shape[-1]
+    _check("kvz_score_colmax", lib().kvz_score_colmax(_ptr(Q), _ptr(K_ctx), B, G, n_c, n_in, d, scale, i_begin,
+                                                      i_end, _ptr(lse2), ld, _ptr(S), int(bool(accumulate)),
+                                                      _ptr(status), _stream(stream)))
+    return S
+
+
+def kvz_select_workspace_size(B: int, n_c: int, mode: int) -> int:
+    return lib().kvz_select_workspace_size(B, n_c, mode)
+
+
+def _mode(mode) -> int:
+    if mode in ("per_head", PER_HEAD):
+        return PER_HEAD
+    if mode in ("global", GLOBAL):
+        return GLOBAL
+    raise ValueError("mode must be 'per_head' or 'global'")
+
+
+def kvz_select(S, ratio: float, mode="per_head", idx=None, counts=None, offsets=None, workspace=None,
+               status=None, stream=None):
+    """Top-ratio selection (KVzip §4.1); returns (idx int32, counts int32 [B], offsets int64 [B+1])."""
+    _need_cuda(S, idx, counts, offsets, workspace, status)
+    if S.dim() != 2 or S.dtype != torch.float32 or not S.is_contiguous():
+        raise ValueError("S must be a contiguous float32 [B, n_c] tensor")
+    m = _mode(mode)
+    B, n_c = S.shape
+    k = kvz_keep_count(B * n_c if m == GLOBAL else n_c, ratio)
+    cap = k if m == GLOBAL else B * k
+    if idx is None:
+        idx = torch.empty(max(cap, 1), dtype=torch.int32, device=S.device)
+    if counts is None:
+        counts = torch.empty(B, dtype=torch.int32, device=S.device)
+    if offsets is None:
+        offsets = torch.empty(B + 1, dtype=torch.int64, device=S.device)
+    need = kvz_select_workspace_size(B, n_c, m)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=S.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check("kvz_select", lib().kvz_select(_ptr(S), B, n_c, float(ratio), m, _ptr(idx), idx.numel(), _ptr(counts),
+                                          _ptr(offsets), _ptr(workspace), nbytes, _ptr(status), _stream(stream)))
+    return idx, counts, offsets
+
+
+def kvz_compact(K, V, idx, counts, offsets, out_offsets=None, K_out=None, V_out=None, in_place: bool = False,
+                out_rows: Optional[int] = None, status=None, stream=None):
+    """Gather kept rows in key order (KVzip §2.1 pruned cache); returns (K_out, V_out).
+
+    Out of place, the outputs are [rows, d] with head b's rows starting at
+    out_offsets[b] (default offsets[b]); ``out_rows`` sizes freshly allocated
+    outputs (default B*n_c, an upper bound).  In place, K and V themselves
+    are returned, each head's kept rows packed to the front of its region.
+    """
+    _need_cuda(K, V, idx, counts, offsets, out_offsets, K_out, V_out, status)
+    if K.dim() != 3 or K.shape != V.shape or K.dtype != torch.bfloat16 or V.dtype != torch.bfloat16:
+        raise ValueError("K and V must be bfloat16 [B, n_c, d] of equal shape")
+    B, n_c, d = K.shape
+    if in_place:
+        K_out, V_out = K, V
+    else:
+        rows = B * n_c if out_rows is None else int(out_rows)
+        if K_out is None:
+            K_out = torch.empty((rows, d), dtype=K.dtype, device=K.device)
+        if V_out is None:
+            V_out = torch.empty((rows, d), dtype=V.dtype, device=V.device)
+    _check("kvz_compact", lib().kvz_compact(_ptr(K), _ptr(V), B, n_c, d, _ptr(idx), _ptr(counts), _ptr(offsets),
+                                            _ptr(out_offsets), _ptr(K_out), _ptr(V_out), _ptr(status),
+                                            _stream(stream)))
+    return K_out, V_out

@@ -1,0 +1,264 @@
+// C ABI of libkvz: argument validation, TMA descriptor encoding and launch
+// planning for the KVzip scoring, selection and compaction kernels.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "kvz.h"
+#include "kvz_internal.h"
+
+namespace {
+
+constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1024;   // TMA coordinates are int32
+constexpr int kNumSMs = 148;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+int64_t roundup(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D view [batch][rows][d] of a bf16 tensor, read in 128-row x 64-column
+// boxes with the 128-byte swizzle the UMMA descriptors expect.  Rows past
+// `rows` read as zeros (and are masked or discarded by the kernels).
+bool make_map(CUtensorMap* m, const void* base, int64_t d, int64_t rows, int64_t batch) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(rows * d * 2)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+float log2e_scale(float scale) { return static_cast<float>(static_cast<double>(scale) * 1.4426950408889634); }
+
+kvz_status check_score_common(const void* Q, const void* K_ctx, int64_t B, int G, int64_t n_c, int64_t n_in,
+                              int d, float scale) {
+  if (Q == nullptr || K_ctx == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return KVZ_ERR_UNSUPPORTED;
+  if (B < 1 || G < 1 || n_c < 1 || n_in < 1) return KVZ_ERR_INVALID_ARG;
+  if (B * static_cast<int64_t>(G) > 0x7FFFFFFF || B > 0x7FFFFFFF) return KVZ_ERR_INVALID_ARG;
+  if (n_c > kMaxRows || n_in > kMaxRows) return KVZ_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.0f)) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(K_ctx, 16)) return KVZ_ERR_ALIGNMENT;
+  return KVZ_OK;
+}
+
+kvz_status run_lse(const void* Q, const void* K_ctx, const void* K_in, int64_t B, int G, int64_t n_c,
+                   int64_t n_in, int d, float scale, int64_t i_begin, int64_t i_end, float* lse2, int64_t ld,
+                   int32_t* status, cudaStream_t stream) {
+  CUtensorMap tmQ, tmKc, tmKi;
+  if (!make_map(&tmQ, Q, d, n_in, B * G) || !make_map(&tmKc, K_ctx, d, n_c, B) ||
+      !make_map(&tmKi, K_in, d, n_in, B))
+    return KVZ_ERR_CUDA;
+  kvz::LseArgs a{};
+  a.B = static_cast<int>(B);
+  a.G = G;
+  a.n_c = n_c;
+  a.n_in = n_in;
+  a.c2 = log2e_scale(scale);
+  a.i_begin = i_begin;
+  a.i_end = i_end;
+  a.rows_pad = roundup(i_end - i_begin, 256);
+  a.ld = ld;
+  a.lse2 = lse2;
+  a.status = status;
+  return kvz::launch_lse(d, tmQ, tmKc, tmKi, a, stream) == cudaSuccess ? KVZ_OK : KVZ_ERR_CUDA;
+}
+
+kvz_status run_colmax(const void* Q, const void* K_ctx, int64_t B, int G, int64_t n_c, int64_t n_in, int d,
+                      float scale, int64_t i_begin, int64_t i_end, const float* lse2, int64_t ld, float* S,
+                      int32_t* status, cudaStream_t stream) {
+  CUtensorMap tmQ, tmKc;
+  if (!make_map(&tmQ, Q, d, n_in, B * G) || !make_map(&tmKc, K_ctx, d, n_c, B)) return KVZ_ERR_CUDA;
+  kvz::ColArgs a{};
+  a.B = static_cast<int>(B);
+  a.G = G;
+  a.n_c = n_c;
+  a.c2 = log2e_scale(scale);
+  a.i_begin = i_begin;
+  a.rows_pad = roundup(i_end - i_begin, 256);
+  a.ld = ld;
+  a.lse2 = lse2;
+  a.S = S;
+  a.status = status;
+  a.n_kblk = static_cast<int>((n_c + 255) / 256);
+  // Split each (head, key block)'s row tiles so the grid fills ~8 waves.
+  const int64_t T = G * (a.rows_pad / 128);
+  const int64_t base_units = B * a.n_kblk;
+  int64_t nsplit = (kNumSMs * 8 + base_units - 1) / base_units;
+  const int64_t max_split = T / 4 > 1 ? T / 4 : 1;
+  if (nsplit > max_split) nsplit = max_split;
+  if (nsplit < 1) nsplit = 1;
+  const int64_t tps = (T + nsplit - 1) / nsplit;
+  nsplit = (T + tps - 1) / tps;
+  if (base_units * nsplit > 0x7FFFFFFF) return KVZ_ERR_INVALID_ARG;
+  a.nsplit = static_cast<int>(nsplit);
+  a.tiles_per_split = static_cast<int>(tps);
+  return kvz::launch_colmax(d, tmQ, tmKc, a, stream) == cudaSuccess ? KVZ_OK : KVZ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvz_version(void) { return 100; }
+
+const char* kvz_status_string(int status) {
+  switch (status) {
+    case KVZ_OK: return "KVZ_OK";
+    case KVZ_ERR_INVALID_ARG: return "KVZ_ERR_INVALID_ARG";
+    case KVZ_ERR_UNSUPPORTED: return "KVZ_ERR_UNSUPPORTED";
+    case KVZ_ERR_ALIGNMENT: return "KVZ_ERR_ALIGNMENT";
+    case KVZ_ERR_WORKSPACE: return "KVZ_ERR_WORKSPACE";
+    case KVZ_ERR_CUDA: return "KVZ_ERR_CUDA";
+    case KVZ_ERR_INVALID_SCORE: return "KVZ_ERR_INVALID_SCORE";
+    case KVZ_ERR_TIMEOUT: return "KVZ_ERR_TIMEOUT";
+    default: return "KVZ_ERR_UNKNOWN";
+  }
+}
+
+size_t kvz_score_workspace_size(int64_t B, int G, int64_t n_in, int64_t row_chunk) {
+  if (B < 1 || G < 1 || n_in < 1 || row_chunk < 0 || (row_chunk % 256) != 0) return 0;
+  const int64_t rows = row_chunk == 0 || row_chunk > n_in ? n_in : row_chunk;
+  const int64_t bytes = B * G * roundup(rows, 256) * 4;
+  return static_cast<size_t>(roundup(bytes, 256));
+}
+
+kvz_status kvz_score_lse2(const void* Q, const void* K_ctx, const void* K_in, int64_t B, int G, int64_t n_c,
+                          int64_t n_in, int d, float scale, int64_t i_begin, int64_t i_end, float* lse2,
+                          int64_t ld_lse2, int32_t* d_status, cudaStream_t stream) {
+  kvz_status st = check_score_common(Q, K_ctx, B, G, n_c, n_in, d, scale);
+  if (st != KVZ_OK) return st;
+  if (K_in == nullptr || lse2 == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(K_in, 16) || !aligned(lse2, 16) || ld_lse2 % 4 != 0) return KVZ_ERR_ALIGNMENT;
+  if (i_begin < 0 || i_begin % 256 != 0 || i_end <= i_begin || i_end > n_in) return KVZ_ERR_INVALID_ARG;
+  if (ld_lse2 < roundup(i_end - i_begin, 256)) return KVZ_ERR_INVALID_ARG;
+  return run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i_begin, i_end, lse2, ld_lse2, d_status, stream);
+}
+
+kvz_status kvz_score_colmax(const void* Q, const void* K_ctx, int64_t B, int G, int64_t n_c, int64_t n_in, int d,
+                            float scale, int64_t i_begin, int64_t i_end, const float* lse2, int64_t ld_lse2,
+                            float* S, int accumulate, int32_t* d_status, cudaStream_t stream) {
+  kvz_status st = check_score_common(Q, K_ctx, B, G, n_c, n_in, d, scale);
+  if (st != KVZ_OK) return st;
+  if (lse2 == nullptr || S == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(lse2, 16) || ld_lse2 % 4 != 0 || !aligned(S, 4)) return KVZ_ERR_ALIGNMENT;
+  if (i_begin < 0 || i_begin % 256 != 0 || i_end <= i_begin || i_end > n_in) return KVZ_ERR_INVALID_ARG;
+  if (ld_lse2 < roundup(i_end - i_begin, 256)) return KVZ_ERR_INVALID_ARG;
+  if (!accumulate && kvz::launch_fill_f32(S, B * n_c, 0.0f, stream) != cudaSuccess) return KVZ_ERR_CUDA;
+  return run_colmax(Q, K_ctx, B, G, n_c, n_in, d, scale, i_begin, i_end, lse2, ld_lse2, S, d_status, stream);
+}
+
+kvz_status kvz_score(const void* Q, const void* K_ctx, const void* K_in, int64_t B, int G, int64_t n_c,
+                     int64_t n_in, int d, float scale, int64_t row_chunk, float* S, void* workspace,
+                     size_t workspace_bytes, int32_t* d_status, cudaStream_t stream) {
+  kvz_status st = check_score_common(Q, K_ctx, B, G, n_c, n_in, d, scale);
+  if (st != KVZ_OK) return st;
+  if (K_in == nullptr || S == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(K_in, 16) || !aligned(S, 4)) return KVZ_ERR_ALIGNMENT;
+  if (row_chunk < 0 || row_chunk % 256 != 0) return KVZ_ERR_INVALID_ARG;
+  const size_t need = kvz_score_workspace_size(B, G, n_in, row_chunk);
+  if (workspace == nullptr || workspace_bytes < need) return KVZ_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return KVZ_ERR_ALIGNMENT;
+  const int64_t chunk = (row_chunk == 0 || row_chunk > n_in) ? n_in : row_chunk;
+  const int64_t ld = roundup(chunk, 256);
+  float* lse2 = static_cast<float*>(workspace);
+  if (kvz::launch_fill_f32(S, B * n_c, 0.0f, stream) != cudaSuccess) return KVZ_ERR_CUDA;
+  for (int64_t i0 = 0; i0 < n_in; i0 += chunk) {
+    const int64_t i1 = i0 + chunk < n_in ? i0 + chunk : n_in;
+    st = run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, d_status, stream);
+    if (st != KVZ_OK) return st;
+    st = run_colmax(Q, K_ctx, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, S, d_status, stream);
+    if (st != KVZ_OK) return st;
+  }
+  return KVZ_OK;
+}
+
+int64_t kvz_keep_count(int64_t n, double ratio) {
+  if (n < 0 || !(ratio >= 0.0 && ratio <= 1.0)) return -1;
+  return static_cast<int64_t>(std::floor(ratio * static_cast<double>(n)));
+}
+
+size_t kvz_select_workspace_size(int64_t B, int64_t n_c, int mode) {
+  if (B < 1 || n_c < 1 || (mode != KVZ_PER_HEAD && mode != KVZ_GLOBAL)) return 0;
+  return kvz::select_workspace(B, n_c, mode).bytes;
+}
+
+kvz_status kvz_select(const float* S, int64_t B, int64_t n_c, double ratio, int mode, int32_t* idx,
+                      int64_t idx_capacity, int32_t* counts, int64_t* offsets, void* workspace,
+                      size_t workspace_bytes, int32_t* d_status, cudaStream_t stream) {
+  if (S == nullptr || counts == nullptr || offsets == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (mode != KVZ_PER_HEAD && mode != KVZ_GLOBAL) return KVZ_ERR_INVALID_ARG;
+  if (B < 1 || B > 65535 || n_c < 1 || n_c > kMaxRows) return KVZ_ERR_INVALID_ARG;
+  if (B * n_c >= (int64_t(1) << 32)) return KVZ_ERR_INVALID_ARG;
+  if (!(ratio >= 0.0 && ratio <= 1.0)) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(S, 4) || !aligned(counts, 4) || !aligned(offsets, 8) || (idx && !aligned(idx, 4)))
+    return KVZ_ERR_ALIGNMENT;
+  const int64_t k = mode == KVZ_GLOBAL ? kvz_keep_count(B * n_c, ratio) : kvz_keep_count(n_c, ratio);
+  const int64_t need = mode == KVZ_GLOBAL ? k : B * k;
+  if (idx_capacity < need || (need > 0 && idx == nullptr)) return KVZ_ERR_INVALID_ARG;
+  const kvz::SelWorkspace lay = kvz::select_workspace(B, n_c, mode);
+  if (workspace == nullptr || workspace_bytes < lay.bytes) return KVZ_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return KVZ_ERR_ALIGNMENT;
+  return kvz::launch_select(S, B, n_c, mode, k, idx, counts, offsets, workspace, lay, d_status, stream) ==
+                 cudaSuccess
+             ? KVZ_OK
+             : KVZ_ERR_CUDA;
+}
+
+kvz_status kvz_compact(const void* K, const void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
+                       const int32_t* counts, const int64_t* offsets, const int64_t* out_offsets, void* K_out,
+                       void* V_out, int32_t* d_status, cudaStream_t stream) {
+  if (K == nullptr || V == nullptr || K_out == nullptr || V_out == nullptr || counts == nullptr ||
+      offsets == nullptr || idx == nullptr)
+    return KVZ_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return KVZ_ERR_UNSUPPORTED;
+  if (B < 1 || B > 0x7FFFFFFF || n_c < 1 || n_c > kMaxRows) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(K, 16) || !aligned(V, 16) || !aligned(K_out, 16) || !aligned(V_out, 16) || !aligned(idx, 4) ||
+      !aligned(counts, 4) || !aligned(offsets, 8) || (out_offsets && !aligned(out_offsets, 8)))
+    return KVZ_ERR_ALIGNMENT;
+  const bool k_same = K_out == K, v_same = V_out == V;
+  if (k_same != v_same) return KVZ_ERR_INVALID_ARG;          // partial in-place aliasing
+  if (K == V) return KVZ_ERR_INVALID_ARG;
+  if (k_same) {
+    if (out_offsets != nullptr) return KVZ_ERR_INVALID_ARG;
+    return kvz::launch_compact_inplace(K_out, V_out, B, n_c, d, idx, counts, offsets, d_status, stream) ==
+                   cudaSuccess
+               ? KVZ_OK
+               : KVZ_ERR_CUDA;
+  }
+  // Out of place: the outputs must not start inside either input.
+  const uintptr_t span = static_cast<uintptr_t>(B * n_c * d * 2);
+  const uintptr_t k0 = reinterpret_cast<uintptr_t>(K), v0 = reinterpret_cast<uintptr_t>(V);
+  for (const void* o : {K_out, V_out}) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(o);
+    if ((x >= k0 && x < k0 + span) || (x >= v0 && x < v0 + span)) return KVZ_ERR_INVALID_ARG;
+  }
+  return kvz::launch_compact_gather(K, V, B, n_c, d, idx, offsets, out_offsets, K_out, V_out, d_status,
+                                    stream) == cudaSuccess
+             ? KVZ_OK
+             : KVZ_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,61 @@
+// Launchers shared between the C ABI (kvz_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace kvz {
+
+// Pass 1 (row log-sum-exp) arguments.  Rows i in [i_begin, i_end) are
+// computed; rows_pad = roundup(i_end - i_begin, 256) entries per (b, g) are
+// written at lse2[(b*G + g)*ld + (i - i_begin)], padding rows set to +inf.
+struct LseArgs {
+  int B, G;
+  int64_t n_c, n_in;
+  float c2;                 // scale * log2(e)
+  int64_t i_begin, i_end, rows_pad, ld;
+  float* lse2;
+  int32_t* status;
+};
+
+// Pass 2 (context-key column max) arguments; lse2 as pass 1 wrote it.
+struct ColArgs {
+  int B, G;
+  int64_t n_c;
+  float c2;
+  int64_t i_begin, rows_pad, ld;
+  const float* lse2;
+  float* S;
+  int n_kblk;               // ceil(n_c / 256)
+  int nsplit;               // row-tile ranges per (head, key block)
+  int tiles_per_split;
+  int32_t* status;
+};
+
+cudaError_t launch_lse(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, const CUtensorMap& tmKi,
+                       const LseArgs& a, cudaStream_t stream);
+cudaError_t launch_colmax(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, const ColArgs& a,
+                          cudaStream_t stream);
+cudaError_t launch_fill_f32(float* x, int64_t n, float v, cudaStream_t stream);
+
+// Selection.  Workspace layout is computed by select_workspace().
+struct SelWorkspace {
+  size_t bytes;
+  size_t off_state, off_hist, off_cg, off_ce, off_eqb, off_cbase, off_head_eq, off_head_base;
+};
+SelWorkspace select_workspace(int64_t B, int64_t n_c, int mode);
+cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int mode, int64_t k, int32_t* idx,
+                          int32_t* counts, int64_t* offsets, void* ws, const SelWorkspace& lay,
+                          int32_t* status, cudaStream_t stream);
+
+// Compaction.
+cudaError_t launch_compact_gather(const void* K, const void* V, int64_t B, int64_t n_c, int d,
+                                  const int32_t* idx, const int64_t* offsets, const int64_t* out_offsets,
+                                  void* K_out, void* V_out, int32_t* status, cudaStream_t stream);
+cudaError_t launch_compact_inplace(void* K, void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
+                                   const int32_t* counts, const int64_t* offsets, int32_t* status,
+                                   cudaStream_t stream);
+
+}  // namespace kvz

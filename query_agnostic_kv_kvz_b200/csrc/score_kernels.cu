@@ -1,0 +1,536 @@
+// KVzip context-reconstruction scoring on sm_100a (tcgen05 + TMEM + TMA).
+//
+// KVzip (analysis report, §3.2 "KV importance scoring", equation for S_{l,h}):
+//   A = Softmax(Q K^T) over the n_c + n_in keys of the repeat-prompt + context
+//   input, sliced to the n_c context keys; S[j] = max_{g,i} A[g,i,j].
+// With c2 = scale * log2(e) and lse2_r = log2 sum_{u visible} 2^(c2 <q_r,k_u>):
+//   A[r, j] = 2^(c2 <q_r, k_j> - lse2_r)  and, exp2 being monotone,
+//   S[j]    = 2^( max_r (c2 <q_r, k_j> - lse2_r) ).
+// Two passes, neither materialising the G*n_in x (n_c+n_in) matrix:
+//   pass 1 (lse_kernel):    one thread per query row, online max / sum over
+//                           key tiles (FlashAttention-style, no P.V);
+//   pass 2 (colmax_kernel): keys in TMEM lanes, one thread per context key,
+//                           running max over query-row columns; no mask
+//                           because every row sees every context key.
+// Both kernels: warp 0 issues TMA loads, warp 1 (one thread) issues
+// tcgen05.mma into tensor memory, warp 2 owns the TMEM allocation, warps
+// 4..11 (two warpgroups) read TMEM and do the softmax / max arithmetic.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "kvz_internal.h"
+#include "kvz_sm100.cuh"
+
+namespace kvz {
+
+namespace {
+
+constexpr int kThreads = 384;     // 12 warps
+constexpr int kTile = 128;        // rows of a Q sub-tile / keys of a K tile
+constexpr int kSubBytes64 = kTile * 128;  // one 128-row x 64-column bf16 block (16 KB)
+constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128);
+
+template <int D>
+struct LseLayout {
+  static constexpr int KB = D / 64;                      // 64-column blocks per row
+  static constexpr int TILE_BYTES = KB * kSubBytes64;    // 128 rows x D
+  static constexpr int NQ = 2;                           // Q sub-tiles per CTA
+  static constexpr int KST = 4;                          // K-tile pipeline depth
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + NQ * TILE_BYTES;
+  static constexpr int BAR_OFF = K_OFF + KST * TILE_BYTES;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;  // + alignment slack
+};
+
+template <int D>
+struct ColLayout {
+  static constexpr int KB = D / 64;
+  static constexpr int TILE_BYTES = KB * kSubBytes64;
+  static constexpr int NA = 2;                           // key tiles per CTA (256 keys)
+  static constexpr int QST = 4;                          // Q-tile pipeline depth
+  static constexpr int A_OFF = 0;
+  static constexpr int Q_OFF = A_OFF + NA * TILE_BYTES;
+  static constexpr int L_OFF = Q_OFF + QST * TILE_BYTES;  // lse2 slices, 128 floats each
+  static constexpr int BAR_OFF = L_OFF + QST * kTile * 4;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Descriptor of k-step `k` (16 bf16 of K) of a 128-row tile at `tile`.
+__device__ __forceinline__ uint64_t kstep_desc(const uint8_t* tile, int k) {
+  return sdesc_kmajor_sw128(smem_u32(tile + (k >> 2) * kSubBytes64 + (k & 3) * 32));
+}
+
+// ============================================================================
+// Pass 1: lse2 of every input row in [i_begin, i_end).
+// CTA = (head b, group g, 256 input rows = two 128-row sub-tiles).  Blocks
+// are numbered longest-first (rows late in the input see more keys).
+// ============================================================================
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    lse_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
+               const __grid_constant__ CUtensorMap tmKi, LseArgs p) {
+  using Lay = LseLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sQ = smem + Lay::Q_OFF;
+  uint8_t* sK = smem + Lay::K_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;                  // [KST]
+  uint64_t* k_empty = k_full + Lay::KST;        // [KST]
+  uint64_t* s_full = k_empty + Lay::KST;        // [2 sub-tiles][2 buffers]
+  uint64_t* s_empty = s_full + 4;               // [2][2]
+  uint64_t* drain = s_empty + 4;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit (longest first) ----
+  const int nblk = static_cast<int>(p.rows_pad / 256);
+  const int BG = p.B * p.G;
+  const int u = blockIdx.x;
+  const int iblk = nblk - 1 - u / BG;
+  const int bg = u % BG;
+  const int b = bg / p.G;
+  const int64_t i0 = p.i_begin + static_cast<int64_t>(iblk) * 256;
+  const int64_t row_hi = p.i_end;               // rows >= row_hi are padding
+  const int nq_valid = (i0 + kTile < row_hi) ? 2 : 1;
+  const int NC = static_cast<int>((p.n_c + kTile - 1) / kTile);
+  int nin[2];
+  nin[0] = static_cast<int>(i0 / kTile) + 1;
+  nin[1] = static_cast<int>((i0 + kTile) / kTile) + 1;
+  const int NT = NC + nin[nq_valid - 1];
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < Lay::KST; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  int issued = 0;   // K tiles whose TMA loads were issued (producer thread)
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmKc);
+      prefetch_tmap(&tmKi);
+      mbar_arrive_expect_tx(q_full, nq_valid * Lay::TILE_BYTES);
+      for (int q = 0; q < nq_valid; ++q)
+        for (int kb = 0; kb < Lay::KB; ++kb)
+          tma_load_3d(sQ + q * Lay::TILE_BYTES + kb * kSubBytes64, &tmQ, q_full, kb * 64,
+                      static_cast<int>(i0 + q * kTile), bg);
+      for (int t = 0; t < NT; ++t) {
+        const int s = t % Lay::KST;
+        const uint32_t use = static_cast<uint32_t>(t / Lay::KST);
+        if (!mbar_wait(&k_empty[s], (use & 1u) ^ 1u, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&k_full[s], Lay::TILE_BYTES);
+        const bool ctx = t < NC;
+        const CUtensorMap* m = ctx ? &tmKc : &tmKi;
+        const int row = ctx ? t * kTile : (t - NC) * kTile;
+        for (int kb = 0; kb < Lay::KB; ++kb)
+          tma_load_3d(sK + s * Lay::TILE_BYTES + kb * kSubBytes64, m, &k_full[s], kb * 64, row, b);
+        issued = t + 1;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t cnt[2] = {0u, 0u};
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+      tc_fence_after();
+      for (int t = 0; ok && t < NT; ++t) {
+        const int s = t % Lay::KST;
+        const uint32_t use = static_cast<uint32_t>(t / Lay::KST);
+        if (!mbar_wait(&k_full[s], use & 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        for (int q = 0; q < nq_valid; ++q) {
+          if (t >= NC && t - NC >= nin[q]) continue;
+          const uint32_t buf = cnt[q] & 1u;
+          const uint32_t bu = cnt[q] >> 1;
+          if (!mbar_wait(&s_empty[q * 2 + buf], (bu & 1u) ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + static_cast<uint32_t>((q * 2 + buf) * kTile);
+          const uint8_t* a_tile = sQ + q * Lay::TILE_BYTES;
+          const uint8_t* b_tile = sK + s * Lay::TILE_BYTES;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k)
+            tc_mma_bf16(d_tmem, kstep_desc(a_tile, k), kstep_desc(b_tile, k), kIdesc, k > 0 ? 1u : 0u);
+          tc_commit(&s_full[q * 2 + buf]);
+          ++cnt[q];
+        }
+        tc_commit(&k_empty[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------ softmax warpgroups
+    const int q = (warp - 4) >> 2;
+    const int wq = warp & 3;
+    const int rl = wq * 32 + lane;                  // row within the sub-tile == TMEM lane
+    const int64_t i = i0 + q * kTile + rl;
+    const float c2 = p.c2;
+    float m = -INFINITY, l = 0.0f;
+    bool ok = true;
+    if (q < nq_valid) {
+      const int ctx_tail = static_cast<int>(p.n_c - static_cast<int64_t>(NC - 1) * kTile);
+      uint32_t cnt = 0;
+      for (int t = 0; t < NT; ++t) {
+        if (t >= NC && t - NC >= nin[q]) continue;
+        const uint32_t buf = cnt & 1u;
+        const uint32_t bu = cnt >> 1;
+        if (!mbar_wait_warp(&s_full[q * 2 + buf], bu & 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float v[128];
+        tmem_ld128(tmem + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>((q * 2 + buf) * kTile), v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[q * 2 + buf]);
+        if (t == NC - 1 && ctx_tail < kTile) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= ctx_tail) v[c] = -INFINITY;
+        }
+        if (t >= NC && t - NC == nin[q] - 1) {       // diagonal input tile
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > rl) v[c] = -INFINITY;
+        }
+        float mx0 = v[0], mx1 = v[1], mx2 = v[2], mx3 = v[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+          mx0 = fmaxf(mx0, v[c]);
+          mx1 = fmaxf(mx1, v[c + 1]);
+          mx2 = fmaxf(mx2, v[c + 2]);
+          mx3 = fmaxf(mx3, v[c + 3]);
+        }
+        const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c2;
+        // Move the reference max only when it grows by more than 2^8; the
+        // sum is exact for any reference, and values stay below 2^8.
+        if (mt > m + 8.0f) {
+          l *= ex2_approx(m - mt);
+          m = mt;
+        }
+        const float nm = -m;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          a0 += ex2_approx(fmaf(v[c], c2, nm));
+          a1 += ex2_approx(fmaf(v[c + 1], c2, nm));
+          a2 += ex2_approx(fmaf(v[c + 2], c2, nm));
+          a3 += ex2_approx(fmaf(v[c + 3], c2, nm));
+        }
+        l += (a0 + a1) + (a2 + a3);
+        ++cnt;
+      }
+    }
+    const float lse2 = (q < nq_valid && ok && i < row_hi) ? m + log2f(l) : INFINITY;
+    p.lse2[static_cast<int64_t>(bg) * p.ld + (i - p.i_begin)] = lse2;
+  }
+
+  __syncthreads();
+  if (*abort_flag) {
+    // Unwinding after a timeout: let this CTA's own copies and MMAs finish
+    // (bounded) before shared and tensor memory are released.
+    if (warp == 0 && lane == 0) {
+      mbar_wait_for(q_full, 0, 20000000ull);
+      for (int s = 0; s < Lay::KST && s < issued; ++s) {
+        const int t_last = s + Lay::KST * ((issued - 1 - s) / Lay::KST);
+        mbar_wait_for(&k_full[s], static_cast<uint32_t>(t_last / Lay::KST) & 1u, 20000000ull);
+      }
+    }
+    if (warp == 1 && lane == 0) {
+      tc_commit(drain);
+      mbar_wait_for(drain, 0, 20000000ull);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ============================================================================
+// Pass 2: S[b, j] = max(S[b, j], 2^(max_r c2 <q_r, k_j> - lse2_r)).
+// CTA = (head b, 256 context keys, a contiguous range of 128-row Q tiles).
+// Keys are the MMA's M side, so TMEM lane = key and each thread keeps the
+// running max of its key over the query-row columns in a register.
+// ============================================================================
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    colmax_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
+                  ColArgs p) {
+  using Lay = ColLayout<D>;
+  const int u = blockIdx.x;
+  const int kblk = u % p.n_kblk;
+  const int rest = u / p.n_kblk;
+  const int sp = rest % p.nsplit;
+  const int b = rest / p.nsplit;
+  const int tpg = static_cast<int>(p.rows_pad / kTile);   // row tiles per group
+  const int T = p.G * tpg;
+  const int t_begin = sp * p.tiles_per_split;
+  const int t_end = min(T, t_begin + p.tiles_per_split);
+  const int ntile = t_end - t_begin;
+  if (ntile <= 0) return;                                  // uniform for the CTA
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem + Lay::A_OFF;
+  uint8_t* sQ = smem + Lay::Q_OFF;
+  float* sL = reinterpret_cast<float*>(smem + Lay::L_OFF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
+  uint64_t* a_full = bars + 0;
+  uint64_t* q_full = bars + 1;                   // [QST]
+  uint64_t* q_empty = q_full + Lay::QST;         // [QST]
+  uint64_t* acc_full = q_empty + Lay::QST;       // [2 key tiles][2 buffers]
+  uint64_t* acc_empty = acc_full + 4;            // [2][2]
+  uint64_t* drain = acc_empty + 4;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t key0 = static_cast<int64_t>(kblk) * 256;
+
+  if (threadIdx.x == 0) {
+    mbar_init(a_full, 1);
+    for (int s = 0; s < Lay::QST; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1 + 8);            // MMA commit + 8 epilogue warps
+    }
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  int issued = 0;   // Q tiles whose loads were issued (producer thread)
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmKc);
+      mbar_arrive_expect_tx(a_full, Lay::NA * Lay::TILE_BYTES);
+      for (int a = 0; a < Lay::NA; ++a)
+        for (int kb = 0; kb < Lay::KB; ++kb)
+          tma_load_3d(sA + a * Lay::TILE_BYTES + kb * kSubBytes64, &tmKc, a_full, kb * 64,
+                      static_cast<int>(key0 + a * kTile), b);
+      for (int n = 0; n < ntile; ++n) {
+        const int s = n % Lay::QST;
+        const uint32_t use = static_cast<uint32_t>(n / Lay::QST);
+        if (!mbar_wait(&q_empty[s], (use & 1u) ^ 1u, abort_flag, p.status)) break;
+        const int tau = t_begin + n;
+        const int g = tau / tpg;
+        const int il = (tau % tpg) * kTile;
+        const int bgq = b * p.G + g;
+        mbar_arrive_expect_tx(&q_full[s], Lay::TILE_BYTES + kTile * 4);
+        for (int kb = 0; kb < Lay::KB; ++kb)
+          tma_load_3d(sQ + s * Lay::TILE_BYTES + kb * kSubBytes64, &tmQ, &q_full[s], kb * 64,
+                      static_cast<int>(p.i_begin + il), bgq);
+        bulk_load(sL + s * kTile, p.lse2 + static_cast<int64_t>(bgq) * p.ld + il, kTile * 4, &q_full[s]);
+        issued = n + 1;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = mbar_wait(a_full, 0, abort_flag, p.status);
+      tc_fence_after();
+      for (int n = 0; ok && n < ntile; ++n) {
+        const int s = n % Lay::QST;
+        const uint32_t use = static_cast<uint32_t>(n / Lay::QST);
+        if (!mbar_wait(&q_full[s], use & 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t buf = static_cast<uint32_t>(n) & 1u;
+        const uint32_t bu = static_cast<uint32_t>(n) >> 1;
+        for (int a = 0; a < Lay::NA; ++a) {
+          if (!mbar_wait(&acc_empty[a * 2 + buf], (bu & 1u) ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + static_cast<uint32_t>((a * 2 + buf) * kTile);
+          const uint8_t* a_tile = sA + a * Lay::TILE_BYTES;
+          const uint8_t* b_tile = sQ + s * Lay::TILE_BYTES;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k)
+            tc_mma_bf16(d_tmem, kstep_desc(a_tile, k), kstep_desc(b_tile, k), kIdesc, k > 0 ? 1u : 0u);
+          tc_commit(&acc_full[a * 2 + buf]);
+        }
+        if (!ok) break;
+        tc_commit(&q_empty[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    const int a = (warp - 4) >> 2;
+    const int wq = warp & 3;
+    const int64_t j = key0 + a * kTile + wq * 32 + lane;   // context key == TMEM lane
+    const float c2 = p.c2;
+    float mx = -INFINITY;
+    bool ok = true;
+    for (int n = 0; n < ntile; ++n) {
+      const int s = n % Lay::QST;
+      const uint32_t use = static_cast<uint32_t>(n / Lay::QST);
+      const uint32_t buf = static_cast<uint32_t>(n) & 1u;
+      const uint32_t bu = static_cast<uint32_t>(n) >> 1;
+      if (!mbar_wait_warp(&acc_full[a * 2 + buf], bu & 1u, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float v[128];
+      tmem_ld128(tmem + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>((a * 2 + buf) * kTile), v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[a * 2 + buf]);
+      // the lse2 slice arrived with the Q tile on q_full[s]
+      if (!mbar_wait_warp(&q_full[s], use & 1u, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      const float4* L = reinterpret_cast<const float4*>(sL + s * kTile);
+      float m0 = mx, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float4 l4 = L[c];
+        m0 = fmaxf(m0, fmaf(v[4 * c + 0], c2, -l4.x));
+        m1 = fmaxf(m1, fmaf(v[4 * c + 1], c2, -l4.y));
+        m2 = fmaxf(m2, fmaf(v[4 * c + 2], c2, -l4.z));
+        m3 = fmaxf(m3, fmaf(v[4 * c + 3], c2, -l4.w));
+      }
+      mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_empty[s]);
+    }
+    if (ok && j < p.n_c) {
+      const float sj = exp2f(mx);   // >= +0, so its bit pattern orders like the value
+      atomicMax(reinterpret_cast<unsigned int*>(p.S + static_cast<int64_t>(b) * p.n_c + j), __float_as_uint(sj));
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 0 && lane == 0) {
+      mbar_wait_for(a_full, 0, 20000000ull);
+      for (int s = 0; s < Lay::QST && s < issued; ++s) {
+        const int n_last = s + Lay::QST * ((issued - 1 - s) / Lay::QST);
+        mbar_wait_for(&q_full[s], static_cast<uint32_t>(n_last / Lay::QST) & 1u, 20000000ull);
+      }
+    }
+    if (warp == 1 && lane == 0) {
+      tc_commit(drain);
+      mbar_wait_for(drain, 0, 20000000ull);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+__global__ void fill_f32_kernel(float* x, int64_t n, float v) {
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    x[e] = v;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace
+
+cudaError_t launch_lse(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, const CUtensorMap& tmKi,
+                       const LseArgs& a, cudaStream_t stream) {
+  const int64_t nblk = a.rows_pad / 256;
+  const int64_t grid = static_cast<int64_t>(a.B) * a.G * nblk;
+  if (grid <= 0 || grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  cudaError_t e;
+  if (d == 128) {
+    e = set_smem(lse_kernel<128>, LseLayout<128>::SMEM);
+    if (e != cudaSuccess) return e;
+    lse_kernel<128><<<static_cast<unsigned>(grid), kThreads, LseLayout<128>::SMEM, stream>>>(tmQ, tmKc, tmKi, a);
+  } else {
+    e = set_smem(lse_kernel<64>, LseLayout<64>::SMEM);
+    if (e != cudaSuccess) return e;
+    lse_kernel<64><<<static_cast<unsigned>(grid), kThreads, LseLayout<64>::SMEM, stream>>>(tmQ, tmKc, tmKi, a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_colmax(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, const ColArgs& a,
+                          cudaStream_t stream) {
+  const int64_t grid = static_cast<int64_t>(a.B) * a.nsplit * a.n_kblk;
+  if (grid <= 0 || grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  cudaError_t e;
+  if (d == 128) {
+    e = set_smem(colmax_kernel<128>, ColLayout<128>::SMEM);
+    if (e != cudaSuccess) return e;
+    colmax_kernel<128><<<static_cast<unsigned>(grid), kThreads, ColLayout<128>::SMEM, stream>>>(tmQ, tmKc, a);
+  } else {
+    e = set_smem(colmax_kernel<64>, ColLayout<64>::SMEM);
+    if (e != cudaSuccess) return e;
+    colmax_kernel<64><<<static_cast<unsigned>(grid), kThreads, ColLayout<64>::SMEM, stream>>>(tmQ, tmKc, a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_f32(float* x, int64_t n, float v, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  fill_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, n, v);
+  return cudaGetLastError();
+}
+
+}  // namespace kvz

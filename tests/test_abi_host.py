@@ -1,0 +1,93 @@
+"""Host-side checks of the C ABI (no GPU): the library builds, loads, exports
+every function include/kvz.h declares, and its host-only helpers agree with
+the definitions (keep count, workspace sizing, status strings)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from oracle import kvz_oracle as orc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvz.h")
+
+
+@pytest.fixture(scope="module")
+def kvz():
+    from query_agnostic_kv_kvz_b200 import build
+    build.build()
+    import query_agnostic_kv_kvz_b200 as k
+    k.lib()
+    return k
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvz_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("kvz_score", "kvz_select", "kvz_compact"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(kvz):
+    handle = ctypes.CDLL(kvz.lib_path)
+    missing = [n for n in declared_functions() if not hasattr(handle, n)]
+    assert not missing, missing
+
+
+def test_version_and_status_strings(kvz):
+    assert kvz.kvz_version() >= 100
+    lib = kvz.lib()
+    for code, name in kvz.STATUS.items():
+        assert lib.kvz_status_string(code).decode() == name
+    assert lib.kvz_status_string(99).decode() == "KVZ_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("n,ratio", [(256, 0.3), (8192, 0.3), (8388608, 0.3), (131072, 0.25),
+                                     (43520000, 0.1), (10, 0.7), (3, 0.1), (7, 0.0), (7, 1.0)])
+def test_keep_count_matches_oracle(kvz, n, ratio):
+    assert kvz.kvz_keep_count(n, ratio) == orc.keep_count(n, ratio)
+
+
+def test_keep_count_rejects_bad_ratio(kvz):
+    assert kvz.kvz_keep_count(10, 1.5) == -1
+    assert kvz.kvz_keep_count(10, float("nan")) == -1
+
+
+def test_score_workspace_size(kvz):
+    # one chunk of rows, padded to 256, fp32, times B*G
+    assert kvz.kvz_score_workspace_size(8, 4, 8224, 0) == 8 * 4 * 8448 * 4
+    assert kvz.kvz_score_workspace_size(384, 5, 131104, 4096) == 384 * 5 * 4096 * 4
+    assert kvz.kvz_score_workspace_size(1, 1, 1, 0) == 256 * 4
+    assert kvz.kvz_score_workspace_size(1, 1, 10, 100) == 0      # chunk not a multiple of 256
+    assert kvz.kvz_score_workspace_size(0, 1, 10, 0) == 0
+
+
+def test_select_workspace_size(kvz):
+    a = kvz.kvz_select_workspace_size(8, 8192, kvz.PER_HEAD)
+    b = kvz.kvz_select_workspace_size(8, 8192, kvz.GLOBAL)
+    assert a > b > 0                      # per-head keeps one histogram per head
+    assert kvz.kvz_select_workspace_size(8, 8192, 7) == 0
+
+
+def test_binding_rejects_host_tensors(kvz):
+    Q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
+    K = torch.zeros(1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        kvz.kvz_score(Q, K, K)
+
+
+def test_product_code_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "query_agnostic_kv_kvz_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", text, flags=re.M), f
+                assert "oracle/" not in text and "kvz_oracle" not in text, f

@@ -1,0 +1,237 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded bf16 inputs.
+
+Scores: |dS| <= 1e-4 everywhere and |dS|/S <= 1e-2 where S > 1e-3.
+Selection and compaction: bit-exact.  Selection is compared on identical
+fp32 scores (the oracle's stable sort run on the scores the GPU selects
+from), because a top-k over floating-point scores is discontinuous.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from kvz_testutil import assert_scores_close, bits, f32_scale, f64, oracle_scores
+from oracle import kvz_oracle as orc
+from query_agnostic_kv_kvz_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+kvz = pytest.importorskip("query_agnostic_kv_kvz_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    kvz.lib()
+
+
+def _inputs(B, G, n_c, n_prompt, d, seed=0, name="llama8b_layer"):
+    return synth.layer_inputs(synth.WORKLOADS[name], seed=seed, device="cuda", heads=B, G=G, n_c=n_c,
+                              n_prompt=n_prompt, d=d)
+
+
+# ---------------------------------------------------------------------------
+# Scoring
+# ---------------------------------------------------------------------------
+SMALL_SHAPES = [
+    # B, G, n_c, n_prompt, d, row_chunk
+    (1, 4, 256, 16, 64, 0),        # the tiny reference workload's shape
+    (1, 1, 1, 0, 128, 0),          # one context key, one input row
+    (2, 3, 127, 5, 128, 0),        # ragged: n_c < tile, n_in not a multiple of 128
+    (3, 2, 129, 40, 64, 0),        # ragged: one key past a tile
+    (2, 5, 1000, 32, 128, 256),    # G=5 and row chunks of 256 positions
+    (1, 1, 300, 0, 128, 0),
+    (2, 4, 513, 300, 128, 512),    # chunk larger than a tile, prompt longer than a tile
+    (1, 2, 2048, 32, 64, 0),
+]
+
+
+@pytest.mark.parametrize("B,G,n_c,n_prompt,d,row_chunk", SMALL_SHAPES)
+def test_score_matches_oracle_small(B, G, n_c, n_prompt, d, row_chunk):
+    x = _inputs(B, G, n_c, n_prompt, d, seed=B * 1000 + n_c)
+    scale = f32_scale(d)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S = kvz.kvz_score(x["Q"], x["K_ctx"], x["K_in"], scale=scale, row_chunk=row_chunk, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref = oracle_scores(x["Q"], x["K_ctx"], x["K_in"], scale)
+    assert_scores_close(S.cpu().numpy(), ref, "score B=%d G=%d n_c=%d" % (B, G, n_c))
+
+
+@pytest.mark.parametrize("B,G,n_c,n_prompt,d", [(1, 4, 256, 16, 64), (2, 3, 300, 70, 128), (1, 2, 129, 0, 128)])
+def test_lse2_matches_oracle_rows(B, G, n_c, n_prompt, d):
+    x = _inputs(B, G, n_c, n_prompt, d, seed=7)
+    n_in = n_c + n_prompt
+    scale = f32_scale(d)
+    lse2 = kvz.kvz_score_lse2(x["Q"], x["K_ctx"], x["K_in"], scale=scale).cpu().numpy()
+    ld = lse2.shape[-1]
+    assert ld == (n_in + 255) // 256 * 256
+    Q, Kc, Ki = f64(x["Q"]), f64(x["K_ctx"]), f64(x["K_in"])
+    for b in range(B):
+        for g in range(G):
+            want = np.array([orc.row_lse(Q[b, g, i], Kc[b], Ki[b], i, scale) for i in range(n_in)]) / math.log(2)
+            np.testing.assert_allclose(lse2[b, g, :n_in], want, rtol=0, atol=2e-4)
+            assert np.all(np.isinf(lse2[b, g, n_in:])) and np.all(lse2[b, g, n_in:] > 0)
+
+
+def test_row_chunks_merge_exactly():
+    x = _inputs(2, 4, 777, 600, 128, seed=3)
+    S0 = kvz.kvz_score(x["Q"], x["K_ctx"], x["K_in"], row_chunk=0)
+    S1 = kvz.kvz_score(x["Q"], x["K_ctx"], x["K_in"], row_chunk=256)
+    S2 = kvz.kvz_score(x["Q"], x["K_ctx"], x["K_in"], row_chunk=512)
+    # each row's lse is computed by the same thread in the same order whatever
+    # the chunking, and max is exact, so the results are bit-identical
+    assert torch.equal(S0, S1) and torch.equal(S0, S2)
+
+
+def test_identical_keys_closed_form():
+    # every causal row is uniform over its visible keys: S[j] = 1/(n_c+1)
+    B, G, n_c, n_prompt, d = 2, 4, 1000, 32, 128
+    x = _inputs(B, G, n_c, n_prompt, d, seed=11)
+    v = x["K_ctx"][:, :1, :]
+    Kc = v.expand(B, n_c, d).contiguous()
+    Ki = v.expand(B, n_c + n_prompt, d).contiguous()
+    S = kvz.kvz_score(x["Q"], Kc, Ki).cpu().double().numpy()
+    assert np.abs(S - 1.0 / (n_c + 1)).max() <= 1e-4 / (n_c + 1) + 1e-9
+
+
+def test_score_is_deterministic():
+    x = _inputs(3, 4, 2000, 32, 128, seed=5)
+    S0 = kvz.kvz_score(x["Q"], x["K_ctx"], x["K_in"])
+    S1 = kvz.kvz_score(x["Q"], x["K_ctx"], x["K_in"])
+    assert torch.equal(S0, S1)
+
+
+def test_llama8b_layer_full_matches_oracle():
+    """The 8-head, 8192-key Llama-3.1-8B-shaped layer, every score checked."""
+    w = synth.WORKLOADS["llama8b_layer"]
+    x = synth.layer_inputs(w, device="cuda")
+    scale = f32_scale(w.d)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S = kvz.kvz_score(x["Q"], x["K_ctx"], x["K_in"], scale=scale, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref = oracle_scores(x["Q"], x["K_ctx"], x["K_in"], scale)
+    assert_scores_close(S.cpu().numpy(), ref, "llama8b_layer")
+
+
+# ---------------------------------------------------------------------------
+# Selection (bit-exact on identical fp32 scores)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,n_c", [(1, 1), (1, 100), (3, 4097), (8, 8192), (5, 12345), (2, 70000)])
+@pytest.mark.parametrize("ratio", [0.0, 0.1, 0.3, 0.5, 1.0])
+@pytest.mark.parametrize("mode", ["per_head", "global"])
+def test_select_matches_oracle(B, n_c, ratio, mode):
+    S = synth.synthetic_scores(B, n_c, seed=B * 7 + n_c, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx, counts, offsets = kvz.kvz_select(S, ratio, mode, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ri, rc, ro = orc.select(S.cpu().numpy(), ratio, mode)
+    np.testing.assert_array_equal(counts.cpu().numpy(), rc)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), ro)
+    np.testing.assert_array_equal(idx.cpu().numpy()[: len(ri)], ri)
+
+
+def test_select_all_ties_takes_lowest_indices():
+    S = torch.full((4, 5000), 0.25, device="cuda")
+    idx, counts, offsets = kvz.kvz_select(S, 0.3, "global")
+    k = orc.keep_count(20000, 0.3)
+    assert counts.cpu().tolist() == [5000, 1000, 0, 0]
+    np.testing.assert_array_equal(idx.cpu().numpy()[:k], np.r_[np.arange(5000), np.arange(1000)])
+
+
+def test_select_reports_invalid_scores():
+    S = synth.synthetic_scores(2, 1000, seed=1, device="cuda")
+    S[1, 17] = float("nan")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvz.kvz_select(S, 0.3, "global", status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 6          # KVZ_ERR_INVALID_SCORE
+    S[1, 17] = -1.0
+    status.zero_()
+    kvz.kvz_select(S, 0.3, "per_head", status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 6
+
+
+# ---------------------------------------------------------------------------
+# Compaction (bit-exact)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,n_c,d,ratio,mode", [(1, 1, 128, 1.0, "per_head"), (3, 1000, 128, 0.3, "per_head"),
+                                                (4, 4097, 64, 0.25, "global"), (8, 8192, 128, 0.3, "per_head"),
+                                                (2, 70000, 128, 0.1, "global"), (5, 333, 64, 0.0, "global")])
+def test_compact_out_of_place_matches_oracle(B, n_c, d, ratio, mode):
+    g = torch.Generator(device="cuda").manual_seed(n_c)
+    K = torch.randn((B, n_c, d), generator=g, device="cuda").to(torch.bfloat16)
+    V = torch.randn((B, n_c, d), generator=g, device="cuda").to(torch.bfloat16)
+    S = synth.synthetic_scores(B, n_c, seed=n_c, device="cuda")
+    idx, counts, offsets = kvz.kvz_select(S, ratio, mode)
+    total = int(offsets[-1].item())
+    K_out, V_out = kvz.kvz_compact(K, V, idx, counts, offsets, out_rows=max(total, 1))
+    torch.cuda.synchronize()
+    rk, rv = orc.compact(bits(K), bits(V), idx.cpu().numpy(), counts.cpu().numpy(), offsets.cpu().numpy())
+    np.testing.assert_array_equal(bits(K_out)[:total], rk)
+    np.testing.assert_array_equal(bits(V_out)[:total], rv)
+
+
+@pytest.mark.parametrize("B,n_c,d,ratio,mode", [(3, 1000, 128, 0.3, "per_head"), (4, 4097, 64, 0.25, "global"),
+                                                (2, 70000, 128, 0.9, "global"), (2, 5000, 128, 1.0, "per_head")])
+def test_compact_in_place_matches_oracle(B, n_c, d, ratio, mode):
+    g = torch.Generator(device="cuda").manual_seed(n_c + 1)
+    K = torch.randn((B, n_c, d), generator=g, device="cuda").to(torch.bfloat16)
+    V = torch.randn((B, n_c, d), generator=g, device="cuda").to(torch.bfloat16)
+    S = synth.synthetic_scores(B, n_c, seed=n_c + 1, device="cuda")
+    idx, counts, offsets = kvz.kvz_select(S, ratio, mode)
+    Kh, Vh = bits(K), bits(V)
+    ic, cc, oc = idx.cpu().numpy(), counts.cpu().numpy(), offsets.cpu().numpy()
+    # canary: every dropped row becomes a sentinel that must never reach the kept prefix
+    for b in range(B):
+        keep = np.zeros(n_c, bool)
+        keep[ic[oc[b]:oc[b + 1]]] = True
+        drop = torch.from_numpy(np.nonzero(~keep)[0]).cuda()
+        K.view(torch.int16)[b, drop] = 0x7FC1
+        V.view(torch.int16)[b, drop] = 0x7FC1
+    Kh, Vh = bits(K), bits(V)
+    rk, rv = orc.compact(Kh, Vh, ic, cc, oc)
+    K2, V2 = kvz.kvz_compact(K, V, idx, counts, offsets, in_place=True)
+    torch.cuda.synchronize()
+    assert K2.data_ptr() == K.data_ptr()
+    Ko, Vo = bits(K), bits(V)
+    for b in range(B):
+        c = int(cc[b])
+        np.testing.assert_array_equal(Ko[b, :c], rk[oc[b]:oc[b] + c])
+        np.testing.assert_array_equal(Vo[b, :c], rv[oc[b]:oc[b] + c])
+        np.testing.assert_array_equal(Ko[b, c:], Kh[b, c:])      # rows past the count are untouched
+        assert not np.any(Ko[b, :c] == 0x7FC1)
+
+
+# ---------------------------------------------------------------------------
+# The whole path on the two small workloads
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["tiny", "llama8b_layer"])
+def test_pipeline_selection_and_compaction_exact(name):
+    w = synth.WORKLOADS[name]
+    x = synth.layer_inputs(w, device="cuda")
+    scale = f32_scale(w.d)
+    S = kvz.kvz_score(x["Q"], x["K_ctx"], x["K_in"], scale=scale)
+    idx, counts, offsets = kvz.kvz_select(S, w.ratio, w.mode)
+    total = int(offsets[-1].item())
+    K_out, V_out = kvz.kvz_compact(x["K_ctx"], x["V"], idx, counts, offsets, out_rows=total)
+    torch.cuda.synchronize()
+    S_np = S.cpu().numpy()
+    ri, rc, ro = orc.select(S_np, w.ratio, w.mode)
+    np.testing.assert_array_equal(idx.cpu().numpy()[:total], ri)
+    np.testing.assert_array_equal(counts.cpu().numpy(), rc)
+    rk, rv = orc.compact(bits(x["K_ctx"]), bits(x["V"]), ri, rc, ro)
+    np.testing.assert_array_equal(bits(K_out), rk)
+    np.testing.assert_array_equal(bits(V_out), rv)
+    if name == "tiny":
+        # overlap with the selection made from the oracle's own fp64 scores
+        ref_S = oracle_scores(x["Q"], x["K_ctx"], x["K_in"], scale).astype(np.float32)
+        oi, _, _ = orc.select(ref_S, w.ratio, w.mode)
+        overlap = len(set(oi.tolist()) & set(ri.tolist())) / max(1, len(set(oi.tolist()) | set(ri.tolist())))
+        assert overlap > 0.9
