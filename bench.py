@@ -1,0 +1,395 @@
+"""Benchmark of the KVzip compression hot path on B200.
+
+One step = score (pass 1 row log-sum-exp + pass 2 context-key column max)
+-> select (top ratio per head) -> compact (gather of the kept K/V rows) over
+one Llama-3.1-8B-shaped layer: 8 KV heads, G=4, d=128, n_c=8192 context keys,
+32-token repeat prompt, keep ratio 0.3 per head, bf16, seeded synthetic
+inputs resident in HBM.  The metric is context KV pairs scored and evicted
+per second (B*n_c per step).  L2 is flushed before every timed step (the
+inputs, ~117 MB, would otherwise stay in the 126 MB L2).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own
+independent layer (different seed): weak scaling, no data-path collective.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "context KV pairs scored+evicted/sec at 1 B200; score TFLOP/s % of bf16 peak"
+UNIT = "context KV pairs/s"
+WORKLOAD = "llama8b_layer"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvz", choices=["kvz", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        d = dict(FALLBACK_PEAKS)
+        d["source"] = "fallback"
+        return d
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's
+    source has not changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+        src = os.path.join(ROOT, rec["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if h != rec["source_sha256_16"]:
+            return None
+        return float(rec["bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        sm_sorted = sorted(sm)
+        return {"sm_mhz": sm_sorted[len(sm_sorted) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def workload_numbers(w):
+    B, G, d, n_c = w.B, w.G, w.d, w.n_c[0]
+    n_in = w.n_in(0)
+    vis = B * G * (n_in * n_c + n_in * (n_in + 1) // 2)          # pass 1 pairs
+    ctx = B * G * n_in * n_c                                       # pass 2 pairs
+    k = int(math.floor(w.ratio * n_c))
+    kept = B * k
+    return {
+        "pairs_per_step": B * n_c,
+        "flops_pass1": 2 * d * vis,
+        "flops_pass2": 2 * d * ctx,
+        "flops_algorithmic": 2 * d * vis,
+        "kept": kept,
+        "compact_bytes": kept * d * 2 * 2 * 2 + 4 * kept,
+        "select_bytes": 5 * 4 * B * n_c,
+    }
+
+
+# ---------------------------------------------------------------------------
+# oracle (CPU baseline / reference arm)
+# ---------------------------------------------------------------------------
+def oracle_head_time(x, w, head):
+    """Time the oracle on one head: score, select, compact (the same work the
+    GPU step does for that head).  Returns (seconds, threads)."""
+    import numpy as np
+    from oracle import kvz_oracle as orc
+
+    def bits(t):
+        return t[head].detach().cpu().contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
+
+    Q, Kc, Ki, V = bits(x["Q"]), bits(x["K_ctx"]), bits(x["K_in"]), bits(x["V"])
+    scale = float(np.float32(1.0 / math.sqrt(w.d)))
+    t0 = time.perf_counter()
+    S = orc.score(orc.bf16_bits_to_f64(Q), orc.bf16_bits_to_f64(Kc), orc.bf16_bits_to_f64(Ki), scale)
+    idx, counts, offsets = orc.select(S[None, :].astype(np.float32), w.ratio, w.mode)
+    orc.compact(Kc[None], V[None], idx, counts, offsets)
+    dt = time.perf_counter() - t0
+    try:
+        threads = len(os.sched_getaffinity(0))
+    except Exception:
+        threads = os.cpu_count() or 1
+    return dt, threads
+
+
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    from query_agnostic_kv_kvz_b200 import synth
+    w = synth.WORKLOADS[WORKLOAD]
+    nums = workload_numbers(w)
+    config = {"workload": "%s (L=%d, H=%d, G=%d, d=%d, n_c=%d, n_prompt=%d, keep %.2f %s)" % (
+        w.name, w.L, w.H, w.G, w.d, w.n_c[0], w.n_prompt, w.ratio, w.mode),
+        "B_heads": w.B, "G": w.G, "d": w.d, "n_c": w.n_c[0], "n_in": w.n_in(0), "ratio": w.ratio,
+        "mode": w.mode, "l2": "flushed before every timed step (256 MB write, outside the timed events)",
+        "parallelism": "replicas (weak)" if world > 1 else "single GPU"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            if world > 1:
+                dist.barrier()
+                dist.destroy_process_group()
+            return
+        x = synth.layer_inputs(w, seed=rank, device="cpu")
+        steps, warm = max(1, args.steps if args.steps < 3 else 3), 0
+        times = []
+        threads = 1
+        for s in range(steps):
+            dt, threads = oracle_head_time(x, w, s % w.B)
+            times.append(dt)
+        per_head = sum(times) / len(times)
+        value = w.n_c[0] / per_head
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": steps, "warmup": warm, "ms_per_step": per_head * w.B * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                 "sample": "%d head(s) of the %d-head layer per step (score+select+compact of "
+                                           "one head); ms_per_step extrapolated x%d heads" % (1, w.B, w.B)},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    import query_agnostic_kv_kvz_b200 as kvz
+    kvz.lib()
+    x = synth.layer_inputs(w, seed=rank, device=dev)
+    B, G, d, n_c, n_in = w.B, w.G, w.d, w.n_c[0], w.n_in(0)
+    scale = float(1.0 / math.sqrt(d))
+    stream = torch.cuda.current_stream(dev)
+    rows_pad = (n_in + 255) // 256 * 256
+    lse2 = torch.empty((B, G, rows_pad), dtype=torch.float32, device=dev)
+    S = torch.empty((B, n_c), dtype=torch.float32, device=dev)
+    k = kvz.kvz_keep_count(n_c, w.ratio)
+    idx = torch.empty(B * k, dtype=torch.int32, device=dev)
+    counts = torch.empty(B, dtype=torch.int32, device=dev)
+    offsets = torch.empty(B + 1, dtype=torch.int64, device=dev)
+    sel_ws = torch.empty(kvz.kvz_select_workspace_size(B, n_c, kvz.PER_HEAD), dtype=torch.uint8, device=dev)
+    K_out = torch.empty((B * k, d), dtype=torch.bfloat16, device=dev)
+    V_out = torch.empty((B * k, d), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    launches_per_step = 3 + 10 + 1      # lse, fill, colmax | select: init, 3x(hist, pick), count, scan, write | compact
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kvz.kvz_score_lse2(x["Q"], x["K_ctx"], x["K_in"], scale=scale, lse2=lse2, status=status, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        kvz.kvz_score_colmax(x["Q"], x["K_ctx"], lse2, scale=scale, S=S, accumulate=False, status=status,
+                             stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        kvz.kvz_select(S, w.ratio, w.mode, idx=idx, counts=counts, offsets=offsets, workspace=sel_ws,
+                       status=status, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        kvz.kvz_compact(x["K_ctx"], x["V"], idx, counts, offsets, K_out=K_out, V_out=V_out, status=status,
+                        stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %d during warm-up" % int(status.item()))
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        for s in range(args.steps):
+            flush.zero_()
+            step(evs[s])
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    parts = [[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs]
+    tot = [sum(p) for p in parts]
+    ms_step = sum(tot) / len(tot)
+    part_ms = [sum(p[i] for p in parts) / len(parts) for i in range(4)]
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %d during timing" % int(status.item()))
+
+    # ---- end to end through host buffers (pinned), copies inside the timed region
+    hx = {n: t.cpu().pin_memory() for n, t in x.items()}
+    dx = {n: torch.empty_like(t) for n, t in x.items()}
+    h_out = {"K": torch.empty((B * k, d), dtype=torch.bfloat16).pin_memory(),
+             "V": torch.empty((B * k, d), dtype=torch.bfloat16).pin_memory(),
+             "idx": torch.empty(B * k, dtype=torch.int32).pin_memory(),
+             "counts": torch.empty(B, dtype=torch.int32).pin_memory(),
+             "offsets": torch.empty(B + 1, dtype=torch.int64).pin_memory()}
+    ws_score = torch.empty(kvz.kvz_score_workspace_size(B, G, n_in, 0), dtype=torch.uint8, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+
+    def e2e_step():
+        for n in dx:
+            dx[n].copy_(hx[n], non_blocking=True)
+        kvz.kvz_score(dx["Q"], dx["K_ctx"], dx["K_in"], scale=scale, S=S, workspace=ws_score, status=status,
+                      stream=stream)
+        kvz.kvz_select(S, w.ratio, w.mode, idx=idx, counts=counts, offsets=offsets, workspace=sel_ws,
+                       status=status, stream=stream)
+        kvz.kvz_compact(dx["K_ctx"], dx["V"], idx, counts, offsets, K_out=K_out, V_out=V_out, status=status,
+                        stream=stream)
+        h_out["K"].copy_(K_out, non_blocking=True)
+        h_out["V"].copy_(V_out, non_blocking=True)
+        h_out["idx"].copy_(idx, non_blocking=True)
+        h_out["counts"].copy_(counts, non_blocking=True)
+        h_out["offsets"].copy_(offsets, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %d during e2e" % int(status.item()))
+
+    if world > 1:
+        t = torch.tensor([ms_step, e2e_ms] + part_ms, dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, e2e_ms = float(t[0]), float(t[1])
+        part_ms = [float(v) for v in t[2:]]
+
+    pk = peaks()
+    lse_ms, col_ms, sel_ms, cmp_ms = part_ms
+    score_ms = lse_ms + col_ms
+    fl1, fl2 = nums["flops_pass1"], nums["flops_pass2"]
+    tf = lambda flops, ms: flops / (ms * 1e-3) / 1e12
+    roof = {
+        "bound": "tensor",
+        "kernel": "lse_kernel (score pass 1: QK^T + online log-sum-exp)",
+        "achieved": tf(fl1, lse_ms),
+        "peak": pk["bf16_tflops"],
+        "unit": "TFLOP/s",
+        "frac": tf(fl1, lse_ms) / pk["bf16_tflops"],
+        "traffic": recorded_traffic("lse_kernel"),
+        "peak_source": "%s bf16 dense (burst)" % pk["source"],
+        "algorithmic_flops_per_launch": fl1,
+        "breakdown": {
+            "score_pass1_ms": lse_ms, "score_pass2_ms": col_ms, "select_ms": sel_ms, "compact_ms": cmp_ms,
+            "score_tflops_executed": tf(fl1 + fl2, score_ms),
+            "score_frac_executed": tf(fl1 + fl2, score_ms) / pk["bf16_tflops"],
+            "score_tflops_algorithmic": tf(nums["flops_algorithmic"], score_ms),
+            "score_frac_algorithmic": tf(nums["flops_algorithmic"], score_ms) / pk["bf16_tflops"],
+            "pass2_tflops": tf(fl2, col_ms), "pass2_frac": tf(fl2, col_ms) / pk["bf16_tflops"],
+            "compact_gbs": nums["compact_bytes"] / (cmp_ms * 1e-3) / 1e9,
+            "compact_frac_hbm": nums["compact_bytes"] / (cmp_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "select_gbs": nums["select_bytes"] / (sel_ms * 1e-3) / 1e9,
+        },
+    }
+    value = nums["pairs_per_step"] * world / (ms_step * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config, "roofline": roof,
+        "e2e": {"value": nums["pairs_per_step"] * world / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, threads = oracle_head_time(x, w, 0)
+        line["cpu_baseline"] = {"value": n_c / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": "head 0 of the %d-head layer: fp64 score + select + compact "
+                                          "(%.1f s)" % (B, dt)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
