@@ -231,8 +231,9 @@ def main():
         return
 
     import query_agnostic_kv_kvz_b200 as kvz
+    from query_agnostic_kv_kvz_b200.dist import max_over_ranks, rank_seed
     kvz.lib()
-    x = synth.layer_inputs(w, seed=rank, device=dev)
+    x = synth.layer_inputs(w, seed=rank_seed(0, rank), device=dev)
     B, G, d, n_c, n_in = w.B, w.G, w.d, w.n_c[0], w.n_in(0)
     scale = float(1.0 / math.sqrt(d))
     stream = torch.cuda.current_stream(dev)
@@ -336,11 +337,8 @@ def main():
     if int(status.item()) != 0:
         raise RuntimeError("device status %d during e2e" % int(status.item()))
 
-    if world > 1:
-        t = torch.tensor([ms_step, e2e_ms] + part_ms, dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, e2e_ms = float(t[0]), float(t[1])
-        part_ms = [float(v) for v in t[2:]]
+    red = max_over_ranks([ms_step, e2e_ms] + part_ms, device=dev)
+    ms_step, e2e_ms, part_ms = red[0], red[1], red[2:]
 
     pk = peaks()
     lse_ms, col_ms, sel_ms, cmp_ms = part_ms

@@ -1,0 +1,132 @@
+"""Argument validation of the C ABI: every rejected call returns its status
+before anything is launched.  Runs on the GPU with real, correctly sized
+buffers (so a validation bug could not reach a kernel with a bad pointer)
+and on the CPU with placeholder addresses (nothing is launched there)."""
+import ctypes
+
+import pytest
+import torch
+
+import query_agnostic_kv_kvz_b200 as kvz
+
+OK, INVALID, UNSUPPORTED, ALIGN, WS = 0, 1, 2, 3, 4
+
+
+class Bufs:
+    """Device buffers when CUDA is present, else fake 256-aligned addresses."""
+
+    def __init__(self):
+        self.cuda = torch.cuda.is_available()
+        self.keep = []
+        self.fake = 1 << 20
+
+    def get(self, nbytes):
+        if self.cuda:
+            t = torch.zeros(max(16, nbytes), dtype=torch.uint8, device="cuda")
+            self.keep.append(t)
+            return t.data_ptr()
+        self.fake += ((nbytes + 255) // 256 + 1) * 256
+        return self.fake
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from query_agnostic_kv_kvz_b200 import build
+    build.build()
+    return kvz.lib()
+
+
+def vp(x):
+    return ctypes.c_void_p(x)
+
+
+def _score(lib, bufs, B=1, G=1, n_c=128, n_in=128, d=128, scale=0.1, row_chunk=0, ws_bytes=None,
+           shift=0, ws_ptr=True):
+    Q = bufs.get(B * G * n_in * d * 2) + shift
+    Kc = bufs.get(B * n_c * d * 2)
+    Ki = bufs.get(B * n_in * d * 2)
+    S = bufs.get(B * n_c * 4)
+    need = lib.kvz_score_workspace_size(B, G, n_in, row_chunk if row_chunk % 256 == 0 else 0)
+    ws = bufs.get(need) if ws_ptr else 0
+    return lib.kvz_score(vp(Q), vp(Kc), vp(Ki), B, G, n_c, n_in, d, scale, row_chunk, vp(S), vp(ws),
+                         need if ws_bytes is None else ws_bytes, None, None)
+
+
+def test_score_rejections(lib):
+    b = Bufs()
+    assert _score(lib, b, d=96) == UNSUPPORTED
+    assert _score(lib, b, d=256) == UNSUPPORTED
+    assert _score(lib, b, scale=0.0) == INVALID
+    assert _score(lib, b, scale=float("nan")) == INVALID
+    assert _score(lib, b, scale=float("inf")) == INVALID
+    assert _score(lib, b, G=0) == INVALID
+    assert _score(lib, b, n_c=0) == INVALID
+    assert _score(lib, b, row_chunk=100) == INVALID
+    assert _score(lib, b, shift=2) == ALIGN
+    assert _score(lib, b, ws_bytes=16) == WS
+    assert _score(lib, b, ws_ptr=False) == WS
+    assert lib.kvz_score(None, None, None, 1, 1, 8, 8, 128, 0.1, 0, None, None, 0, None, None) == INVALID
+
+
+def test_pass_rejections(lib):
+    b = Bufs()
+    Q, Kc, Ki = b.get(4 * 512 * 128 * 2), b.get(512 * 128 * 2), b.get(512 * 128 * 2)
+    lse = b.get(4 * 512 * 4)
+    S = b.get(512 * 4)
+    # i_begin not a multiple of 256, range outside n_in, ld too small
+    assert lib.kvz_score_lse2(vp(Q), vp(Kc), vp(Ki), 1, 4, 512, 512, 128, 0.1, 100, 512, vp(lse), 512, None,
+                              None) == INVALID
+    assert lib.kvz_score_lse2(vp(Q), vp(Kc), vp(Ki), 1, 4, 512, 512, 128, 0.1, 0, 513, vp(lse), 512, None,
+                              None) == INVALID
+    assert lib.kvz_score_lse2(vp(Q), vp(Kc), vp(Ki), 1, 4, 512, 512, 128, 0.1, 0, 512, vp(lse), 256, None,
+                              None) == INVALID
+    assert lib.kvz_score_lse2(vp(Q), vp(Kc), vp(Ki), 1, 4, 512, 512, 128, 0.1, 0, 512, vp(lse), 510, None,
+                              None) == ALIGN
+    assert lib.kvz_score_colmax(vp(Q), vp(Kc), 1, 4, 512, 512, 128, 0.1, 256, 128, vp(lse), 512, vp(S), 0, None,
+                                None) == INVALID
+    assert lib.kvz_score_colmax(vp(Q), vp(Kc), 1, 4, 512, 512, 128, 0.1, 0, 512, None, 512, vp(S), 0, None,
+                                None) == INVALID
+
+
+def test_select_rejections(lib):
+    b = Bufs()
+    B, n_c = 4, 1000
+    S = b.get(B * n_c * 4)
+    idx, cnt, off = b.get(B * n_c * 4), b.get(B * 4), b.get((B + 1) * 8)
+    ws_n = lib.kvz_select_workspace_size(B, n_c, 0)
+    ws = b.get(ws_n)
+
+    def call(ratio=0.3, mode=0, cap=B * n_c, wsb=ws_n, s_shift=0, Bx=B):
+        return lib.kvz_select(vp(S + s_shift), Bx, n_c, ratio, mode, vp(idx), cap, vp(cnt), vp(off), vp(ws), wsb,
+                              None, None)
+
+    assert call(ratio=1.5) == INVALID
+    assert call(ratio=-0.1) == INVALID
+    assert call(ratio=float("nan")) == INVALID
+    assert call(mode=3) == INVALID
+    assert call(cap=B * 300 - 1) == INVALID          # per head: 4 * floor(0.3*1000) = 1200 needed
+    assert call(wsb=16) == WS
+    assert call(s_shift=2) == ALIGN
+    assert call(Bx=70000) == INVALID
+
+
+def test_compact_rejections(lib):
+    b = Bufs()
+    B, n_c, d = 2, 256, 128
+    K, V = b.get(B * n_c * d * 2), b.get(B * n_c * d * 2)
+    Ko, Vo = b.get(B * n_c * d * 2), b.get(B * n_c * d * 2)
+    idx, cnt, off = b.get(B * n_c * 4), b.get(B * 4), b.get((B + 1) * 8)
+    outo = b.get((B + 1) * 8)
+
+    def call(K_=K, V_=V, Ko_=Ko, Vo_=Vo, d_=d, oo=None):
+        return lib.kvz_compact(vp(K_), vp(V_), B, n_c, d_, vp(idx), vp(cnt), vp(off), vp(oo) if oo else None,
+                               vp(Ko_), vp(Vo_), None, None)
+
+    assert call(d_=96) == UNSUPPORTED
+    assert call(Ko_=K) == INVALID                    # K in place, V not
+    assert call(Ko_=K, Vo_=V, oo=outo) == INVALID    # in place takes no output offsets
+    assert call(V_=K) == INVALID                     # K and V are the same buffer
+    assert call(Ko_=K + 4096) == INVALID             # output starts inside an input
+    assert call(Ko_=Ko + 8) == ALIGN
+    assert lib.kvz_compact(vp(K), vp(V), B, n_c, d, None, vp(cnt), vp(off), None, vp(Ko), vp(Vo), None,
+                           None) == INVALID
