@@ -14,7 +14,8 @@
 //                           because every row sees every context key.
 // Both kernels: warp 0 issues TMA loads, warp 1 (one thread) issues
 // tcgen05.mma into tensor memory, warp 2 owns the TMEM allocation, warps
-// 4..11 (two warpgroups) read TMEM and do the softmax / max arithmetic.
+// 4..19 (four warpgroups, each owning half of a tile's 128 TMEM columns)
+// read TMEM and do the softmax / max arithmetic.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -28,10 +29,18 @@ namespace kvz {
 
 namespace {
 
-constexpr int kThreads = 384;     // 12 warps
+constexpr int kThreads = 640;     // 4 control warps + 4 epilogue warpgroups
 constexpr int kTile = 128;        // rows of a Q sub-tile / keys of a K tile
 constexpr int kSubBytes64 = kTile * 128;  // one 128-row x 64-column bf16 block (16 KB)
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128);
+
+// Of every 16 exp2 evaluations in pass 1, how many run as a polynomial on
+// the FMA pipe instead of the SFU (even, 0..16).
+#ifndef KVZ_POLY_PER16
+#define KVZ_POLY_PER16 4
+#endif
+constexpr int kPolyPer16 = KVZ_POLY_PER16;
+static_assert(kPolyPer16 % 2 == 0 && kPolyPer16 >= 0 && kPolyPer16 <= 16, "pairs of exp2");
 
 template <int D>
 struct LseLayout {
@@ -41,7 +50,8 @@ struct LseLayout {
   static constexpr int KST = 4;                          // K-tile pipeline depth
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + NQ * TILE_BYTES;
-  static constexpr int BAR_OFF = K_OFF + KST * TILE_BYTES;
+  static constexpr int MERGE_OFF = K_OFF + KST * TILE_BYTES;  // (max, sum) of the second column half
+  static constexpr int BAR_OFF = MERGE_OFF + NQ * kTile * 2 * 4;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;  // + alignment slack
 };
@@ -52,11 +62,12 @@ struct ColLayout {
   static constexpr int TILE_BYTES = KB * kSubBytes64;
   static constexpr int NA = 2;                           // key tiles per CTA (256 keys)
   static constexpr int QST = 4;                          // Q-tile pipeline depth
+  static constexpr int LST = 8;                          // lse2-slice ring depth
   static constexpr int A_OFF = 0;
   static constexpr int Q_OFF = A_OFF + NA * TILE_BYTES;
   static constexpr int L_OFF = Q_OFF + QST * TILE_BYTES;  // lse2 slices, 128 floats each
-  static constexpr int BAR_OFF = L_OFF + QST * kTile * 4;
-  static constexpr int BAR_BYTES = 256;
+  static constexpr int BAR_OFF = L_OFF + LST * kTile * 4;
+  static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;
 };
 
@@ -83,6 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sQ = smem + Lay::Q_OFF;
   uint8_t* sK = smem + Lay::K_OFF;
+  float* sMerge = reinterpret_cast<float*>(smem + Lay::MERGE_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;                  // [KST]
@@ -120,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 4; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 4);
+      mbar_init(&s_empty[s], 8);                // 8 softmax warps read each buffer
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -194,75 +206,109 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ------------------------------------------------ softmax warpgroups
-    const int q = (warp - 4) >> 2;
+  }
+
+  // ------------------------------------------------ softmax warpgroups
+  // Four warpgroups: (sub-tile q, column half h).  A thread owns one query
+  // row (its TMEM lane) and 64 of the 128 key columns of every tile; the
+  // two halves' (max, sum) pairs merge exactly at the end.
+  const int ew = warp - 4;
+  const int q = (ew >> 3) & 1;
+  const int h = (ew >> 2) & 1;
+  const int rl = (warp & 3) * 32 + lane;            // row within the sub-tile == TMEM lane
+  float m = -INFINITY, l = 0.0f;
+  bool ok = true;
+  if (warp >= 4 && q < nq_valid) {
     const int wq = warp & 3;
-    const int rl = wq * 32 + lane;                  // row within the sub-tile == TMEM lane
-    const int64_t i = i0 + q * kTile + rl;
     const float c2 = p.c2;
-    float m = -INFINITY, l = 0.0f;
-    bool ok = true;
-    if (q < nq_valid) {
-      const int ctx_tail = static_cast<int>(p.n_c - static_cast<int64_t>(NC - 1) * kTile);
-      uint32_t cnt = 0;
-      for (int t = 0; t < NT; ++t) {
-        if (t >= NC && t - NC >= nin[q]) continue;
-        const uint32_t buf = cnt & 1u;
-        const uint32_t bu = cnt >> 1;
-        if (!mbar_wait_warp(&s_full[q * 2 + buf], bu & 1u, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        float v[128];
-        tmem_ld128(tmem + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>((q * 2 + buf) * kTile), v);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[q * 2 + buf]);
-        if (t == NC - 1 && ctx_tail < kTile) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= ctx_tail) v[c] = -INFINITY;
-        }
-        if (t >= NC && t - NC == nin[q] - 1) {       // diagonal input tile
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c > rl) v[c] = -INFINITY;
-        }
-        float mx0 = v[0], mx1 = v[1], mx2 = v[2], mx3 = v[3];
-#pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          mx0 = fmaxf(mx0, v[c]);
-          mx1 = fmaxf(mx1, v[c + 1]);
-          mx2 = fmaxf(mx2, v[c + 2]);
-          mx3 = fmaxf(mx3, v[c + 3]);
-        }
-        const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c2;
-        // Move the reference max only when it grows by more than 2^8; the
-        // sum is exact for any reference, and values stay below 2^8.
-        if (mt > m + 8.0f) {
-          l *= ex2_approx(m - mt);
-          m = mt;
-        }
-        const float nm = -m;
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-        for (int c = 0; c < 128; c += 4) {
-          a0 += ex2_approx(fmaf(v[c], c2, nm));
-          a1 += ex2_approx(fmaf(v[c + 1], c2, nm));
-          a2 += ex2_approx(fmaf(v[c + 2], c2, nm));
-          a3 += ex2_approx(fmaf(v[c + 3], c2, nm));
-        }
-        l += (a0 + a1) + (a2 + a3);
-        ++cnt;
+    const int ctx_tail = static_cast<int>(p.n_c - static_cast<int64_t>(NC - 1) * kTile) - h * 64;
+    const int diag_lim = rl - h * 64;                 // diagonal tile: column c visible iff c <= diag_lim
+    uint32_t cnt = 0;
+    for (int t = 0; t < NT; ++t) {
+      if (t >= NC && t - NC >= nin[q]) continue;
+      const uint32_t buf = cnt & 1u;
+      const uint32_t bu = cnt >> 1;
+      if (!mbar_wait_warp(&s_full[q * 2 + buf], bu & 1u, abort_flag, p.status)) {
+        ok = false;
+        break;
       }
+      tc_fence_after();
+      float v[64];
+      tmem_ld64(tmem + (static_cast<uint32_t>(wq * 32) << 16) +
+                    static_cast<uint32_t>((q * 2 + buf) * kTile + h * 64), v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[q * 2 + buf]);
+      if (t == NC - 1 && ctx_tail < 64) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c >= ctx_tail) v[c] = -INFINITY;
+      }
+      if (t >= NC && t - NC == nin[q] - 1) {       // diagonal input tile
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c > diag_lim) v[c] = -INFINITY;
+      }
+      // tile max: two independent chains of 3-input max
+      float mx[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        float a = v[32 * k];
+#pragma unroll
+        for (int c = 1; c < 31; c += 2) a = fmax3(a, v[32 * k + c], v[32 * k + c + 1]);
+        mx[k] = fmaxf(a, v[32 * k + 31]);
+      }
+      const float mt = fmaxf(mx[0], mx[1]) * c2;
+      // Move the reference max only when it grows by more than 2^8; the
+      // sum is exact for any reference, and values stay below 2^8.  A half
+      // that is fully masked (mt = -inf) changes nothing.
+      if (mt > m + 8.0f) {
+        l *= ex2_approx(m - mt);
+        m = mt;
+      }
+      if (m != -INFINITY) {
+        // 2^(c2*s - m): 16 - kPolyPer16 of every 16 on the SFU, the rest on
+        // the FMA pipe, so neither unit limits the pass on its own.
+        const float2 c22 = make_float2(c2, c2);
+        const float2 nm2 = make_float2(-m, -m);
+        float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0;
+#pragma unroll
+        for (int c = 0; c < 64; c += 16) {
+#pragma unroll
+          for (int k = 0; k < 16 - kPolyPer16; k += 2) {
+            const float2 x = __ffma2_rn(make_float2(v[c + k], v[c + k + 1]), c22, nm2);
+            const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (k & 2) s0 = __fadd2_rn(s0, e); else s1 = __fadd2_rn(s1, e);
+          }
+#pragma unroll
+          for (int k = 16 - kPolyPer16; k < 16; k += 2) {
+            const float2 x = __ffma2_rn(make_float2(v[c + k], v[c + k + 1]), c22, nm2);
+            s2 = __fadd2_rn(s2, exp2_poly2(x));
+          }
+        }
+        l += ((s0.x + s0.y) + (s1.x + s1.y)) + (s2.x + s2.y);
+      }
+      ++cnt;
     }
-    const float lse2 = (q < nq_valid && ok && i < row_hi) ? m + log2f(l) : INFINITY;
-    p.lse2[static_cast<int64_t>(bg) * p.ld + (i - p.i_begin)] = lse2;
+  }
+  if (warp >= 4 && h == 1) {
+    sMerge[(q * kTile + rl) * 2 + 0] = m;
+    sMerge[(q * kTile + rl) * 2 + 1] = ok ? l : -1.0f;
   }
 
   __syncthreads();
+  if (warp >= 4 && h == 0) {
+    const int64_t i = i0 + q * kTile + rl;
+    const float m1 = sMerge[(q * kTile + rl) * 2 + 0];
+    const float l1 = sMerge[(q * kTile + rl) * 2 + 1];
+    float lse2 = INFINITY;
+    if (q < nq_valid && ok && l1 >= 0.0f && i < row_hi) {
+      const float mm = fmaxf(m, m1);                 // finite: every row sees a key
+      const float ll = (m == -INFINITY ? 0.0f : l * exp2f(m - mm)) + (m1 == -INFINITY ? 0.0f : l1 * exp2f(m1 - mm));
+      lse2 = mm + log2f(ll);
+    }
+    p.lse2[static_cast<int64_t>(bg) * p.ld + (i - p.i_begin)] = lse2;
+  }
   if (*abort_flag) {
     // Unwinding after a timeout: let this CTA's own copies and MMAs finish
     // (bounded) before shared and tensor memory are released.
@@ -287,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ============================================================================
-// Pass 2: S[b, j] = max(S[b, j], 2^(max_r c2 <q_r, k_j> - lse2_r)).
+// Pass 2: S[b, j] = max(S[b, j], 2^-(min_r lse2_r - c2 <q_r, k_j>)).
 // CTA = (head b, 256 context keys, a contiguous range of 128-row Q tiles).
 // Keys are the MMA's M side, so TMEM lane = key and each thread keeps the
 // running max of its key over the query-row columns in a register.
@@ -318,7 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* a_full = bars + 0;
   uint64_t* q_full = bars + 1;                   // [QST]
   uint64_t* q_empty = q_full + Lay::QST;         // [QST]
-  uint64_t* acc_full = q_empty + Lay::QST;       // [2 key tiles][2 buffers]
+  uint64_t* l_full = q_empty + Lay::QST;         // [LST]
+  uint64_t* l_empty = l_full + Lay::LST;         // [LST]
+  uint64_t* acc_full = l_empty + Lay::LST;       // [2 key tiles][2 buffers]
   uint64_t* acc_empty = acc_full + 4;            // [2][2]
   uint64_t* drain = acc_empty + 4;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -332,11 +380,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(a_full, 1);
     for (int s = 0; s < Lay::QST; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1 + 8);            // MMA commit + 8 epilogue warps
+      mbar_init(&q_empty[s], 1);                // freed by the MMA commit alone
+    }
+    for (int s = 0; s < Lay::LST; ++s) {
+      mbar_init(&l_full[s], 1);
+      mbar_init(&l_empty[s], 16);               // 16 epilogue warps read each slice
     }
     for (int s = 0; s < 4; ++s) {
       mbar_init(&acc_full[s], 1);
-      mbar_init(&acc_empty[s], 4);
+      mbar_init(&acc_empty[s], 8);              // 8 epilogue warps read each buffer
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -351,7 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  int issued = 0;   // Q tiles whose loads were issued (producer thread)
+  int issued = 0;     // Q tiles whose loads were issued (producer thread)
+  int l_issued = 0;   // lse2 slices whose loads were issued
   if (warp == 0) {
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -364,17 +417,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int n = 0; n < ntile; ++n) {
         const int s = n % Lay::QST;
         const uint32_t use = static_cast<uint32_t>(n / Lay::QST);
-        if (!mbar_wait(&q_empty[s], (use & 1u) ^ 1u, abort_flag, p.status)) break;
+        const int sl = n % Lay::LST;
+        const uint32_t luse = static_cast<uint32_t>(n / Lay::LST);
         const int tau = t_begin + n;
         const int g = tau / tpg;
         const int il = (tau % tpg) * kTile;
         const int bgq = b * p.G + g;
-        mbar_arrive_expect_tx(&q_full[s], Lay::TILE_BYTES + kTile * 4);
+        if (!mbar_wait(&q_empty[s], (use & 1u) ^ 1u, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&q_full[s], Lay::TILE_BYTES);
         for (int kb = 0; kb < Lay::KB; ++kb)
           tma_load_3d(sQ + s * Lay::TILE_BYTES + kb * kSubBytes64, &tmQ, &q_full[s], kb * 64,
                       static_cast<int>(p.i_begin + il), bgq);
-        bulk_load(sL + s * kTile, p.lse2 + static_cast<int64_t>(bgq) * p.ld + il, kTile * 4, &q_full[s]);
         issued = n + 1;
+        if (!mbar_wait(&l_empty[sl], (luse & 1u) ^ 1u, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&l_full[sl], kTile * 4);
+        bulk_load(sL + sl * kTile, p.lse2 + static_cast<int64_t>(bgq) * p.ld + il, kTile * 4, &l_full[sl]);
+        l_issued = n + 1;
       }
     }
     __syncwarp();
@@ -409,15 +467,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int a = (warp - 4) >> 2;
+    // Four epilogue warpgroups: (key tile a, row half h).  A thread owns one
+    // context key (its TMEM lane) and 64 of the 128 query-row columns.
+    const int ew = warp - 4;
+    const int a = ew >> 3;
+    const int h = (ew >> 2) & 1;
     const int wq = warp & 3;
     const int64_t j = key0 + a * kTile + wq * 32 + lane;   // context key == TMEM lane
     const float c2 = p.c2;
-    float mx = -INFINITY;
+    float ymin = INFINITY;     // min over rows of lse2_r - c2*<q_r, k_j>
     bool ok = true;
     for (int n = 0; n < ntile; ++n) {
-      const int s = n % Lay::QST;
-      const uint32_t use = static_cast<uint32_t>(n / Lay::QST);
+      const int sl = n % Lay::LST;
+      const uint32_t luse = static_cast<uint32_t>(n / Lay::LST);
       const uint32_t buf = static_cast<uint32_t>(n) & 1u;
       const uint32_t bu = static_cast<uint32_t>(n) >> 1;
       if (!mbar_wait_warp(&acc_full[a * 2 + buf], bu & 1u, abort_flag, p.status)) {
@@ -425,32 +487,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float v[128];
-      tmem_ld128(tmem + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>((a * 2 + buf) * kTile), v);
+      float v[64];
+      tmem_ld64(tmem + (static_cast<uint32_t>(wq * 32) << 16) +
+                    static_cast<uint32_t>((a * 2 + buf) * kTile + h * 64), v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[a * 2 + buf]);
-      // the lse2 slice arrived with the Q tile on q_full[s]
-      if (!mbar_wait_warp(&q_full[s], use & 1u, abort_flag, p.status)) {
+      if (!mbar_wait_warp(&l_full[sl], luse & 1u, abort_flag, p.status)) {
         ok = false;
         break;
       }
-      const float4* L = reinterpret_cast<const float4*>(sL + s * kTile);
-      float m0 = mx, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+      // min over rows of lse2_r - c2*s (the negated exponent), two chains
+      const float4* L = reinterpret_cast<const float4*>(sL + sl * kTile + h * 64);
+      const float2 nc22 = make_float2(-c2, -c2);
+      float y0 = ymin, y1 = INFINITY;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < 16; ++c) {
         const float4 l4 = L[c];
-        m0 = fmaxf(m0, fmaf(v[4 * c + 0], c2, -l4.x));
-        m1 = fmaxf(m1, fmaf(v[4 * c + 1], c2, -l4.y));
-        m2 = fmaxf(m2, fmaf(v[4 * c + 2], c2, -l4.z));
-        m3 = fmaxf(m3, fmaf(v[4 * c + 3], c2, -l4.w));
+        const float2 ya = __ffma2_rn(make_float2(v[4 * c + 0], v[4 * c + 1]), nc22, make_float2(l4.x, l4.y));
+        const float2 yb = __ffma2_rn(make_float2(v[4 * c + 2], v[4 * c + 3]), nc22, make_float2(l4.z, l4.w));
+        y0 = fmin3(y0, ya.x, ya.y);
+        y1 = fmin3(y1, yb.x, yb.y);
       }
-      mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+      ymin = fminf(y0, y1);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&q_empty[s]);
+      if (lane == 0) mbar_arrive(&l_empty[sl]);
     }
     if (ok && j < p.n_c) {
-      const float sj = exp2f(mx);   // >= +0, so its bit pattern orders like the value
+      const float sj = exp2f(-ymin);   // >= +0, so its bit pattern orders like the value
       atomicMax(reinterpret_cast<unsigned int*>(p.S + static_cast<int64_t>(b) * p.n_c + j), __float_as_uint(sj));
     }
   }
@@ -462,6 +526,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < Lay::QST && s < issued; ++s) {
         const int n_last = s + Lay::QST * ((issued - 1 - s) / Lay::QST);
         mbar_wait_for(&q_full[s], static_cast<uint32_t>(n_last / Lay::QST) & 1u, 20000000ull);
+      }
+      for (int s = 0; s < Lay::LST && s < l_issued; ++s) {
+        const int n_last = s + Lay::LST * ((l_issued - 1 - s) / Lay::LST);
+        mbar_wait_for(&l_full[s], static_cast<uint32_t>(n_last / Lay::LST) & 1u, 20000000ull);
       }
     }
     if (warp == 1 && lane == 0) {
