@@ -134,6 +134,43 @@ kvz_status kvz_score_colmax(const void* Q, const void* K_ctx,
                             int32_t* d_status, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Scoring without any caller-provided or allocated scratch memory.          */
+/*                                                                          */
+/* The KVzip paper has no counterpart to this call; it exists for callers   */
+/* that cannot allocate device memory at the point where they score: an     */
+/* engine whose memory pool owns the whole GPU and forbids further          */
+/* cudaMalloc, a plugin or callback that has no access to the host          */
+/* program's allocator, or a latency-critical path that must not risk the   */
+/* implicit device synchronisation a cudaMalloc/cudaFree can cause.         */
+/*                                                                          */
+/* It computes exactly what kvz_score computes (same arguments minus the    */
+/* workspace and row_chunk; Q, K_ctx, K_in and S are still the caller's).   */
+/* The per-row log-sum-exp scratch is a fixed static device array of        */
+/* KVZ_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads */
+/* the library holds until the process exits.  Rows are processed in        */
+/* chunks of as many 256-row blocks as fit in it, which does not change the */
+/* result.                                                                  */
+/*                                                                          */
+/* - Returns KVZ_ERR_WORKSPACE, launching nothing, when one 256-row block   */
+/*   of every head and group does not fit: B*G*256*4 > KVZ_NOALLOC_SCRATCH_ */
+/*   BYTES (B*G > 8192).  Other argument errors are those of kvz_score.     */
+/* - The first call on each device looks up the array's device address     */
+/*   (cudaGetSymbolAddress) with that device current; make that first call  */
+/*   before any stream capture that would contain a later one.              */
+/* - Every call on a device uses the same array and leaves its contents     */
+/*   behind.  Nothing in it needs to start at zero (each call writes every  */
+/*   entry before reading it), but calls that overlap on the GPU (two       */
+/*   streams, or two host threads) race on it: keep them ordered, e.g. on   */
+/*   one stream.                                                             */
+/* ------------------------------------------------------------------------ */
+#define KVZ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+kvz_status kvz_score_noalloc(const void* Q, const void* K_ctx, const void* K_in,
+                             int64_t B, int G, int64_t n_c, int64_t n_in, int d,
+                             float scale, float* S,
+                             int32_t* d_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Selection.                                                                */
 /*                                                                          */
 /* KVzip §4.1 keeps the r% highest-scoring KV pairs across all heads         */

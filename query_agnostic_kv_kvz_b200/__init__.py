@@ -59,6 +59,7 @@ _SIGS = {
                               _vp]),
     "kvz_score_colmax": (_i32, [_vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _i64, _i64, _vp, _i64, _vp,
                                 _i32, _vp, _vp]),
+    "kvz_score_noalloc": (_i32, [_vp, _vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _vp, _vp, _vp]),
     "kvz_keep_count": (_i64, [_i64, _f64]),
     "kvz_select_workspace_size": (_sz, [_i64, _i64, _i32]),
     "kvz_select": (_i32, [_vp, _i64, _i64, _f64, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
@@ -147,6 +148,22 @@ def kvz_score(Q, K_ctx, K_in, scale: Optional[float] = None, row_chunk: int = 0,
     nbytes = workspace.numel() * workspace.element_size()
     _check("kvz_score", lib().kvz_score(_ptr(Q), _ptr(K_ctx), _ptr(K_in), B, G, n_c, n_in, d, scale, row_chunk,
                                         _ptr(S), _ptr(workspace), nbytes, _ptr(status), _stream(stream)))
+    return S
+
+
+def kvz_score_noalloc(Q, K_ctx, K_in, scale: Optional[float] = None, S=None, status=None, stream=None):
+    """kvz_score without a workspace: for callers that cannot allocate device
+    memory when they score.  The library's fixed static scratch is used
+    instead (see include/kvz.h); only S is allocated here, and only when the
+    caller passes none.  Calls that overlap on the GPU share that scratch."""
+    _need_cuda(Q, K_ctx, K_in, S, status)
+    B, G, n_in, d, n_c = _score_shapes(Q, K_ctx, K_in)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if S is None:
+        S = torch.empty((B, n_c), dtype=torch.float32, device=Q.device)
+    _check("kvz_score_noalloc", lib().kvz_score_noalloc(_ptr(Q), _ptr(K_ctx), _ptr(K_in), B, G, n_c, n_in, d,
+                                                        scale, _ptr(S), _ptr(status), _stream(stream)))
     return S
 
 

@@ -195,6 +195,65 @@ kvz_status kvz_score(const void* Q, const void* K_ctx, const void* K_in, int64_t
   return KVZ_OK;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free scoring: the lse2 scratch is this file-scope device array.
+// In host code its name only stands in for the symbol; the device address
+// comes from cudaGetSymbolAddress, once per device.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) float kvz_noalloc_lse2[KVZ_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mu;
+float* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device.
+kvz_status noalloc_scratch(float** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVZ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, kvz_noalloc_lse2) != cudaSuccess || p == nullptr) return KVZ_ERR_CUDA;
+    g_noalloc_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return KVZ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvz_status kvz_score_noalloc(const void* Q, const void* K_ctx, const void* K_in, int64_t B, int G, int64_t n_c,
+                             int64_t n_in, int d, float scale, float* S, int32_t* d_status, cudaStream_t stream) {
+  kvz_status st = check_score_common(Q, K_ctx, B, G, n_c, n_in, d, scale);
+  if (st != KVZ_OK) return st;
+  if (K_in == nullptr || S == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(K_in, 16) || !aligned(S, 4)) return KVZ_ERR_ALIGNMENT;
+  constexpr int64_t cap = KVZ_NOALLOC_SCRATCH_BYTES / sizeof(float);
+  const int64_t per_block = B * G * 256;                 // floats for one 256-row block of every (b, g)
+  if (per_block > cap) return KVZ_ERR_WORKSPACE;
+  int64_t chunk = (cap / per_block) * 256;
+  if (chunk >= n_in) chunk = n_in;
+  const int64_t ld = roundup(chunk, 256);
+  float* lse2 = nullptr;
+  st = noalloc_scratch(&lse2);
+  if (st != KVZ_OK) return st;
+  if (kvz::launch_fill_f32(S, B * n_c, 0.0f, stream) != cudaSuccess) return KVZ_ERR_CUDA;
+  for (int64_t i0 = 0; i0 < n_in; i0 += chunk) {
+    const int64_t i1 = i0 + chunk < n_in ? i0 + chunk : n_in;
+    st = run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, d_status, stream);
+    if (st != KVZ_OK) return st;
+    st = run_colmax(Q, K_ctx, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, S, d_status, stream);
+    if (st != KVZ_OK) return st;
+  }
+  return KVZ_OK;
+}
+
 int64_t kvz_keep_count(int64_t n, double ratio) {
   if (n < 0 || !(ratio >= 0.0 && ratio <= 1.0)) return -1;
   return static_cast<int64_t>(std::floor(ratio * static_cast<double>(n)));
