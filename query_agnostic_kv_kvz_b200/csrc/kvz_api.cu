@@ -14,7 +14,6 @@
 namespace {
 
 constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1024;   // TMA coordinates are int32
-constexpr int kNumSMs = 148;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 int64_t roundup(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -102,19 +101,6 @@ kvz_status run_colmax(const void* Q, const void* K_ctx, int64_t B, int G, int64_
   a.lse2 = lse2;
   a.S = S;
   a.status = status;
-  a.n_kblk = static_cast<int>((n_c + 255) / 256);
-  // Split each (head, key block)'s row tiles so the grid fills ~8 waves.
-  const int64_t T = G * (a.rows_pad / 128);
-  const int64_t base_units = B * a.n_kblk;
-  int64_t nsplit = (kNumSMs * 8 + base_units - 1) / base_units;
-  const int64_t max_split = T / 4 > 1 ? T / 4 : 1;
-  if (nsplit > max_split) nsplit = max_split;
-  if (nsplit < 1) nsplit = 1;
-  const int64_t tps = (T + nsplit - 1) / nsplit;
-  nsplit = (T + tps - 1) / tps;
-  if (base_units * nsplit > 0x7FFFFFFF) return KVZ_ERR_INVALID_ARG;
-  a.nsplit = static_cast<int>(nsplit);
-  a.tiles_per_split = static_cast<int>(tps);
   return kvz::launch_colmax(d, tmQ, tmKc, a, stream) == cudaSuccess ? KVZ_OK : KVZ_ERR_CUDA;
 }
 

@@ -28,9 +28,9 @@ struct ColArgs {
   int64_t i_begin, rows_pad, ld;
   const float* lse2;
   float* S;
-  int n_kblk;               // ceil(n_c / 256)
-  int nsplit;               // row-tile ranges per (head, key block)
-  int tiles_per_split;
+  int n_kblk;               // key blocks per head (set by launch_colmax)
+  int nsplit;               // row-tile ranges per (head, key block) (set by launch_colmax)
+  int tiles_per_split;      // (set by launch_colmax)
   int32_t* status;
 };
 

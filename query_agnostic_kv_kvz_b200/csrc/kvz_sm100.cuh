@@ -185,6 +185,29 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of a K-major operand without swizzle whose
+// K extent is 16 bf16 (two 8x16-byte core matrices per 8-row group): the
+// second K core matrix sits 128 B after the first, 8-row groups are 256 B
+// apart.  Element (row r, col c) is at (r/8)*256 + (c/8)*128 + (r%8)*16 + (c%8)*2.
+__device__ __forceinline__ uint64_t sdesc_kmajor_k16_noswizzle(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);  // start address
+  d |= static_cast<uint64_t>(128 >> 4) << 16;         // leading byte offset: next K core matrix
+  d |= static_cast<uint64_t>(256 >> 4) << 32;         // stride byte offset: next 8-row group
+  d |= static_cast<uint64_t>(1) << 46;                // descriptor version (sm_100)
+  return d;                                           // layout type 0: no swizzle
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the
+// async proxy (TMA, tensor core).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Load 128 consecutive fp32 columns of this warp's 32 TMEM lanes (one lane
 // per thread) and wait for them.
 __device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {

@@ -1,4 +1,5 @@
-// KVzip context-reconstruction scoring on sm_100a (tcgen05 + TMEM + TMA).
+// KVzip context-reconstruction scoring on sm_100a (tcgen05 + TMEM + TMA):
+// pass 1 and shared launch helpers; pass 2 lives in colmax_kernel.cu.
 //
 // KVzip (analysis report, §3.2 "KV importance scoring", equation for S_{l,h}):
 //   A = Softmax(Q K^T) over the n_c + n_in keys of the repeat-prompt + context
@@ -56,24 +57,7 @@ struct LseLayout {
   static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;  // + alignment slack
 };
 
-template <int D>
-struct ColLayout {
-  static constexpr int KB = D / 64;
-  static constexpr int TILE_BYTES = KB * kSubBytes64;
-  static constexpr int NA = 2;                           // key tiles per CTA (256 keys)
-  static constexpr int QST = 4;                          // Q-tile pipeline depth
-  static constexpr int LST = 8;                          // lse2-slice ring depth
-  static constexpr int A_OFF = 0;
-  static constexpr int Q_OFF = A_OFF + NA * TILE_BYTES;
-  static constexpr int L_OFF = Q_OFF + QST * TILE_BYTES;  // lse2 slices, 128 floats each
-  static constexpr int BAR_OFF = L_OFF + LST * kTile * 4;
-  static constexpr int BAR_BYTES = 512;
-  static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;
-};
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
 
 // Descriptor of k-step `k` (16 bf16 of K) of a 128-row tile at `tile`.
 __device__ __forceinline__ uint64_t kstep_desc(const uint8_t* tile, int k) {
@@ -332,219 +316,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// ============================================================================
-// Pass 2: S[b, j] = max(S[b, j], 2^-(min_r lse2_r - c2 <q_r, k_j>)).
-// CTA = (head b, 256 context keys, a contiguous range of 128-row Q tiles).
-// Keys are the MMA's M side, so TMEM lane = key and each thread keeps the
-// running max of its key over the query-row columns in a register.
-// ============================================================================
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-    colmax_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
-                  ColArgs p) {
-  using Lay = ColLayout<D>;
-  const int u = blockIdx.x;
-  const int kblk = u % p.n_kblk;
-  const int rest = u / p.n_kblk;
-  const int sp = rest % p.nsplit;
-  const int b = rest / p.nsplit;
-  const int tpg = static_cast<int>(p.rows_pad / kTile);   // row tiles per group
-  const int T = p.G * tpg;
-  const int t_begin = sp * p.tiles_per_split;
-  const int t_end = min(T, t_begin + p.tiles_per_split);
-  const int ntile = t_end - t_begin;
-  if (ntile <= 0) return;                                  // uniform for the CTA
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint8_t* sA = smem + Lay::A_OFF;
-  uint8_t* sQ = smem + Lay::Q_OFF;
-  float* sL = reinterpret_cast<float*>(smem + Lay::L_OFF);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
-  uint64_t* a_full = bars + 0;
-  uint64_t* q_full = bars + 1;                   // [QST]
-  uint64_t* q_empty = q_full + Lay::QST;         // [QST]
-  uint64_t* l_full = q_empty + Lay::QST;         // [LST]
-  uint64_t* l_empty = l_full + Lay::LST;         // [LST]
-  uint64_t* acc_full = l_empty + Lay::LST;       // [2 key tiles][2 buffers]
-  uint64_t* acc_empty = acc_full + 4;            // [2][2]
-  uint64_t* drain = acc_empty + 4;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int64_t key0 = static_cast<int64_t>(kblk) * 256;
-
-  if (threadIdx.x == 0) {
-    mbar_init(a_full, 1);
-    for (int s = 0; s < Lay::QST; ++s) {
-      mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);                // freed by the MMA commit alone
-    }
-    for (int s = 0; s < Lay::LST; ++s) {
-      mbar_init(&l_full[s], 1);
-      mbar_init(&l_empty[s], 16);               // 16 epilogue warps read each slice
-    }
-    for (int s = 0; s < 4; ++s) {
-      mbar_init(&acc_full[s], 1);
-      mbar_init(&acc_empty[s], 8);              // 8 epilogue warps read each buffer
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 2) {
-    tmem_alloc(tmem_holder, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-
-  int issued = 0;     // Q tiles whose loads were issued (producer thread)
-  int l_issued = 0;   // lse2 slices whose loads were issued
-  if (warp == 0) {
-    if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmKc);
-      mbar_arrive_expect_tx(a_full, Lay::NA * Lay::TILE_BYTES);
-      for (int a = 0; a < Lay::NA; ++a)
-        for (int kb = 0; kb < Lay::KB; ++kb)
-          tma_load_3d(sA + a * Lay::TILE_BYTES + kb * kSubBytes64, &tmKc, a_full, kb * 64,
-                      static_cast<int>(key0 + a * kTile), b);
-      for (int n = 0; n < ntile; ++n) {
-        const int s = n % Lay::QST;
-        const uint32_t use = static_cast<uint32_t>(n / Lay::QST);
-        const int sl = n % Lay::LST;
-        const uint32_t luse = static_cast<uint32_t>(n / Lay::LST);
-        const int tau = t_begin + n;
-        const int g = tau / tpg;
-        const int il = (tau % tpg) * kTile;
-        const int bgq = b * p.G + g;
-        if (!mbar_wait(&q_empty[s], (use & 1u) ^ 1u, abort_flag, p.status)) break;
-        mbar_arrive_expect_tx(&q_full[s], Lay::TILE_BYTES);
-        for (int kb = 0; kb < Lay::KB; ++kb)
-          tma_load_3d(sQ + s * Lay::TILE_BYTES + kb * kSubBytes64, &tmQ, &q_full[s], kb * 64,
-                      static_cast<int>(p.i_begin + il), bgq);
-        issued = n + 1;
-        if (!mbar_wait(&l_empty[sl], (luse & 1u) ^ 1u, abort_flag, p.status)) break;
-        mbar_arrive_expect_tx(&l_full[sl], kTile * 4);
-        bulk_load(sL + sl * kTile, p.lse2 + static_cast<int64_t>(bgq) * p.ld + il, kTile * 4, &l_full[sl]);
-        l_issued = n + 1;
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-      bool ok = mbar_wait(a_full, 0, abort_flag, p.status);
-      tc_fence_after();
-      for (int n = 0; ok && n < ntile; ++n) {
-        const int s = n % Lay::QST;
-        const uint32_t use = static_cast<uint32_t>(n / Lay::QST);
-        if (!mbar_wait(&q_full[s], use & 1u, abort_flag, p.status)) break;
-        tc_fence_after();
-        const uint32_t buf = static_cast<uint32_t>(n) & 1u;
-        const uint32_t bu = static_cast<uint32_t>(n) >> 1;
-        for (int a = 0; a < Lay::NA; ++a) {
-          if (!mbar_wait(&acc_empty[a * 2 + buf], (bu & 1u) ^ 1u, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d_tmem = tmem + static_cast<uint32_t>((a * 2 + buf) * kTile);
-          const uint8_t* a_tile = sA + a * Lay::TILE_BYTES;
-          const uint8_t* b_tile = sQ + s * Lay::TILE_BYTES;
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k)
-            tc_mma_bf16(d_tmem, kstep_desc(a_tile, k), kstep_desc(b_tile, k), kIdesc, k > 0 ? 1u : 0u);
-          tc_commit(&acc_full[a * 2 + buf]);
-        }
-        if (!ok) break;
-        tc_commit(&q_empty[s]);
-      }
-    }
-    __syncwarp();
-  } else if (warp >= 4) {
-    // Four epilogue warpgroups: (key tile a, row half h).  A thread owns one
-    // context key (its TMEM lane) and 64 of the 128 query-row columns.
-    const int ew = warp - 4;
-    const int a = ew >> 3;
-    const int h = (ew >> 2) & 1;
-    const int wq = warp & 3;
-    const int64_t j = key0 + a * kTile + wq * 32 + lane;   // context key == TMEM lane
-    const float c2 = p.c2;
-    float ymin = INFINITY;     // min over rows of lse2_r - c2*<q_r, k_j>
-    bool ok = true;
-    for (int n = 0; n < ntile; ++n) {
-      const int sl = n % Lay::LST;
-      const uint32_t luse = static_cast<uint32_t>(n / Lay::LST);
-      const uint32_t buf = static_cast<uint32_t>(n) & 1u;
-      const uint32_t bu = static_cast<uint32_t>(n) >> 1;
-      if (!mbar_wait_warp(&acc_full[a * 2 + buf], bu & 1u, abort_flag, p.status)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float v[64];
-      tmem_ld64(tmem + (static_cast<uint32_t>(wq * 32) << 16) +
-                    static_cast<uint32_t>((a * 2 + buf) * kTile + h * 64), v);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[a * 2 + buf]);
-      if (!mbar_wait_warp(&l_full[sl], luse & 1u, abort_flag, p.status)) {
-        ok = false;
-        break;
-      }
-      // min over rows of lse2_r - c2*s (the negated exponent), two chains
-      const float4* L = reinterpret_cast<const float4*>(sL + sl * kTile + h * 64);
-      const float2 nc22 = make_float2(-c2, -c2);
-      float y0 = ymin, y1 = INFINITY;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float4 l4 = L[c];
-        const float2 ya = __ffma2_rn(make_float2(v[4 * c + 0], v[4 * c + 1]), nc22, make_float2(l4.x, l4.y));
-        const float2 yb = __ffma2_rn(make_float2(v[4 * c + 2], v[4 * c + 3]), nc22, make_float2(l4.z, l4.w));
-        y0 = fmin3(y0, ya.x, ya.y);
-        y1 = fmin3(y1, yb.x, yb.y);
-      }
-      ymin = fminf(y0, y1);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&l_empty[sl]);
-    }
-    if (ok && j < p.n_c) {
-      const float sj = exp2f(-ymin);   // >= +0, so its bit pattern orders like the value
-      atomicMax(reinterpret_cast<unsigned int*>(p.S + static_cast<int64_t>(b) * p.n_c + j), __float_as_uint(sj));
-    }
-  }
-
-  __syncthreads();
-  if (*abort_flag) {
-    if (warp == 0 && lane == 0) {
-      mbar_wait_for(a_full, 0, 20000000ull);
-      for (int s = 0; s < Lay::QST && s < issued; ++s) {
-        const int n_last = s + Lay::QST * ((issued - 1 - s) / Lay::QST);
-        mbar_wait_for(&q_full[s], static_cast<uint32_t>(n_last / Lay::QST) & 1u, 20000000ull);
-      }
-      for (int s = 0; s < Lay::LST && s < l_issued; ++s) {
-        const int n_last = s + Lay::LST * ((l_issued - 1 - s) / Lay::LST);
-        mbar_wait_for(&l_full[s], static_cast<uint32_t>(n_last / Lay::LST) & 1u, 20000000ull);
-      }
-    }
-    if (warp == 1 && lane == 0) {
-      tc_commit(drain);
-      mbar_wait_for(drain, 0, 20000000ull);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 2) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
 __global__ void fill_f32_kernel(float* x, int64_t n, float v) {
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x)
@@ -572,23 +343,6 @@ cudaError_t launch_lse(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, c
     e = set_smem(lse_kernel<64>, LseLayout<64>::SMEM);
     if (e != cudaSuccess) return e;
     lse_kernel<64><<<static_cast<unsigned>(grid), kThreads, LseLayout<64>::SMEM, stream>>>(tmQ, tmKc, tmKi, a);
-  }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_colmax(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, const ColArgs& a,
-                          cudaStream_t stream) {
-  const int64_t grid = static_cast<int64_t>(a.B) * a.nsplit * a.n_kblk;
-  if (grid <= 0 || grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
-  cudaError_t e;
-  if (d == 128) {
-    e = set_smem(colmax_kernel<128>, ColLayout<128>::SMEM);
-    if (e != cudaSuccess) return e;
-    colmax_kernel<128><<<static_cast<unsigned>(grid), kThreads, ColLayout<128>::SMEM, stream>>>(tmQ, tmKc, a);
-  } else {
-    e = set_smem(colmax_kernel<64>, ColLayout<64>::SMEM);
-    if (e != cudaSuccess) return e;
-    colmax_kernel<64><<<static_cast<unsigned>(grid), kThreads, ColLayout<64>::SMEM, stream>>>(tmQ, tmKc, a);
   }
   return cudaGetLastError();
 }
