@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--impl", default="kvz", choices=["kvz", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="llama8b_layer (default, the headline), tiny, llama8b_stack, qwen14b_128k, stress_ragged")
     return ap.parse_args()
 
 
@@ -134,21 +136,22 @@ class ClockSampler:
 
 
 def workload_numbers(w):
-    B, G, d, n_c = w.B, w.G, w.d, w.n_c[0]
-    n_in = w.n_in(0)
-    vis = B * G * (n_in * n_c + n_in * (n_in + 1) // 2)          # pass 1 pairs
-    ctx = B * G * n_in * n_c                                       # pass 2 pairs
-    k = int(math.floor(w.ratio * n_c))
-    kept = B * k
-    return {
-        "pairs_per_step": B * n_c,
-        "flops_pass1": 2 * d * vis,
-        "flops_pass2": 2 * d * ctx,
-        "flops_algorithmic": 2 * d * vis,
-        "kept": kept,
-        "compact_bytes": kept * d * 2 * 2 * 2 + 4 * kept,
-        "select_bytes": 5 * 4 * B * n_c,
-    }
+    """Per-step work units of a workload, summed over its contexts."""
+    B, G, d = w.B, w.G, w.d
+    out = {"pairs_per_step": 0, "flops_pass1": 0, "flops_pass2": 0, "kept": 0, "select_bytes": 0}
+    for c, n_c in enumerate(w.n_c):
+        n_in = w.n_in(c)
+        vis = B * G * (n_in * n_c + n_in * (n_in + 1) // 2)          # pass 1 pairs
+        ctx = B * G * n_in * n_c                                       # pass 2 pairs
+        kept = int(math.floor(w.ratio * B * n_c)) if w.mode == "global" else B * int(math.floor(w.ratio * n_c))
+        out["pairs_per_step"] += B * n_c
+        out["flops_pass1"] += 2 * d * vis
+        out["flops_pass2"] += 2 * d * ctx
+        out["kept"] += kept
+        out["select_bytes"] += 5 * 4 * B * n_c
+    out["flops_algorithmic"] = out["flops_pass1"]
+    out["compact_bytes"] = out["kept"] * d * 2 * 2 * 2 + 4 * out["kept"]
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -194,12 +197,14 @@ def main():
     torch.cuda.set_device(dev)
 
     from query_agnostic_kv_kvz_b200 import synth
-    w = synth.WORKLOADS[WORKLOAD]
+    w = synth.WORKLOADS[args.workload]
     nums = workload_numbers(w)
-    config = {"workload": "%s (L=%d, H=%d, G=%d, d=%d, n_c=%d, n_prompt=%d, keep %.2f %s)" % (
-        w.name, w.L, w.H, w.G, w.d, w.n_c[0], w.n_prompt, w.ratio, w.mode),
-        "B_heads": w.B, "G": w.G, "d": w.d, "n_c": w.n_c[0], "n_in": w.n_in(0), "ratio": w.ratio,
-        "mode": w.mode, "l2": "flushed before every timed step (256 MB write, outside the timed events)",
+    config = {"workload": "%s (L=%d, H=%d, G=%d, d=%d, n_c=%s, n_prompt=%d, keep %.2f %s%s%s)" % (
+        w.name, w.L, w.H, w.G, w.d, "/".join(str(n) for n in w.n_c), w.n_prompt, w.ratio, w.mode,
+        ", rows in chunks of %d" % w.row_chunk if w.row_chunk else "", ", in-place compaction" if w.in_place else ""),
+        "B_heads": w.B, "G": w.G, "d": w.d, "n_c": list(w.n_c), "n_in": [w.n_in(c) for c in range(len(w.n_c))],
+        "ratio": w.ratio, "mode": w.mode,
+        "l2": "flushed before every timed step (256 MB write, outside the timed events)",
         "parallelism": "replicas (weak)" if world > 1 else "single GPU"}
 
     if args.impl == "reference":
@@ -233,111 +238,129 @@ def main():
     import query_agnostic_kv_kvz_b200 as kvz
     from query_agnostic_kv_kvz_b200.dist import max_over_ranks, rank_seed
     kvz.lib()
-    x = synth.layer_inputs(w, seed=rank_seed(0, rank), device=dev)
-    B, G, d, n_c, n_in = w.B, w.G, w.d, w.n_c[0], w.n_in(0)
-    scale = float(1.0 / math.sqrt(d))
     stream = torch.cuda.current_stream(dev)
-    rows_pad = (n_in + 255) // 256 * 256
-    lse2 = torch.empty((B, G, rows_pad), dtype=torch.float32, device=dev)
-    S = torch.empty((B, n_c), dtype=torch.float32, device=dev)
-    k = kvz.kvz_keep_count(n_c, w.ratio)
-    idx = torch.empty(B * k, dtype=torch.int32, device=dev)
-    counts = torch.empty(B, dtype=torch.int32, device=dev)
-    offsets = torch.empty(B + 1, dtype=torch.int64, device=dev)
-    sel_ws = torch.empty(kvz.kvz_select_workspace_size(B, n_c, kvz.PER_HEAD), dtype=torch.uint8, device=dev)
-    K_out = torch.empty((B * k, d), dtype=torch.bfloat16, device=dev)
-    V_out = torch.empty((B * k, d), dtype=torch.bfloat16, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    scale = float(1.0 / math.sqrt(w.d))
+    ctxs = [Context(w, c, rank_seed(0, rank), dev, kvz) for c in range(len(w.n_c))]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    launches_per_step = 3 + 10 + 1      # lse, fill, colmax | select: init, 3x(hist, pick), count, scan, write | compact
+    launches_per_step = sum(c.launches for c in ctxs)
 
     def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        kvz.kvz_score_lse2(x["Q"], x["K_ctx"], x["K_in"], scale=scale, lse2=lse2, status=status, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
-        kvz.kvz_score_colmax(x["Q"], x["K_ctx"], lse2, scale=scale, S=S, accumulate=False, status=status,
-                             stream=stream)
-        if ev is not None:
-            ev[2].record(stream)
-        kvz.kvz_select(S, w.ratio, w.mode, idx=idx, counts=counts, offsets=offsets, workspace=sel_ws,
-                       status=status, stream=stream)
-        if ev is not None:
-            ev[3].record(stream)
-        kvz.kvz_compact(x["K_ctx"], x["V"], idx, counts, offsets, K_out=K_out, V_out=V_out, status=status,
-                        stream=stream)
-        if ev is not None:
-            ev[4].record(stream)
+        """One pass of the whole path over the workload; with `ev`, returns the
+        device time (ms) of pass 1, pass 2, selection and compaction."""
+        marks = []
+        def mark(tag):
+            if ev is not None:
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(stream)
+                marks.append((tag, e))
+        for c in ctxs:
+            H = w.H
+            for l in range(w.L):
+                Kl = c.K[l * H:(l + 1) * H]
+                Sl = c.S[l * H:(l + 1) * H]
+                for (i0, i1) in c.chunks:
+                    mark("p1")
+                    kvz.kvz_score_lse2(c.Q[l], Kl, c.Kin[l], i_begin=i0, i_end=i1, scale=scale, lse2=c.lse2,
+                                       ld=c.ld, status=status, stream=stream)
+                    mark("p2")
+                    kvz.kvz_score_colmax(c.Q[l], Kl, c.lse2, i_begin=i0, i_end=i1, scale=scale, S=Sl,
+                                         accumulate=i0 > 0, status=status, stream=stream)
+                    mark("end")
+            mark("sel")
+            kvz.kvz_select(c.S, w.ratio, w.mode, idx=c.idx, counts=c.counts, offsets=c.offsets,
+                           workspace=c.sel_ws, status=status, stream=stream)
+            mark("cmp")
+            if w.in_place:
+                kvz.kvz_compact(c.K, c.V, c.idx, c.counts, c.offsets, in_place=True, status=status, stream=stream)
+            else:
+                kvz.kvz_compact(c.K, c.V, c.idx, c.counts, c.offsets, K_out=c.K_out, V_out=c.V_out,
+                                status=status, stream=stream)
+            mark("end")
+        return marks
 
-    for _ in range(max(3, args.warmup)):
+    def phase_ms(marks):
+        acc = {"p1": 0.0, "p2": 0.0, "sel": 0.0, "cmp": 0.0}
+        for (tag, e0), (_, e1) in zip(marks, marks[1:]):
+            if tag in acc:
+                acc[tag] += e0.elapsed_time(e1)
+        return [acc["p1"], acc["p2"], acc["sel"], acc["cmp"]]
+
+    # the headline workload always gets >= 3 warm-up steps; the large ones
+    # (tens of seconds per step) take what the caller asks for
+    n_warm = max(3, args.warmup) if w.name == WORKLOAD else max(1, args.warmup)
+    for _ in range(n_warm):
         flush.zero_()
         step()
     torch.cuda.synchronize(dev)
     if int(status.item()) != 0:
         raise RuntimeError("device status %d during warm-up" % int(status.item()))
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
+    all_marks = []
     with ClockSampler(dev.index) as clk:
-        for s in range(args.steps):
+        for s_ in range(args.steps):
             flush.zero_()
-            step(evs[s])
+            all_marks.append(step(ev=True))
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    parts = [[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs]
-    tot = [sum(p) for p in parts]
-    ms_step = sum(tot) / len(tot)
+    parts = [phase_ms(m) for m in all_marks]
+    ms_step = sum(sum(p) for p in parts) / len(parts)
     part_ms = [sum(p[i] for p in parts) / len(parts) for i in range(4)]
     if int(status.item()) != 0:
         raise RuntimeError("device status %d during timing" % int(status.item()))
 
     # ---- end to end through host buffers (pinned), copies inside the timed region
-    hx = {n: t.cpu().pin_memory() for n, t in x.items()}
-    dx = {n: torch.empty_like(t) for n, t in x.items()}
-    h_out = {"K": torch.empty((B * k, d), dtype=torch.bfloat16).pin_memory(),
-             "V": torch.empty((B * k, d), dtype=torch.bfloat16).pin_memory(),
-             "idx": torch.empty(B * k, dtype=torch.int32).pin_memory(),
-             "counts": torch.empty(B, dtype=torch.int32).pin_memory(),
-             "offsets": torch.empty(B + 1, dtype=torch.int64).pin_memory()}
-    ws_score = torch.empty(kvz.kvz_score_workspace_size(B, G, n_in, 0), dtype=torch.uint8, device=dev)
-    h2d = sum(t.numel() * t.element_size() for t in hx.values())
-    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    e2e = None
+    if len(ctxs) == 1 and w.L == 1 and not w.in_place:
+        c = ctxs[0]
+        hx = {"Q": c.Q[0].cpu().pin_memory(), "K_ctx": c.K.cpu().pin_memory(), "K_in": c.Kin[0].cpu().pin_memory(),
+              "V": c.V.cpu().pin_memory()}
+        dx = {n: torch.empty_like(t, device=dev) for n, t in hx.items()}
+        h_out = {"K": torch.empty_like(c.K_out, device="cpu").pin_memory(),
+                 "V": torch.empty_like(c.V_out, device="cpu").pin_memory(),
+                 "idx": torch.empty_like(c.idx, device="cpu").pin_memory(),
+                 "counts": torch.empty_like(c.counts, device="cpu").pin_memory(),
+                 "offsets": torch.empty_like(c.offsets, device="cpu").pin_memory()}
+        ws_score = torch.empty(kvz.kvz_score_workspace_size(w.H, w.G, c.n_in, 0), dtype=torch.uint8, device=dev)
+        h2d = sum(t.numel() * t.element_size() for t in hx.values())
+        d2h = sum(t.numel() * t.element_size() for t in h_out.values())
 
-    def e2e_step():
-        for n in dx:
-            dx[n].copy_(hx[n], non_blocking=True)
-        kvz.kvz_score(dx["Q"], dx["K_ctx"], dx["K_in"], scale=scale, S=S, workspace=ws_score, status=status,
-                      stream=stream)
-        kvz.kvz_select(S, w.ratio, w.mode, idx=idx, counts=counts, offsets=offsets, workspace=sel_ws,
-                       status=status, stream=stream)
-        kvz.kvz_compact(dx["K_ctx"], dx["V"], idx, counts, offsets, K_out=K_out, V_out=V_out, status=status,
-                        stream=stream)
-        h_out["K"].copy_(K_out, non_blocking=True)
-        h_out["V"].copy_(V_out, non_blocking=True)
-        h_out["idx"].copy_(idx, non_blocking=True)
-        h_out["counts"].copy_(counts, non_blocking=True)
-        h_out["offsets"].copy_(offsets, non_blocking=True)
+        def e2e_step():
+            for n in dx:
+                dx[n].copy_(hx[n], non_blocking=True)
+            kvz.kvz_score(dx["Q"], dx["K_ctx"], dx["K_in"], scale=scale, S=c.S, workspace=ws_score, status=status,
+                          stream=stream)
+            kvz.kvz_select(c.S, w.ratio, w.mode, idx=c.idx, counts=c.counts, offsets=c.offsets,
+                           workspace=c.sel_ws, status=status, stream=stream)
+            kvz.kvz_compact(dx["K_ctx"], dx["V"], c.idx, c.counts, c.offsets, K_out=c.K_out, V_out=c.V_out,
+                            status=status, stream=stream)
+            h_out["K"].copy_(c.K_out, non_blocking=True)
+            h_out["V"].copy_(c.V_out, non_blocking=True)
+            h_out["idx"].copy_(c.idx, non_blocking=True)
+            h_out["counts"].copy_(c.counts, non_blocking=True)
+            h_out["offsets"].copy_(c.offsets, non_blocking=True)
 
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if int(status.item()) != 0:
-        raise RuntimeError("device status %d during e2e" % int(status.item()))
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if int(status.item()) != 0:
+            raise RuntimeError("device status %d during e2e" % int(status.item()))
+        e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
 
-    red = max_over_ranks([ms_step, e2e_ms] + part_ms, device=dev)
+    red = max_over_ranks([ms_step, e2e["ms"] if e2e else 0.0] + part_ms, device=dev)
     ms_step, e2e_ms, part_ms = red[0], red[1], red[2:]
 
     pk = peaks()
@@ -345,6 +368,7 @@ def main():
     score_ms = lse_ms + col_ms
     fl1, fl2 = nums["flops_pass1"], nums["flops_pass2"]
     tf = lambda flops, ms: flops / (ms * 1e-3) / 1e12
+    n_p1 = sum(w.L * len(c.chunks) for c in ctxs)
     roof = {
         "bound": "tensor",
         "kernel": "lse_kernel (score pass 1: QK^T + online log-sum-exp)",
@@ -352,9 +376,10 @@ def main():
         "peak": pk["bf16_tflops"],
         "unit": "TFLOP/s",
         "frac": tf(fl1, lse_ms) / pk["bf16_tflops"],
-        "traffic": recorded_traffic("lse_kernel"),
+        "traffic": recorded_traffic("lse_kernel") if w.name == WORKLOAD else None,
         "peak_source": "%s bf16 dense (burst)" % pk["source"],
-        "algorithmic_flops_per_launch": fl1,
+        "algorithmic_flops_per_launch": fl1 / n_p1,
+        "launches_per_step": n_p1,
         "breakdown": {
             "score_pass1_ms": lse_ms, "score_pass2_ms": col_ms, "select_ms": sel_ms, "compact_ms": cmp_ms,
             "score_tflops_executed": tf(fl1 + fl2, score_ms),
@@ -362,6 +387,7 @@ def main():
             "score_tflops_algorithmic": tf(nums["flops_algorithmic"], score_ms),
             "score_frac_algorithmic": tf(nums["flops_algorithmic"], score_ms) / pk["bf16_tflops"],
             "pass2_tflops": tf(fl2, col_ms), "pass2_frac": tf(fl2, col_ms) / pk["bf16_tflops"],
+            "compact_bytes": nums["compact_bytes"],
             "compact_gbs": nums["compact_bytes"] / (cmp_ms * 1e-3) / 1e9,
             "compact_frac_hbm": nums["compact_bytes"] / (cmp_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
             "select_gbs": nums["select_bytes"] / (sel_ms * 1e-3) / 1e9,
@@ -370,23 +396,65 @@ def main():
     value = nums["pairs_per_step"] * world / (ms_step * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": n_warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config, "roofline": roof,
-        "e2e": {"value": nums["pairs_per_step"] * world / (e2e_ms * 1e-3), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, threads = oracle_head_time(x, w, 0)
-        line["cpu_baseline"] = {"value": n_c / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+    if e2e is not None:
+        line["e2e"] = {"value": nums["pairs_per_step"] * world / (e2e_ms * 1e-3), "unit": UNIT,
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and w.name == WORKLOAD:
+        c = ctxs[0]
+        x0 = {"Q": c.Q[0], "K_ctx": c.K[: w.H], "K_in": c.Kin[0], "V": c.V[: w.H]}
+        dt, threads = oracle_head_time(x0, w, 0)
+        line["cpu_baseline"] = {"value": c.n_c / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": "head 0 of the %d-head layer: fp64 score + select + compact "
-                                          "(%.1f s)" % (B, dt)}
+                                          "(%.1f s)" % (w.B, dt)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+class Context:
+    """Device-resident inputs and outputs of one context of a workload: all
+    layers' Q / K_in, the whole K/V cache, scores, selection and outputs."""
+
+    def __init__(self, w, c, seed, dev, kvz):
+        import torch
+        from query_agnostic_kv_kvz_b200 import synth
+        H, G, d, L = w.H, w.G, w.d, w.L
+        B = L * H
+        self.n_c, self.n_in = w.n_c[c], w.n_in(c)
+        self.K = torch.empty((B, self.n_c, d), dtype=torch.bfloat16, device=dev)
+        self.V = torch.empty((B, self.n_c, d), dtype=torch.bfloat16, device=dev)
+        self.Q, self.Kin = [], []
+        for l in range(L):
+            x = synth.layer_inputs(w, layer=l, ctx=c, seed=seed, device=dev)
+            self.K[l * H:(l + 1) * H].copy_(x["K_ctx"])
+            self.V[l * H:(l + 1) * H].copy_(x["V"])
+            self.Q.append(x["Q"])
+            self.Kin.append(x["K_in"])
+            del x
+        chunk = min(w.row_chunk or self.n_in, self.n_in)
+        self.chunks = [(i0, min(self.n_in, i0 + chunk)) for i0 in range(0, self.n_in, chunk)]
+        self.ld = (chunk + 255) // 256 * 256
+        self.lse2 = torch.empty((H, G, self.ld), dtype=torch.float32, device=dev)
+        self.S = torch.empty((B, self.n_c), dtype=torch.float32, device=dev)
+        mode = kvz.GLOBAL if w.mode == "global" else kvz.PER_HEAD
+        k = kvz.kvz_keep_count(B * self.n_c if mode == kvz.GLOBAL else self.n_c, w.ratio)
+        cap = max(1, k if mode == kvz.GLOBAL else B * k)
+        self.idx = torch.empty(cap, dtype=torch.int32, device=dev)
+        self.counts = torch.empty(B, dtype=torch.int32, device=dev)
+        self.offsets = torch.empty(B + 1, dtype=torch.int64, device=dev)
+        self.sel_ws = torch.empty(kvz.kvz_select_workspace_size(B, self.n_c, mode), dtype=torch.uint8, device=dev)
+        if not w.in_place:
+            self.K_out = torch.empty((cap, d), dtype=torch.bfloat16, device=dev)
+            self.V_out = torch.empty((cap, d), dtype=torch.bfloat16, device=dev)
+        # lse (+ colmax, + S fill on the first chunk) per (layer, chunk); select 10; compact 1
+        self.launches = L * (2 * len(self.chunks) + 1) + 10 + 1
 
 
 if __name__ == "__main__":

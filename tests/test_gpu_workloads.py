@@ -1,0 +1,202 @@
+"""Full-size workloads on the GPU (through the C ABI), checked against the
+oracle where it can run and by properties that hold at any size elsewhere:
+
+* every workload: selection bit-exact against the oracle's stable sort on the
+  GPU's own scores (all heads); compaction bit-exact on sampled heads;
+* pass 1 (lse2) against the oracle on sampled rows of sampled heads;
+* S[j] >= A[r, j] for every key j and every sampled row r (oracle rows);
+* planted dominant keys: S[j*] equals one oracle row value A[r*, j*];
+* the 1000-key context of the ragged batch: every score of every head
+  against the oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from kvz_testutil import ABS_TOL, REL_FLOOR, REL_TOL, assert_scores_close, bits, f32_scale, f64, oracle_scores
+from oracle import kvz_oracle as orc
+from query_agnostic_kv_kvz_b200 import synth
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+kvz = pytest.importorskip("query_agnostic_kv_kvz_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    kvz.lib()
+    yield
+    torch.cuda.empty_cache()
+
+
+def run_path(w, ctx=0, keep_layers=(0,), plant=None, in_place=None):
+    """Score every layer, select over the whole call, compact.  Returns a
+    dict with S, the selection, compaction outputs and the kept layers'
+    inputs (for oracle checks)."""
+    dev = "cuda"
+    H, G, d = w.H, w.G, w.d
+    n_c, n_in = w.n_c[ctx], w.n_in(ctx)
+    B = w.L * H
+    scale = f32_scale(d)
+    K_ctx = torch.empty((B, n_c, d), dtype=torch.bfloat16, device=dev)
+    V = torch.empty((B, n_c, d), dtype=torch.bfloat16, device=dev)
+    S = torch.empty((B, n_c), dtype=torch.float32, device=dev)
+    ws = torch.empty(kvz.kvz_score_workspace_size(H, G, n_in, w.row_chunk), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    kept = {}
+    for l in range(w.L):
+        x = synth.layer_inputs(w, layer=l, ctx=ctx, device=dev)
+        if plant is not None and l == 0:
+            plant(x)
+        K_ctx[l * H:(l + 1) * H] = x["K_ctx"]
+        V[l * H:(l + 1) * H] = x["V"]
+        kvz.kvz_score(x["Q"], K_ctx[l * H:(l + 1) * H], x["K_in"], scale=scale, row_chunk=w.row_chunk,
+                      S=S[l * H:(l + 1) * H], workspace=ws, status=status)
+        if l in keep_layers:
+            kept[l] = x
+        else:
+            del x
+    idx, counts, offsets = kvz.kvz_select(S, w.ratio, w.mode, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return {"S": S, "K": K_ctx, "V": V, "idx": idx, "counts": counts, "offsets": offsets, "kept": kept,
+            "scale": scale, "n_c": n_c, "n_in": n_in, "B": B}
+
+
+def check_selection(r, w):
+    S_np = r["S"].cpu().numpy()
+    assert np.all(S_np >= 0) and np.all(S_np <= 1.0 + 1e-4)
+    ri, rc, ro = orc.select(S_np, w.ratio, w.mode)
+    np.testing.assert_array_equal(r["counts"].cpu().numpy(), rc)
+    np.testing.assert_array_equal(r["offsets"].cpu().numpy(), ro)
+    np.testing.assert_array_equal(r["idx"].cpu().numpy()[: len(ri)], ri)
+    return ri, rc, ro
+
+
+def check_compaction(r, sel, heads, in_place):
+    ri, rc, ro = sel
+    if in_place:
+        Kh = {b: bits(r["K"][b]) for b in heads}
+        Vh = {b: bits(r["V"][b]) for b in heads}
+        kvz.kvz_compact(r["K"], r["V"], r["idx"], r["counts"], r["offsets"], in_place=True)
+        torch.cuda.synchronize()
+        for b in heads:
+            c = int(rc[b])
+            sel_b = ri[ro[b]:ro[b + 1]]
+            np.testing.assert_array_equal(bits(r["K"][b, :c]), Kh[b][sel_b])
+            np.testing.assert_array_equal(bits(r["V"][b, :c]), Vh[b][sel_b])
+    else:
+        total = int(ro[-1])
+        K_out, V_out = kvz.kvz_compact(r["K"], r["V"], r["idx"], r["counts"], r["offsets"], out_rows=max(total, 1))
+        torch.cuda.synchronize()
+        for b in heads:
+            sel_b = ri[ro[b]:ro[b + 1]]
+            np.testing.assert_array_equal(bits(K_out[ro[b]:ro[b + 1]]), bits(r["K"][b])[sel_b])
+            np.testing.assert_array_equal(bits(V_out[ro[b]:ro[b + 1]]), bits(r["V"][b])[sel_b])
+
+
+def sampled_rows(n_in, n_prompt, rng, k=6):
+    base = {0, 1, max(0, n_prompt - 1), n_prompt, n_in // 2, n_in - 1}
+    return sorted(base | set(rng.integers(0, n_in, size=k).tolist()))
+
+
+def check_sampled_rows(r, w, layer, head, rows, groups):
+    """pass-1 lse2 on sampled rows vs the oracle, and S >= those rows' A."""
+    x = r["kept"][layer]
+    H, G = w.H, w.G
+    b = layer * H + head
+    scale = r["scale"]
+    Qh = f64(x["Q"][head])
+    Kc = f64(x["K_ctx"][head])
+    Ki = f64(x["K_in"][head])
+    S_b = r["S"][b].double().cpu().numpy()
+    n_in = r["n_in"]
+    chunk = w.row_chunk or n_in
+    for i0 in sorted({(i // chunk) * chunk for i in rows}):
+        i1 = min(n_in, i0 + chunk)
+        lse2 = kvz.kvz_score_lse2(x["Q"], x["K_ctx"], x["K_in"], i_begin=i0, i_end=i1, scale=scale)
+        lse2 = lse2.cpu().numpy()
+        for g in groups:
+            for i in rows:
+                if not (i0 <= i < i1):
+                    continue
+                lse = orc.row_lse(Qh[g, i], Kc, Ki, i, scale)
+                assert abs(lse2[head, g, i - i0] * math.log(2) - lse) <= 2e-4 * math.log(2) * 2, (g, i)
+                A = np.exp(orc.row_logits(Qh[g, i], Kc, Ki, i, scale)[: r["n_c"]] - lse)
+                gap = A - S_b
+                assert gap.max() <= ABS_TOL, (g, i, gap.max())
+                big = A > REL_FLOOR
+                if big.any():
+                    assert (gap[big] / A[big]).max() <= REL_TOL
+
+
+def planter(rows_keys, alpha=1.8):
+    """Make context key j of head 0 an enlarged copy of query row (g, i)."""
+    def plant(x):
+        for (g, i, j) in rows_keys:
+            x["K_ctx"][0, j] = (alpha * x["Q"][0, g, i].float()).to(torch.bfloat16)
+    return plant
+
+
+def check_planted(r, rows_keys):
+    x = r["kept"][0]
+    Qh, Kc, Ki = f64(x["Q"][0]), f64(x["K_ctx"][0]), f64(x["K_in"][0])
+    S0 = r["S"][0].double().cpu().numpy()
+    for (g, i, j) in rows_keys:
+        z = orc.row_logits(Qh[g, i], Kc, Ki, i, r["scale"])
+        A = math.exp(z[j] - orc.row_lse(Qh[g, i], Kc, Ki, i, r["scale"]))
+        assert A > 0.5, "planted key does not dominate its row"
+        assert abs(S0[j] - A) <= ABS_TOL and abs(S0[j] - A) <= REL_TOL * A, (g, i, j, S0[j], A)
+
+
+# ---------------------------------------------------------------------------
+def test_llama8b_stack_32k_global():
+    w = synth.WORKLOADS["llama8b_stack"]
+    rng = np.random.default_rng(3)
+    plant = [(0, 5, 100), (3, 20000, 31000), (1, 32799, 7)]
+    r = run_path(w, keep_layers=(0, 31), plant=planter(plant))
+    check_planted(r, plant)
+    sel = check_selection(r, w)
+    check_compaction(r, sel, heads=[0, 7, 100, 255], in_place=False)
+    rows = sampled_rows(r["n_in"], w.n_prompt, rng)
+    check_sampled_rows(r, w, layer=0, head=3, rows=rows, groups=[0, 3])
+    check_sampled_rows(r, w, layer=31, head=7, rows=rows, groups=[1])
+
+
+def test_qwen14b_128k_row_chunks_in_place():
+    w = synth.WORKLOADS["qwen14b_128k"]
+    rng = np.random.default_rng(4)
+    plant = [(0, 3, 5), (4, 70000, 131071), (2, 131103, 65536)]
+    r = run_path(w, keep_layers=(0, 47), plant=planter(plant))
+    check_planted(r, plant)
+    sel = check_selection(r, w)
+    rows = sampled_rows(r["n_in"], w.n_prompt, rng, k=4)
+    check_sampled_rows(r, w, layer=0, head=1, rows=rows, groups=[0, 4])
+    check_sampled_rows(r, w, layer=47, head=6, rows=rows[:6], groups=[2])
+    check_compaction(r, sel, heads=[0, 1, 200, 383], in_place=True)
+
+
+@pytest.mark.parametrize("ctx", [0, 1, 2, 3])
+def test_stress_ragged_context(ctx):
+    w = synth.WORKLOADS["stress_ragged"]
+    rng = np.random.default_rng(10 + ctx)
+    n_c = w.n_c[ctx]
+    r = run_path(w, ctx=ctx, keep_layers=(0, 31) if ctx == 0 else (0,))
+    sel = check_selection(r, w)
+    S_np = r["S"].cpu().numpy()
+    ties = int(S_np.size - len(np.unique(S_np)))
+    assert ties > 0                                  # duplicated keys produce exact ties
+    check_compaction(r, sel, heads=[0, 255, int(rng.integers(1, 255))], in_place=False)
+    if ctx == 0:
+        # n_c = 1000: every score of every head against the oracle (layers kept: 0 and 31)
+        for layer in (0, 31):
+            x = r["kept"][layer]
+            ref = oracle_scores(x["Q"], x["K_ctx"], x["K_in"], r["scale"])
+            assert_scores_close(r["S"][layer * w.H:(layer + 1) * w.H].cpu().numpy(), ref, "ctx0 layer %d" % layer)
+    else:
+        rows = sampled_rows(r["n_in"], w.n_prompt, rng, k=3)
+        check_sampled_rows(r, w, layer=0, head=int(rng.integers(0, w.H)), rows=rows, groups=[0, 3])
