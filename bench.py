@@ -272,7 +272,8 @@ def main():
                            workspace=c.sel_ws, status=status, stream=stream)
             mark("cmp")
             if w.in_place:
-                kvz.kvz_compact(c.K, c.V, c.idx, c.counts, c.offsets, in_place=True, status=status, stream=stream)
+                kvz.kvz_compact(c.K, c.V, c.idx, c.counts, c.offsets, in_place=True, workspace=c.cmp_ws,
+                                status=status, stream=stream)
             else:
                 kvz.kvz_compact(c.K, c.V, c.idx, c.counts, c.offsets, K_out=c.K_out, V_out=c.V_out,
                                 status=status, stream=stream)
@@ -450,6 +451,7 @@ class Context:
         self.counts = torch.empty(B, dtype=torch.int32, device=dev)
         self.offsets = torch.empty(B + 1, dtype=torch.int64, device=dev)
         self.sel_ws = torch.empty(kvz.kvz_select_workspace_size(B, self.n_c, mode), dtype=torch.uint8, device=dev)
+        self.cmp_ws = torch.empty(kvz.kvz_compact_workspace_size(B, self.n_c), dtype=torch.uint8, device=dev)
         if not w.in_place:
             self.K_out = torch.empty((cap, d), dtype=torch.bfloat16, device=dev)
             self.V_out = torch.empty((cap, d), dtype=torch.bfloat16, device=dev)

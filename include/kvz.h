@@ -214,17 +214,29 @@ kvz_status kvz_select(const float* S, int64_t B, int64_t n_c, double ratio,
 /*                                                                          */
 /* Out of place (K_out != K): dst_b = out_offsets[b] if out_offsets is not   */
 /*   NULL, else offsets[b] (a packed CSR cache).  K_out/V_out must hold every */
-/*   destination row and must not overlap K or V.                             */
+/*   destination row and must not overlap K or V.  No workspace is needed   */
+/*   (workspace may be NULL).                                                */
 /* In place (K_out == K and V_out == V): dst_b = b*n_c, i.e. each head's     */
 /*   kept rows are packed to the front of its own region; rows at and after  */
-/*   counts[b] keep stale data.  out_offsets must be NULL.  Safe because a    */
-/*   kept row never moves to a higher position.                               */
+/*   counts[b] keep stale data.  out_offsets must be NULL.  Needs a          */
+/*   workspace of kvz_compact_workspace_size(B, n_c) bytes (chunk claims,   */
+/*   "sources read" flags and each chunk's first reader slot, all rebuilt by */
+/*   the call).  Safe because a kept row never moves to a higher position: a */
+/*   chunk of slots writes only after every earlier chunk that reads one of  */
+/*   its destination rows has read (a bounded wait; if it ever expires,      */
+/*   KVZ_ERR_TIMEOUT is set and that head's remaining chunks are left        */
+/*   unwritten).                                                             */
 /* Layout: K, V [B][n_c][d] bf16; idx/counts/offsets as kvz_select writes.   */
+/* Device-detected errors: idx out of [0, n_c), or idx[p] < p in place       */
+/* (not ascending) -> KVZ_ERR_INVALID_ARG, the offending slot is skipped.    */
 /* ------------------------------------------------------------------------ */
+size_t kvz_compact_workspace_size(int64_t B, int64_t n_c);
+
 kvz_status kvz_compact(const void* K, const void* V, int64_t B, int64_t n_c,
                        int d, const int32_t* idx, const int32_t* counts,
                        const int64_t* offsets, const int64_t* out_offsets,
                        void* K_out, void* V_out,
+                       void* workspace, size_t workspace_bytes,
                        int32_t* d_status, cudaStream_t stream);
 
 #ifdef __cplusplus

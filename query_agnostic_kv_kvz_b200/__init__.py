@@ -19,7 +19,7 @@ __all__ = [
     "KvzError", "KvzLibraryError", "lib", "lib_path", "STATUS",
     "kvz_version", "kvz_keep_count",
     "kvz_score_workspace_size", "kvz_score", "kvz_score_lse2", "kvz_score_colmax",
-    "kvz_select_workspace_size", "kvz_select", "kvz_compact",
+    "kvz_select_workspace_size", "kvz_select", "kvz_compact_workspace_size", "kvz_compact",
     "PER_HEAD", "GLOBAL",
 ]
 
@@ -63,7 +63,8 @@ _SIGS = {
     "kvz_keep_count": (_i64, [_i64, _f64]),
     "kvz_select_workspace_size": (_sz, [_i64, _i64, _i32]),
     "kvz_select": (_i32, [_vp, _i64, _i64, _f64, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
-    "kvz_compact": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "kvz_compact_workspace_size": (_sz, [_i64, _i64]),
+    "kvz_compact": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
 }
 
 
@@ -238,8 +239,12 @@ def kvz_select(S, ratio: float, mode="per_head", idx=None, counts=None, offsets=
     return idx, counts, offsets
 
 
+def kvz_compact_workspace_size(B: int, n_c: int) -> int:
+    return lib().kvz_compact_workspace_size(B, n_c)
+
+
 def kvz_compact(K, V, idx, counts, offsets, out_offsets=None, K_out=None, V_out=None, in_place: bool = False,
-                out_rows: Optional[int] = None, status=None, stream=None):
+                out_rows: Optional[int] = None, workspace=None, status=None, stream=None):
     """Gather kept rows in key order (KVzip §2.1 pruned cache); returns (K_out, V_out).
 
     Out of place, the outputs are [rows, d] with head b's rows starting at
@@ -247,19 +252,22 @@ def kvz_compact(K, V, idx, counts, offsets, out_offsets=None, K_out=None, V_out=
     outputs (default B*n_c, an upper bound).  In place, K and V themselves
     are returned, each head's kept rows packed to the front of its region.
     """
-    _need_cuda(K, V, idx, counts, offsets, out_offsets, K_out, V_out, status)
+    _need_cuda(K, V, idx, counts, offsets, out_offsets, K_out, V_out, workspace, status)
     if K.dim() != 3 or K.shape != V.shape or K.dtype != torch.bfloat16 or V.dtype != torch.bfloat16:
         raise ValueError("K and V must be bfloat16 [B, n_c, d] of equal shape")
     B, n_c, d = K.shape
     if in_place:
         K_out, V_out = K, V
+        if workspace is None:
+            workspace = torch.empty(kvz_compact_workspace_size(B, n_c), dtype=torch.uint8, device=K.device)
     else:
         rows = B * n_c if out_rows is None else int(out_rows)
         if K_out is None:
             K_out = torch.empty((rows, d), dtype=K.dtype, device=K.device)
         if V_out is None:
             V_out = torch.empty((rows, d), dtype=V.dtype, device=V.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("kvz_compact", lib().kvz_compact(_ptr(K), _ptr(V), B, n_c, d, _ptr(idx), _ptr(counts), _ptr(offsets),
-                                            _ptr(out_offsets), _ptr(K_out), _ptr(V_out), _ptr(status),
-                                            _stream(stream)))
+                                            _ptr(out_offsets), _ptr(K_out), _ptr(V_out), _ptr(workspace), ws_bytes,
+                                            _ptr(status), _stream(stream)))
     return K_out, V_out

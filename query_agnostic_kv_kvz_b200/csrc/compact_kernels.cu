@@ -13,22 +13,63 @@ namespace kvz {
 
 namespace {
 
+// Launch-shape tuning (measured on B200; override with -D for sweeps).
+#ifndef KVZ_GATHER_UNROLL
+#define KVZ_GATHER_UNROLL 4
+#endif
+#ifndef KVZ_GATHER_CTAS_PER_SM
+#define KVZ_GATHER_CTAS_PER_SM 8
+#endif
+#ifndef KVZ_INPLACE_THREADS
+#define KVZ_INPLACE_THREADS 128
+#endif
+#ifndef KVZ_INPLACE_ROWS
+#define KVZ_INPLACE_ROWS 16
+#endif
+#ifndef KVZ_INPLACE_DEPTH
+#define KVZ_INPLACE_DEPTH 2
+#endif
+#ifndef KVZ_INPLACE_OVERSUB
+#define KVZ_INPLACE_OVERSUB 3
+#endif
 constexpr int kGatherThreads = 256;
-constexpr int kGatherUnroll = 4;
-constexpr int kInplaceThreads = 512;
-constexpr int kInplaceUnroll = 4;
+constexpr int kGatherUnroll = KVZ_GATHER_UNROLL;
+constexpr int kInplaceThreads = KVZ_INPLACE_THREADS;
+constexpr int kInplaceRows = KVZ_INPLACE_ROWS;           // slots per chunk (one warp moves a chunk)
+constexpr int kInplaceDepth = KVZ_INPLACE_DEPTH;         // chunks in each warp's register ring
+constexpr int kInplaceOversub = KVZ_INPLACE_OVERSUB;     // warps launched per resident warp slot
+static_assert(kInplaceThreads % 32 == 0, "whole warps");
+static_assert(kInplaceDepth >= 2, "a ring holds the chunk being stored and at least one loading");
+static_assert(kInplaceRows % 4 == 0, "a warp-wide access covers 2 (d = 128) or 4 (d = 64) rows");
+static_assert(kInplaceDepth * kInplaceRows / 2 <= 32, "one validity bit per row, lane and stage in 32 bits");
+constexpr uint64_t kWaitNs = 1000ull * 1000ull * 1000ull;   // 1 s: far beyond any legitimate wait
 
 __device__ __forceinline__ void report_err(int32_t* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
-// Read-only streaming load (inputs are never written by this kernel).
+// Streaming load through the read-only path: no kernel here reads a row
+// after writing it.
 __device__ __forceinline__ int4 ld_stream(const int4* p) {
   int4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.s32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
 }
 
 // Out of place.  Grid-stride over blocks of output slots; the head of a
@@ -88,62 +129,199 @@ __global__ void __launch_bounds__(kGatherThreads)
   }
 }
 
-// In place.  One CTA owns one column segment (vps vectors) of every row of
-// one head of one tensor and walks the kept slots in increasing order, a
-// batch at a time.  Slot p moves row idx[p] >= p down to row p.  The loads of
-// batch t+1 read rows >= the first slot of batch t+1, which batch t never
-// writes; the barrier orders every load of batches <= t before the stores
-// of batch t, so no row is overwritten before it has been read.
-__global__ void __launch_bounds__(kInplaceThreads)
-    compact_inplace_kernel(int4* K, int4* V, int64_t n_c, int vpr, int cs, const int32_t* __restrict__ idx,
-                           const int32_t* __restrict__ counts, const int64_t* __restrict__ offsets,
-                           int32_t* status) {
-  const int64_t b = blockIdx.x;
-  const int tsel = blockIdx.y / cs;
-  const int part = blockIdx.y % cs;
-  const int vps = vpr / cs;
-  int4* X = (tsel == 0 ? K : V) + b * n_c * vpr + part * vps;
+// Dependencies of in-place compaction.  Slot chunk c (slots [cC, (c+1)C))
+// writes rows [cC, (c+1)C).  Because idx ascends within a head, the slots
+// whose source rows lie in that range form one contiguous run
+// [lo_slot[c], lo_slot[c+1]), where lo_slot[r] is the first slot whose
+// source row is >= rC (count if none).  Only the chunks holding that run
+// read what chunk c overwrites.  One thread per slot p fills lo_slot[r] for
+// the row chunks r in (chunk(idx[p-1]), chunk(idx[p])], capped at nchunks;
+// the last slot also fills the row chunks past its source.
+__global__ void __launch_bounds__(256)
+    inplace_deps_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
+                        const int64_t* __restrict__ offsets, int64_t n_c, int64_t blocks_per_head,
+                        uint32_t* lo_slot, int64_t lo_stride) {
+  const int64_t b = blockIdx.x / blocks_per_head;
+  const int64_t p = (blockIdx.x % blocks_per_head) * 256 + threadIdx.x;
   const int64_t count = counts[b];
-  const int64_t base = offsets[b];
-  const int rows_per_batch = kInplaceThreads * kInplaceUnroll / vps;
-  const int64_t nb = (count + rows_per_batch - 1) / rows_per_batch;
+  if (count < 0 || count > n_c || p >= count) return;   // the compaction kernel reports a bad count
+  const int64_t nchunks = (count + kInplaceRows - 1) / kInplaceRows;
+  const int32_t* hidx = idx + offsets[b];
+  auto row_chunk = [&](int64_t v) -> int64_t {
+    return v < 0 ? -1 : (v / kInplaceRows < nchunks ? v / kInplaceRows : nchunks);
+  };
+  const int64_t r1 = p == 0 ? -1 : row_chunk(hidx[p - 1]);
+  const int64_t r2 = row_chunk(hidx[p]);
+  uint32_t* lo = lo_slot + b * lo_stride;
+  for (int64_t r = r1 + 1; r <= r2; ++r) lo[r] = static_cast<uint32_t>(p);
+  if (p == count - 1)
+    for (int64_t r = (r2 > r1 ? r2 : r1) + 1; r <= nchunks; ++r) lo[r] = static_cast<uint32_t>(count);
+}
+
+// In place.  Slot p of head b moves row idx[p] >= p down to row p, in K and
+// in V.  Slots are cut into chunks of kInplaceRows; chunk c writes rows
+// [cC, (c+1)C).  A row q is the source of at most one slot p', with
+// p' <= idx[p'] = q, so only chunks <= c read rows that chunk c writes, and
+// of those only the chunks holding slots [lo_slot[c], lo_slot[c+1]).
+// Each warp is an independent worker: it claims chunks of its head from a
+// per-head counter (lower chunks are claimed first) and keeps kInplaceDepth
+// of them in a register ring, loads issued kInplaceDepth - 1 chunks ahead.
+// For its oldest (current) chunk c the warp
+//   - checks, acquiring with a bounded wait, that the chunks below c that
+//     read chunk c's rows have published "sources read",
+//   - writes chunk c's rows from registers (which needs its own loads of c
+//     to have landed), then publishes chunk c's flag (release),
+//   - refills the freed ring stage with a later chunk.
+// At a keep ratio rho the readers of chunk c sit near chunk rho*c, long
+// finished, so warps rarely wait.  A warp's current chunk is its lowest
+// unpublished one and waits only on lower chunks, so the lowest unpublished
+// chunk of a head always belongs to a warp whose waits are satisfied: every
+// wait ends.  No row is written before its reader has loaded it, so the
+// loads may take the read-only path.
+template <int VPR>
+__global__ void __launch_bounds__(kInplaceThreads)
+    compact_inplace_kernel(int4* K, int4* V, int64_t B, int64_t n_c, int64_t warps_per_head,
+                           const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
+                           const int64_t* __restrict__ offsets, uint32_t* next_chunk, uint32_t* chunk_read,
+                           int64_t chunks_per_head, const uint32_t* lo_slot, int32_t* status) {
+  constexpr int kRowsPerAccess = 32 / VPR;                    // rows one warp-wide access covers
+  constexpr int NR = kInplaceRows / kRowsPerAccess;           // rows of a chunk each lane moves
+  constexpr int D = kInplaceDepth;
+  constexpr uint32_t kFull = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = (static_cast<int64_t>(blockIdx.x) * kInplaceThreads + threadIdx.x) >> 5;
+  const int64_t b = gw / warps_per_head;
+  if (b >= B) return;                                         // warp-uniform
+  const int64_t count = counts[b];
   if (count < 0 || count > n_c) {
-    if (threadIdx.x == 0) report_err(status, KVZ_ERR_INVALID_ARG);
+    if (lane == 0 && gw % warps_per_head == 0) report_err(status, KVZ_ERR_INVALID_ARG);
     return;
   }
-  int4 cur[kInplaceUnroll], nxt[kInplaceUnroll];
-  bool cur_ok[kInplaceUnroll], nxt_ok[kInplaceUnroll];
-  auto load = [&](int64_t t, int4 (&v)[kInplaceUnroll], bool (&ok)[kInplaceUnroll]) {
+  const uint32_t nchunks = static_cast<uint32_t>((count + kInplaceRows - 1) / kInplaceRows);
+  int4* const Xk = K + b * n_c * VPR;
+  int4* const Xv = V + b * n_c * VPR;
+  uint32_t* const flags = chunk_read + b * chunks_per_head;
+  const uint32_t* const lo = lo_slot + b * (chunks_per_head + 1);
+  const int32_t* const hidx = idx + offsets[b];
+  const int col = lane % VPR;                                 // 16-byte vector within the row
+  const int rsub = lane / VPR;                                // row within an access
+
+  int4 dk[D][NR], dv[D][NR];                                  // the register ring
+  uint32_t valid = 0;                                         // bit s*NR + k: element k of stage s
+  int32_t jn[NR];                                             // source rows of the next chunk to load
+  uint32_t cl[D];                                             // chunk held by each stage (warp-uniform)
+
+  auto fetch_idx = [&](uint32_t c) {
 #pragma unroll
-    for (int u = 0; u < kInplaceUnroll; ++u) {
-      const int item = threadIdx.x + u * kInplaceThreads;
-      const int64_t p = t * rows_per_batch + item / vps;
-      ok[u] = false;
-      if (p < count) {
-        const int64_t j = idx[base + p];
-        if (j < p || j >= n_c) {             // ascending idx guarantees j >= p
-          report_err(status, KVZ_ERR_INVALID_ARG);
-        } else {
-          v[u] = __ldcg(X + j * vpr + item % vps);
-          ok[u] = true;
-        }
-      }
+    for (int k = 0; k < NR; ++k) {
+      const int64_t p = static_cast<int64_t>(c) * kInplaceRows + rsub + k * kRowsPerAccess;
+      jn[k] = (c < nchunks && p < count) ? hidx[p] : -1;
     }
   };
-  if (nb > 0) load(0, cur, cur_ok);
-  for (int64_t t = 0; t < nb; ++t) {
-    if (t + 1 < nb) load(t + 1, nxt, nxt_ok);
-    __syncthreads();
+  auto issue = [&](int st, uint32_t c) {
+    uint32_t bits = 0;
 #pragma unroll
-    for (int u = 0; u < kInplaceUnroll; ++u) {
-      const int item = threadIdx.x + u * kInplaceThreads;
-      const int64_t p = t * rows_per_batch + item / vps;
-      if (cur_ok[u]) X[p * vpr + item % vps] = cur[u];
+    for (int k = 0; k < NR; ++k) {
+      const int64_t p = static_cast<int64_t>(c) * kInplaceRows + rsub + k * kRowsPerAccess;
+      if (c >= nchunks || p >= count) continue;
+      const int64_t j = jn[k];
+      if (j >= p && j < n_c) {
+        dk[st][k] = ld_stream(Xk + j * VPR + col);
+        dv[st][k] = ld_stream(Xv + j * VPR + col);
+        bits |= 1u << k;
+      } else {
+        report_err(status, KVZ_ERR_INVALID_ARG);              // ascending idx guarantees p <= j < n_c
+      }
     }
+    valid = (valid & ~(((1u << NR) - 1u) << (st * NR))) | (bits << (st * NR));
+  };
+
+  {
+    uint32_t first[D];
 #pragma unroll
-    for (int u = 0; u < kInplaceUnroll; ++u) {
-      cur[u] = nxt[u];
-      cur_ok[u] = nxt_ok[u];
+    for (int s = 0; s < D; ++s) first[s] = lane == 0 ? atomicAdd(&next_chunk[b], 1u) : 0u;
+#pragma unroll
+    for (int s = 0; s < D; ++s) cl[s] = __shfl_sync(kFull, first[s], 0);
+  }
+#pragma unroll
+  for (int s = 0; s < D - 1; ++s) {
+    fetch_idx(cl[s]);
+    issue(s, cl[s]);
+  }
+  fetch_idx(cl[D - 1]);                                       // issued at the first step
+  uint32_t pend = lane == 0 ? atomicAdd(&next_chunk[b], 1u) : 0u;   // the claim after that
+
+  // Readers of chunk c: chunks [k0, k_end) (see inplace_deps_kernel).  The
+  // run bounds of a chunk are loaded two steps before it is current and its
+  // readers' flags one step before (lane l takes reader k0 + l); only a flag
+  // seen unset, or a run longer than a warp, is polled at the current step.
+  auto reader_range = [&](uint32_t c, uint32_t run_lo, uint32_t run_hi, uint32_t& k0, uint32_t& k_end) {
+    const uint32_t k_last = run_hi > run_lo ? (run_hi - 1) / kInplaceRows + 1 : 0u;
+    k0 = run_lo / kInplaceRows;
+    k_end = c < nchunks ? (k_last < c ? k_last : c) : 0u;
+  };
+  auto first_flag = [&](uint32_t k0, uint32_t k_end) -> uint32_t {
+    return k0 + lane < k_end ? ld_acquire_gpu(&flags[k0 + lane]) : 1u;
+  };
+  uint32_t k0 = 0, k_end = 0, seen = 1;                       // the current chunk's readers
+  uint32_t nlo = 0, nhi = 0;                                  // run bounds of the next chunk
+  if (cl[0] < nchunks) {
+    reader_range(cl[0], lo[cl[0]], lo[cl[0] + 1], k0, k_end);
+    seen = first_flag(k0, k_end);
+  }
+  if (cl[1 % D] < nchunks) {
+    nlo = lo[cl[1 % D]];
+    nhi = lo[cl[1 % D] + 1];
+  }
+  bool done = false;
+  while (!done) {
+#pragma unroll
+    for (int s = 0; s < D; ++s) {
+      const uint32_t cur = cl[s];
+      if (cur >= nchunks) {                                   // later claims are higher chunks
+        done = true;
+        break;
+      }
+      int ok = 1;
+      for (uint32_t k = k0 + lane; k < k_end; k += 32) {
+        if (k == k0 + lane && seen != 0u) continue;
+        if (ld_acquire_gpu(&flags[k]) != 0u) continue;
+        const uint64_t t0 = now_ns();
+        while (ld_acquire_gpu(&flags[k]) == 0u) {
+          if (now_ns() - t0 > kWaitNs) {
+            ok = 0;
+            break;
+          }
+        }
+        if (!ok) break;
+      }
+      if (!__all_sync(kFull, ok)) {                           // a reader never published: stop
+        if (lane == 0) report_err(status, KVZ_ERR_TIMEOUT);
+        done = true;
+        break;
+      }
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        if (!((valid >> (s * NR + k)) & 1u)) continue;
+        const int64_t p = static_cast<int64_t>(cur) * kInplaceRows + rsub + k * kRowsPerAccess;
+        Xk[p * VPR + col] = dk[s][k];
+        Xv[p * VPR + col] = dv[s][k];
+      }
+      __syncwarp();                                           // every lane's loads of cur have landed
+      if (lane == 0) st_release_gpu(&flags[cur], 1u);
+      const int sn = (s + D - 1) % D;                         // the stage written out last step
+      issue(sn, cl[sn]);
+      const uint32_t c_next = __shfl_sync(kFull, pend, 0);
+      fetch_idx(c_next);
+      if (lane == 0) pend = atomicAdd(&next_chunk[b], 1u);
+      cl[s] = c_next;
+      const uint32_t c1 = cl[(s + 1) % D], c2 = cl[(s + 2) % D];   // the next two steps' chunks
+      reader_range(c1, nlo, nhi, k0, k_end);
+      seen = first_flag(k0, k_end);
+      if (c2 < nchunks) {
+        nlo = lo[c2];
+        nhi = lo[c2 + 1];
+      }
     }
   }
 }
@@ -156,7 +334,7 @@ cudaError_t launch_compact_gather(const void* K, const void* V, int64_t B, int64
   const int vpr = d / 8;                       // 16-byte vectors per row
   const int rows_per_blk = (kGatherThreads / vpr) * kGatherUnroll;
   int64_t blocks = (B * n_c + rows_per_blk - 1) / rows_per_blk;
-  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (blocks > 148 * KVZ_GATHER_CTAS_PER_SM) blocks = 148 * KVZ_GATHER_CTAS_PER_SM;
   if (blocks < 1) blocks = 1;
   compact_gather_kernel<<<static_cast<unsigned>(blocks), kGatherThreads, 0, stream>>>(
       static_cast<const int4*>(K), static_cast<const int4*>(V), B, n_c, vpr, idx, offsets, out_offsets,
@@ -164,14 +342,42 @@ cudaError_t launch_compact_gather(const void* K, const void* V, int64_t B, int64
   return cudaGetLastError();
 }
 
+size_t compact_workspace_bytes(int64_t B, int64_t n_c) {
+  const int64_t chunks = (n_c + kInplaceRows - 1) / kInplaceRows;
+  return static_cast<size_t>((B * (2 + 2 * chunks) * 4 + 255) / 256 * 256);
+}
+
 cudaError_t launch_compact_inplace(void* K, void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
-                                   const int32_t* counts, const int64_t* offsets, int32_t* status,
+                                   const int32_t* counts, const int64_t* offsets, uint32_t* ws, int32_t* status,
                                    cudaStream_t stream) {
-  const int vpr = d / 8;
-  const int cs = vpr / 8;                      // 128-byte column segments
-  const dim3 grid(static_cast<unsigned>(B), static_cast<unsigned>(2 * cs));
-  compact_inplace_kernel<<<grid, kInplaceThreads, 0, stream>>>(static_cast<int4*>(K), static_cast<int4*>(V),
-                                                               n_c, vpr, cs, idx, counts, offsets, status);
+  const int64_t chunks = (n_c + kInplaceRows - 1) / kInplaceRows;
+  // next_chunk[B] | chunk_read[B][chunks] | lo_slot[B][chunks + 1], all zeroed (all-zero bits)
+  uint32_t* next_chunk = ws;
+  uint32_t* chunk_read = next_chunk + B;
+  uint32_t* lo_slot = chunk_read + B * chunks;
+  cudaError_t e = launch_fill_f32(reinterpret_cast<float*>(ws), B * (2 + 2 * chunks), 0.0f, stream);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks_per_head = (n_c + 255) / 256;
+  if (B * blocks_per_head > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  inplace_deps_kernel<<<static_cast<unsigned>(B * blocks_per_head), 256, 0, stream>>>(
+      idx, counts, offsets, n_c, blocks_per_head, lo_slot, chunks + 1);
+  auto kern = d == 128 ? compact_inplace_kernel<16> : compact_inplace_kernel<8>;
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kInplaceThreads, 0)) != cudaSuccess) return e;
+  // Enough warp workers to fill every resident warp slot kInplaceOversub times,
+  // spread evenly over the heads, at most one per chunk.
+  const int64_t slots = static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1) * (kInplaceThreads / 32);
+  int64_t wph = (slots * kInplaceOversub + B - 1) / B;
+  if (wph > chunks) wph = chunks;
+  if (wph < 1) wph = 1;
+  const int64_t warps_per_cta = kInplaceThreads / 32;
+  const int64_t grid = (B * wph + warps_per_cta - 1) / warps_per_cta;
+  if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(grid), kInplaceThreads, 0, stream>>>(
+      static_cast<int4*>(K), static_cast<int4*>(V), B, n_c, wph, idx, counts, offsets, next_chunk, chunk_read, chunks,
+      lo_slot, status);
   return cudaGetLastError();
 }
 

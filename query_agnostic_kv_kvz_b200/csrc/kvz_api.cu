@@ -272,14 +272,19 @@ kvz_status kvz_select(const float* S, int64_t B, int64_t n_c, double ratio, int 
              : KVZ_ERR_CUDA;
 }
 
+size_t kvz_compact_workspace_size(int64_t B, int64_t n_c) {
+  if (B < 1 || n_c < 1) return 0;
+  return kvz::compact_workspace_bytes(B, n_c);
+}
+
 kvz_status kvz_compact(const void* K, const void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
                        const int32_t* counts, const int64_t* offsets, const int64_t* out_offsets, void* K_out,
-                       void* V_out, int32_t* d_status, cudaStream_t stream) {
+                       void* V_out, void* workspace, size_t workspace_bytes, int32_t* d_status, cudaStream_t stream) {
   if (K == nullptr || V == nullptr || K_out == nullptr || V_out == nullptr || counts == nullptr ||
       offsets == nullptr || idx == nullptr)
     return KVZ_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return KVZ_ERR_UNSUPPORTED;
-  if (B < 1 || B > 0x7FFFFFFF || n_c < 1 || n_c > kMaxRows) return KVZ_ERR_INVALID_ARG;
+  if (B < 1 || B > 0x7FFFFFFF / 8 || n_c < 1 || n_c > kMaxRows) return KVZ_ERR_INVALID_ARG;
   if (!aligned(K, 16) || !aligned(V, 16) || !aligned(K_out, 16) || !aligned(V_out, 16) || !aligned(idx, 4) ||
       !aligned(counts, 4) || !aligned(offsets, 8) || (out_offsets && !aligned(out_offsets, 8)))
     return KVZ_ERR_ALIGNMENT;
@@ -288,8 +293,10 @@ kvz_status kvz_compact(const void* K, const void* V, int64_t B, int64_t n_c, int
   if (K == V) return KVZ_ERR_INVALID_ARG;
   if (k_same) {
     if (out_offsets != nullptr) return KVZ_ERR_INVALID_ARG;
-    return kvz::launch_compact_inplace(K_out, V_out, B, n_c, d, idx, counts, offsets, d_status, stream) ==
-                   cudaSuccess
+    if (workspace == nullptr || workspace_bytes < kvz::compact_workspace_bytes(B, n_c)) return KVZ_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return KVZ_ERR_ALIGNMENT;
+    return kvz::launch_compact_inplace(K_out, V_out, B, n_c, d, idx, counts, offsets,
+                                       static_cast<uint32_t*>(workspace), d_status, stream) == cudaSuccess
                ? KVZ_OK
                : KVZ_ERR_CUDA;
   }

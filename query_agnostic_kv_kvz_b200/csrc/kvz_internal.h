@@ -54,8 +54,11 @@ cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int mode, int6
 cudaError_t launch_compact_gather(const void* K, const void* V, int64_t B, int64_t n_c, int d,
                                   const int32_t* idx, const int64_t* offsets, const int64_t* out_offsets,
                                   void* K_out, void* V_out, int32_t* status, cudaStream_t stream);
+// In place: `ws` holds B + B*ceil(n_c/chunk) uint32 (per-head chunk claims and
+// per-chunk "sources read" flags); the launcher zeroes it on `stream`.
 cudaError_t launch_compact_inplace(void* K, void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
-                                   const int32_t* counts, const int64_t* offsets, int32_t* status,
+                                   const int32_t* counts, const int64_t* offsets, uint32_t* ws, int32_t* status,
                                    cudaStream_t stream);
+size_t compact_workspace_bytes(int64_t B, int64_t n_c);
 
 }  // namespace kvz

@@ -118,9 +118,12 @@ def test_compact_rejections(lib):
     idx, cnt, off = b.get(B * n_c * 4), b.get(B * 4), b.get((B + 1) * 8)
     outo = b.get((B + 1) * 8)
 
-    def call(K_=K, V_=V, Ko_=Ko, Vo_=Vo, d_=d, oo=None):
+    ws = b.get(lib.kvz_compact_workspace_size(B, n_c))
+
+    def call(K_=K, V_=V, Ko_=Ko, Vo_=Vo, d_=d, oo=None, ws_=ws, wsb=None):
+        wsb = lib.kvz_compact_workspace_size(B, n_c) if wsb is None else wsb
         return lib.kvz_compact(vp(K_), vp(V_), B, n_c, d_, vp(idx), vp(cnt), vp(off), vp(oo) if oo else None,
-                               vp(Ko_), vp(Vo_), None, None)
+                               vp(Ko_), vp(Vo_), vp(ws_) if ws_ else None, wsb, None, None)
 
     assert call(d_=96) == UNSUPPORTED
     assert call(Ko_=K) == INVALID                    # K in place, V not
@@ -128,5 +131,7 @@ def test_compact_rejections(lib):
     assert call(V_=K) == INVALID                     # K and V are the same buffer
     assert call(Ko_=K + 4096) == INVALID             # output starts inside an input
     assert call(Ko_=Ko + 8) == ALIGN
-    assert lib.kvz_compact(vp(K), vp(V), B, n_c, d, None, vp(cnt), vp(off), None, vp(Ko), vp(Vo), None,
-                           None) == INVALID
+    assert call(Ko_=K, Vo_=V, ws_=0) == WS           # in place needs the progress counters
+    assert call(Ko_=K, Vo_=V, wsb=8) == WS
+    assert lib.kvz_compact(vp(K), vp(V), B, n_c, d, None, vp(cnt), vp(off), None, vp(Ko), vp(Vo), None, 0,
+                           None, None) == INVALID

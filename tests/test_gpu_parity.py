@@ -209,6 +209,41 @@ def test_compact_in_place_matches_oracle(B, n_c, d, ratio, mode):
         assert not np.any(Ko[b, :c] == 0x7FC1)
 
 
+@pytest.mark.parametrize("pattern", ["tail", "head", "blocks", "sparse_tail"])
+def test_compact_in_place_structured(pattern):
+    """Kept keys clustered so that destination chunks and their source rows
+    sit at every distance: all at the end (every row moves far down), all at
+    the start (every row stays), alternating blocks of 50, and a thin tail."""
+    B, n_c, d = 3, 20000, 128
+    j = torch.arange(n_c, device="cuda", dtype=torch.float32)
+    if pattern == "tail":
+        S, ratio = (j + 1) / n_c, 0.6
+    elif pattern == "head":
+        S, ratio = (n_c - j) / n_c, 0.6
+    elif pattern == "blocks":
+        S, ratio = ((j // 50) % 2 == 0).float() + 1e-6 * (n_c - j) / n_c, 0.5
+    else:
+        S, ratio = (j + 1) / n_c, 0.03
+    S = S.expand(B, n_c).contiguous()
+    g = torch.Generator(device="cuda").manual_seed(7)
+    K = torch.randn((B, n_c, d), generator=g, device="cuda").to(torch.bfloat16)
+    V = torch.randn((B, n_c, d), generator=g, device="cuda").to(torch.bfloat16)
+    idx, counts, offsets = kvz.kvz_select(S, ratio, "per_head")
+    Kh, Vh = bits(K), bits(V)
+    ic, cc, oc = idx.cpu().numpy(), counts.cpu().numpy(), offsets.cpu().numpy()
+    rk, rv = orc.compact(Kh, Vh, ic, cc, oc)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvz.kvz_compact(K, V, idx, counts, offsets, in_place=True, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    Ko, Vo = bits(K), bits(V)
+    for b in range(B):
+        c = int(cc[b])
+        np.testing.assert_array_equal(Ko[b, :c], rk[oc[b]:oc[b] + c])
+        np.testing.assert_array_equal(Vo[b, :c], rv[oc[b]:oc[b] + c])
+        np.testing.assert_array_equal(Ko[b, c:], Kh[b, c:])
+
+
 # ---------------------------------------------------------------------------
 # The whole path on the two small workloads
 # ---------------------------------------------------------------------------
