@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--workload", default=WORKLOAD,
                     help="llama8b_layer (default, the headline), tiny, llama8b_stack, qwen14b_128k, stress_ragged")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="run only the first L layers of the workload (a smaller case for profiling; "
+                         "config.workload then names the truncation)")
     return ap.parse_args()
 
 
@@ -198,10 +201,15 @@ def main():
 
     from query_agnostic_kv_kvz_b200 import synth
     w = synth.WORKLOADS[args.workload]
+    n_layers_full = w.L
+    if 0 < args.layers < w.L:
+        import dataclasses
+        w = dataclasses.replace(w, L=args.layers)
     nums = workload_numbers(w)
     config = {"workload": "%s (L=%d, H=%d, G=%d, d=%d, n_c=%s, n_prompt=%d, keep %.2f %s%s%s)" % (
         w.name, w.L, w.H, w.G, w.d, "/".join(str(n) for n in w.n_c), w.n_prompt, w.ratio, w.mode,
-        ", rows in chunks of %d" % w.row_chunk if w.row_chunk else "", ", in-place compaction" if w.in_place else ""),
+        ", rows in chunks of %d" % w.row_chunk if w.row_chunk else "", ", in-place compaction" if w.in_place else "")
+        + ("; first %d of its %d layers only" % (w.L, n_layers_full) if w.L < n_layers_full else ""),
         "B_heads": w.B, "G": w.G, "d": w.d, "n_c": list(w.n_c), "n_in": [w.n_in(c) for c in range(len(w.n_c))],
         "ratio": w.ratio, "mode": w.mode,
         "l2": "flushed before every timed step (256 MB write, outside the timed events)",
@@ -456,7 +464,8 @@ class Context:
             self.K_out = torch.empty((cap, d), dtype=torch.bfloat16, device=dev)
             self.V_out = torch.empty((cap, d), dtype=torch.bfloat16, device=dev)
         # lse (+ colmax, + S fill on the first chunk) per (layer, chunk); select 10; compact 1
-        self.launches = L * (2 * len(self.chunks) + 1) + 10 + 1
+        # (in place: workspace fill, reader-run pre-pass, compaction)
+        self.launches = L * (2 * len(self.chunks) + 1) + 10 + (3 if w.in_place else 1)
 
 
 if __name__ == "__main__":

@@ -32,12 +32,16 @@ namespace {
 #ifndef KVZ_INPLACE_OVERSUB
 #define KVZ_INPLACE_OVERSUB 3
 #endif
+#ifndef KVZ_INPLACE_MIN_CTAS
+#define KVZ_INPLACE_MIN_CTAS 3
+#endif
 constexpr int kGatherThreads = 256;
 constexpr int kGatherUnroll = KVZ_GATHER_UNROLL;
 constexpr int kInplaceThreads = KVZ_INPLACE_THREADS;
 constexpr int kInplaceRows = KVZ_INPLACE_ROWS;           // slots per chunk (one warp moves a chunk)
 constexpr int kInplaceDepth = KVZ_INPLACE_DEPTH;         // chunks in each warp's register ring
 constexpr int kInplaceOversub = KVZ_INPLACE_OVERSUB;     // warps launched per resident warp slot
+constexpr int kInplaceMinCtas = KVZ_INPLACE_MIN_CTAS;    // resident CTAs per SM the registers must allow
 static_assert(kInplaceThreads % 32 == 0, "whole warps");
 static_assert(kInplaceDepth >= 2, "a ring holds the chunk being stored and at least one loading");
 static_assert(kInplaceRows % 4 == 0, "a warp-wide access covers 2 (d = 128) or 4 (d = 64) rows");
@@ -58,13 +62,20 @@ __device__ __forceinline__ int4 ld_stream(const int4* p) {
   return v;
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
   uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ void red_relaxed_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// A zero computed from x that the compiler cannot fold: a value built with it
+// carries a data dependency on the load that produced x.
+__device__ __forceinline__ uint32_t dep_zero(uint32_t x) {
+  uint32_t z;
+  asm volatile("and.b32 %0, %1, 0;" : "=r"(z) : "r"(x));
+  return z;
 }
 __device__ __forceinline__ uint64_t now_ns() {
   uint64_t t;
@@ -166,20 +177,23 @@ __global__ void __launch_bounds__(256)
 // Each warp is an independent worker: it claims chunks of its head from a
 // per-head counter (lower chunks are claimed first) and keeps kInplaceDepth
 // of them in a register ring, loads issued kInplaceDepth - 1 chunks ahead.
-// For its oldest (current) chunk c the warp
-//   - checks, acquiring with a bounded wait, that the chunks below c that
-//     read chunk c's rows have published "sources read",
-//   - writes chunk c's rows from registers (which needs its own loads of c
-//     to have landed), then publishes chunk c's flag (release),
-//   - refills the freed ring stage with a later chunk.
-// At a keep ratio rho the readers of chunk c sit near chunk rho*c, long
-// finished, so warps rarely wait.  A warp's current chunk is its lowest
-// unpublished one and waits only on lower chunks, so the lowest unpublished
-// chunk of a head always belongs to a warp whose waits are satisfied: every
-// wait ends.  No row is written before its reader has loaded it, so the
-// loads may take the read-only path.
+// For its oldest (current) chunk c every lane of the warp
+//   - reads the "sources read" counters of the chunks below c that read
+//     chunk c's rows (at most two: each of chunk c's rows feeds at most one
+//     slot) and waits, bounded, until each shows all 32 lanes,
+//   - writes its part of chunk c's rows from registers, then adds
+//     1 + (a zero computed from the rows it loaded) to chunk c's counter.
+// The add's value depends on the lane's loads and each row store is
+// control-dependent on the counters its lane read, so a load can only see a
+// row's old contents; no fence is needed (a release fence would wait for
+// every load in flight).  At a keep ratio rho the readers of chunk c sit
+// near chunk rho*c, long finished, so warps rarely wait.  A warp's current
+// chunk is its lowest unpublished one and waits only on lower chunks, so
+// the lowest unpublished chunk of a head always belongs to a warp whose
+// waits are satisfied: every wait ends.  No row is written before its
+// reader has loaded it, so the loads may take the read-only path.
 template <int VPR>
-__global__ void __launch_bounds__(kInplaceThreads)
+__global__ void __launch_bounds__(kInplaceThreads, kInplaceMinCtas)
     compact_inplace_kernel(int4* K, int4* V, int64_t B, int64_t n_c, int64_t warps_per_head,
                            const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
                            const int64_t* __restrict__ offsets, uint32_t* next_chunk, uint32_t* chunk_read,
@@ -253,17 +267,17 @@ __global__ void __launch_bounds__(kInplaceThreads)
 
   // Readers of chunk c: chunks [k0, k_end) (see inplace_deps_kernel).  The
   // run bounds of a chunk are loaded two steps before it is current and its
-  // readers' flags one step before (lane l takes reader k0 + l); only a flag
-  // seen unset, or a run longer than a warp, is polled at the current step.
+  // first reader's counter one step before; anything not yet complete is
+  // polled at the current step.
   auto reader_range = [&](uint32_t c, uint32_t run_lo, uint32_t run_hi, uint32_t& k0, uint32_t& k_end) {
     const uint32_t k_last = run_hi > run_lo ? (run_hi - 1) / kInplaceRows + 1 : 0u;
     k0 = run_lo / kInplaceRows;
     k_end = c < nchunks ? (k_last < c ? k_last : c) : 0u;
   };
   auto first_flag = [&](uint32_t k0, uint32_t k_end) -> uint32_t {
-    return k0 + lane < k_end ? ld_acquire_gpu(&flags[k0 + lane]) : 1u;
+    return k0 < k_end ? ld_relaxed_gpu(&flags[k0]) : 32u;
   };
-  uint32_t k0 = 0, k_end = 0, seen = 1;                       // the current chunk's readers
+  uint32_t k0 = 0, k_end = 0, seen = 32;                      // the current chunk's readers
   uint32_t nlo = 0, nhi = 0;                                  // run bounds of the next chunk
   if (cl[0] < nchunks) {
     reader_range(cl[0], lo[cl[0]], lo[cl[0] + 1], k0, k_end);
@@ -283,11 +297,11 @@ __global__ void __launch_bounds__(kInplaceThreads)
         break;
       }
       int ok = 1;
-      for (uint32_t k = k0 + lane; k < k_end; k += 32) {
-        if (k == k0 + lane && seen != 0u) continue;
-        if (ld_acquire_gpu(&flags[k]) != 0u) continue;
+      for (uint32_t k = k0; k < k_end; ++k) {
+        if (k == k0 && seen == 32u) continue;
+        if (ld_relaxed_gpu(&flags[k]) == 32u) continue;
         const uint64_t t0 = now_ns();
-        while (ld_acquire_gpu(&flags[k]) == 0u) {
+        while (ld_relaxed_gpu(&flags[k]) != 32u) {
           if (now_ns() - t0 > kWaitNs) {
             ok = 0;
             break;
@@ -300,15 +314,16 @@ __global__ void __launch_bounds__(kInplaceThreads)
         done = true;
         break;
       }
+      uint32_t got = 0;                                       // a word of every row this lane loaded
 #pragma unroll
       for (int k = 0; k < NR; ++k) {
         if (!((valid >> (s * NR + k)) & 1u)) continue;
         const int64_t p = static_cast<int64_t>(cur) * kInplaceRows + rsub + k * kRowsPerAccess;
         Xk[p * VPR + col] = dk[s][k];
         Xv[p * VPR + col] = dv[s][k];
+        got |= static_cast<uint32_t>(dk[s][k].x) | static_cast<uint32_t>(dv[s][k].x);
       }
-      __syncwarp();                                           // every lane's loads of cur have landed
-      if (lane == 0) st_release_gpu(&flags[cur], 1u);
+      red_relaxed_gpu_add(&flags[cur], 1u + dep_zero(got));   // this lane's sources of cur are read
       const int sn = (s + D - 1) % D;                         // the stage written out last step
       issue(sn, cl[sn]);
       const uint32_t c_next = __shfl_sync(kFull, pend, 0);
