@@ -38,7 +38,7 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128);
 // Of every 16 exp2 evaluations in pass 1, how many run as a polynomial on
 // the FMA pipe instead of the SFU (even, 0..16).
 #ifndef KVZ_POLY_PER16
-#define KVZ_POLY_PER16 4
+#define KVZ_POLY_PER16 2
 #endif
 constexpr int kPolyPer16 = KVZ_POLY_PER16;
 static_assert(kPolyPer16 % 2 == 0 && kPolyPer16 >= 0 && kPolyPer16 <= 16, "pairs of exp2");

@@ -303,6 +303,126 @@ __global__ void __launch_bounds__(kSelThreads) sel_write(const float* S, int64_t
   }
 }
 
+// Per-head mode, one CTA per head: the same radix select and stable write as
+// the kernels above, with the histograms, the digit picks and the scans in
+// shared memory, so the whole selection is one launch.  With STAGED the
+// head's keys stay in shared memory after the first pass.
+constexpr int kHeadThreads = 1024;
+constexpr int kHeadItems = 8;                            // consecutive scores per thread when writing
+constexpr int kHeadTile = kHeadThreads * kHeadItems;
+constexpr int64_t kHeadStageMax = 49152;                 // scores staged in shared memory (192 KB)
+
+template <bool STAGED>
+__global__ void __launch_bounds__(kHeadThreads) sel_head_kernel(const float* S, int64_t B, int64_t n_c,
+                                                                int64_t k, int32_t* idx, int32_t* counts,
+                                                                int64_t* offsets, int32_t* status) {
+  extern __shared__ uint32_t skey[];                     // STAGED: the head's keys
+  __shared__ uint32_t hist[kBins];
+  __shared__ unsigned long long wbuf[32];
+  __shared__ uint32_t s_prefix, s_mask;
+  __shared__ unsigned long long s_krem, s_keep, s_eq;
+  const int64_t b = blockIdx.x;
+  const float* src = S + b * n_c;
+  if (threadIdx.x == 0) {
+    counts[b] = static_cast<int32_t>(k);
+    offsets[b] = b * k;
+    if (b == B - 1) offsets[B] = B * k;
+    s_prefix = 0u;
+    s_mask = 0u;
+    s_krem = static_cast<unsigned long long>(k);
+    s_keep = 0ull;
+    s_eq = 0ull;
+  }
+  if (k == 0) return;
+  auto key_at = [&](int64_t j) -> uint32_t { return STAGED ? skey[j] : score_key(__ldg(src + j), nullptr); };
+
+  for (int pass = 0; pass < 3; ++pass) {
+    for (int e = threadIdx.x; e < kBins; e += kHeadThreads) hist[e] = 0u;
+    __syncthreads();
+    const uint32_t prefix = s_prefix, mask = s_mask;
+    const int sh = digit_shift(pass);
+    const uint32_t dm = digit_mask(pass);
+    for (int64_t j = threadIdx.x; j < n_c; j += kHeadThreads) {
+      uint32_t key;
+      if (pass == 0) {
+        key = score_key(__ldg(src + j), status);
+        if (STAGED) skey[j] = key;
+      } else {
+        key = key_at(j);
+      }
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> sh) & dm], 1u);
+    }
+    __syncthreads();
+    const unsigned long long k_rem = s_krem;
+    // position x = 0 is the highest digit; thread t owns positions 2t, 2t+1
+    const int nb = pass == 2 ? 1024 : 2048;
+    const int x0 = 2 * static_cast<int>(threadIdx.x);
+    const unsigned long long c0 = x0 < nb ? hist[nb - 1 - x0] : 0ull;
+    const unsigned long long c1 = x0 + 1 < nb ? hist[nb - 2 - x0] : 0ull;
+    const unsigned long long incl = block_inclusive_sum<unsigned long long>(c0 + c1, wbuf);
+    const unsigned long long excl = incl - c0 - c1;
+    int x = -1;
+    unsigned long long above = 0ull;
+    if (excl < k_rem && excl + c0 >= k_rem) {
+      x = x0;
+      above = excl;
+    } else if (excl + c0 < k_rem && excl + c0 + c1 >= k_rem) {
+      x = x0 + 1;
+      above = excl + c0;
+    }
+    if (x >= 0) {                                        // exactly one thread
+      const uint32_t digit = static_cast<uint32_t>(nb - 1 - x);
+      s_prefix = prefix | (digit << sh);
+      s_mask = mask | (dm << sh);
+      s_krem = k_rem - above;
+    }
+    __syncthreads();
+  }
+
+  const uint32_t T = s_prefix;
+  const unsigned long long r_t = s_krem;                 // keys equal to T that are kept
+  int32_t* out = idx + b * k;
+  for (int64_t base = 0; base < n_c; base += kHeadTile) {
+    const unsigned long long keep0 = s_keep, eq0 = s_eq; // kept / equal keys before this tile
+    const int64_t j0 = base + static_cast<int64_t>(threadIdx.x) * kHeadItems;
+    uint32_t key[kHeadItems];
+    uint32_t neq = 0u;
+#pragma unroll
+    for (int it = 0; it < kHeadItems; ++it) {
+      const int64_t j = j0 + it;
+      key[it] = j < n_c ? key_at(j) : 0u;
+      neq += (j < n_c && key[it] == T) ? 1u : 0u;
+    }
+    const unsigned long long eq_incl = block_inclusive_sum<unsigned long long>(neq, wbuf);
+    unsigned long long e = eq0 + eq_incl - neq;
+    uint32_t keep_bits = 0u, nkeep = 0u;
+#pragma unroll
+    for (int it = 0; it < kHeadItems; ++it) {
+      bool keep = false;
+      if (j0 + it < n_c) {
+        if (key[it] > T) {
+          keep = true;
+        } else if (key[it] == T) {
+          keep = e < r_t;
+          ++e;
+        }
+      }
+      keep_bits |= keep ? (1u << it) : 0u;
+      nkeep += keep ? 1u : 0u;
+    }
+    const unsigned long long keep_incl = block_inclusive_sum<unsigned long long>(nkeep, wbuf);
+    int64_t pos = static_cast<int64_t>(keep0 + keep_incl - nkeep);
+#pragma unroll
+    for (int it = 0; it < kHeadItems; ++it)
+      if (keep_bits & (1u << it)) out[pos++] = static_cast<int32_t>(j0 + it);
+    if (threadIdx.x == kHeadThreads - 1) {               // after every thread read the carries
+      s_keep = keep0 + keep_incl;
+      s_eq = eq0 + eq_incl;
+    }
+    __syncthreads();
+  }
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
@@ -337,6 +457,20 @@ cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int mode, int6
   uint32_t* cbase = reinterpret_cast<uint32_t*>(base + lay.off_cbase);
   unsigned long long* head_eq = reinterpret_cast<unsigned long long*>(base + lay.off_head_eq);
   unsigned long long* head_base = reinterpret_cast<unsigned long long*>(base + lay.off_head_base);
+  if (mode == KVZ_PER_HEAD && (n_c <= kHeadStageMax || B >= 128)) {
+    if (n_c <= kHeadStageMax) {
+      const int smem = static_cast<int>(n_c * 4);
+      cudaError_t e = cudaFuncSetAttribute(sel_head_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kHeadStageMax * 4));
+      if (e != cudaSuccess) return e;
+      sel_head_kernel<true><<<static_cast<unsigned>(B), kHeadThreads, smem, stream>>>(S, B, n_c, k, idx, counts,
+                                                                                    offsets, status);
+    } else {
+      sel_head_kernel<false><<<static_cast<unsigned>(B), kHeadThreads, 0, stream>>>(S, B, n_c, k, idx, counts,
+                                                                                   offsets, status);
+    }
+    return cudaGetLastError();
+  }
   const int nseg = mode == KVZ_GLOBAL ? 1 : static_cast<int>(B);
   const int nchunk = static_cast<int>((n_c + kSelChunk - 1) / kSelChunk);
   const dim3 grid(static_cast<unsigned>(nchunk), static_cast<unsigned>(B));

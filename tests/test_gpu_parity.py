@@ -121,7 +121,7 @@ def test_llama8b_layer_full_matches_oracle():
 # ---------------------------------------------------------------------------
 # Selection (bit-exact on identical fp32 scores)
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("B,n_c", [(1, 1), (1, 100), (3, 4097), (8, 8192), (5, 12345), (2, 70000)])
+@pytest.mark.parametrize("B,n_c", [(1, 1), (1, 100), (3, 4097), (8, 8192), (5, 12345), (2, 70000), (130, 50000)])
 @pytest.mark.parametrize("ratio", [0.0, 0.1, 0.3, 0.5, 1.0])
 @pytest.mark.parametrize("mode", ["per_head", "global"])
 def test_select_matches_oracle(B, n_c, ratio, mode):
@@ -142,6 +142,19 @@ def test_select_all_ties_takes_lowest_indices():
     k = orc.keep_count(20000, 0.3)
     assert counts.cpu().tolist() == [5000, 1000, 0, 0]
     np.testing.assert_array_equal(idx.cpu().numpy()[:k], np.r_[np.arange(5000), np.arange(1000)])
+
+
+@pytest.mark.parametrize("n_c,ratio", [(30000, 0.37), (49152, 0.5), (60000, 0.05)])
+def test_select_per_head_ties_across_tiles(n_c, ratio):
+    """Four score levels: the threshold's ties span several write tiles of
+    the one-CTA-per-head path (and the multi-kernel path past its limit)."""
+    g = torch.Generator(device="cuda").manual_seed(n_c)
+    S = torch.randint(0, 4, (3, n_c), generator=g, device="cuda").float() / 4
+    idx, counts, offsets = kvz.kvz_select(S, ratio, "per_head")
+    ri, rc, ro = orc.select(S.cpu().numpy(), ratio, "per_head")
+    np.testing.assert_array_equal(counts.cpu().numpy(), rc)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), ro)
+    np.testing.assert_array_equal(idx.cpu().numpy()[: len(ri)], ri)
 
 
 def test_select_reports_invalid_scores():
