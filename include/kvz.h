@@ -239,6 +239,40 @@ kvz_status kvz_compact(const void* K, const void* V, int64_t B, int64_t n_c,
                        void* workspace, size_t workspace_bytes,
                        int32_t* d_status, cudaStream_t stream);
 
+/* ------------------------------------------------------------------------ */
+/* End to end from host memory.                                              */
+/*                                                                          */
+/* The whole path of one context (kvz_score, then kvz_select, then an        */
+/* out-of-place kvz_compact into a packed cache) with inputs read from and   */
+/* results written to HOST buffers, for callers whose KV cache and queries   */
+/* come from the host.  The host->device copies go by head chunks (at most   */
+/* 8) on `copy_stream`; each chunk is scored on `stream` as soon as it has   */
+/* landed, so the copies overlap the scoring.  V is copied last (only the    */
+/* compaction reads it).  The results come back on `stream`: h_counts[B],    */
+/* h_offsets[B+1], h_idx[kept], hK_out[kept][d], hV_out[kept][d], where      */
+/* kept = B*floor(ratio*n_c) per head or floor(ratio*B*n_c) globally.  The   */
+/* call is asynchronous: the host outputs are valid once `stream` has        */
+/* finished; page-locked host buffers are needed for the copies to overlap  */
+/* (pageable ones work, serialised).  `stream` may equal `copy_stream`      */
+/* (no overlap).  The pages have no counterpart; it composes the three      */
+/* calls above.                                                              */
+/* Layout: hQ [B][G][n_in][d], hK_ctx and hV [B][n_c][d], hK_in [B][n_in][d] */
+/* bf16.  `workspace` is a device buffer of                                  */
+/* kvz_compress_host_workspace_size(...) bytes, 256-byte aligned: device    */
+/* copies of the inputs and outputs plus the scratch of the three calls.     */
+/* Errors: as the three calls, plus KVZ_ERR_INVALID_ARG for a null host      */
+/* pointer or idx_capacity < kept.                                           */
+/* ------------------------------------------------------------------------ */
+size_t kvz_compress_host_workspace_size(int64_t B, int G, int64_t n_c, int64_t n_in, int d, double ratio,
+                                        int mode);
+
+kvz_status kvz_compress_host(const void* hQ, const void* hK_ctx, const void* hK_in, const void* hV,
+                             int64_t B, int G, int64_t n_c, int64_t n_in, int d, float scale,
+                             double ratio, int mode, int32_t* h_idx, int64_t idx_capacity,
+                             int32_t* h_counts, int64_t* h_offsets, void* hK_out, void* hV_out,
+                             void* workspace, size_t workspace_bytes, int32_t* d_status,
+                             cudaStream_t stream, cudaStream_t copy_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -65,6 +65,9 @@ _SIGS = {
     "kvz_select": (_i32, [_vp, _i64, _i64, _f64, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
     "kvz_compact_workspace_size": (_sz, [_i64, _i64]),
     "kvz_compact": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "kvz_compress_host_workspace_size": (_sz, [_i64, _i32, _i64, _i64, _i32, _f64, _i32]),
+    "kvz_compress_host": (_i32, [_vp, _vp, _vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _f64, _i32, _vp, _i64,
+                                 _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp]),
 }
 
 
@@ -271,3 +274,46 @@ def kvz_compact(K, V, idx, counts, offsets, out_offsets=None, K_out=None, V_out=
                                             _ptr(out_offsets), _ptr(K_out), _ptr(V_out), _ptr(workspace), ws_bytes,
                                             _ptr(status), _stream(stream)))
     return K_out, V_out
+
+
+def kvz_compress_host_workspace_size(B: int, G: int, n_c: int, n_in: int, d: int, ratio: float, mode) -> int:
+    return lib().kvz_compress_host_workspace_size(B, G, n_c, n_in, d, float(ratio), _mode(mode))
+
+
+def kvz_compress_host(Q, K_ctx, K_in, V, ratio: float, mode="per_head", scale: Optional[float] = None, out=None,
+                      workspace=None, status=None, stream=None, copy_stream=None):
+    """The whole path of one context from host tensors to host tensors
+    (score, select, out-of-place compact); returns a dict with ``idx``,
+    ``counts``, ``offsets``, ``K_out`` and ``V_out`` (CPU tensors, valid once
+    ``stream`` has finished).  Inputs should be page-locked for the copies to
+    overlap the scoring; ``out`` may pass preallocated (pinned) outputs."""
+    for t in (Q, K_ctx, K_in, V):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("kvz_compress_host: Q, K_ctx, K_in and V must be contiguous bfloat16 CPU tensors")
+    _need_cuda(workspace, status)
+    B, G, n_in, d = Q.shape
+    n_c = K_ctx.shape[1]
+    if K_ctx.shape != (B, n_c, d) or V.shape != (B, n_c, d) or K_in.shape != (B, n_in, d):
+        raise ValueError("kvz_compress_host: shapes must be Q [B,G,n_in,d], K_ctx/V [B,n_c,d], K_in [B,n_in,d]")
+    m = _mode(mode)
+    k = kvz_keep_count(B * n_c if m == GLOBAL else n_c, ratio)
+    kept = k if m == GLOBAL else B * k
+    if out is None:
+        pin = Q.is_pinned()
+        out = {"idx": torch.empty(max(kept, 1), dtype=torch.int32, pin_memory=pin),
+               "counts": torch.empty(B, dtype=torch.int32, pin_memory=pin),
+               "offsets": torch.empty(B + 1, dtype=torch.int64, pin_memory=pin),
+               "K_out": torch.empty((max(kept, 1), d), dtype=torch.bfloat16, pin_memory=pin),
+               "V_out": torch.empty((max(kept, 1), d), dtype=torch.bfloat16, pin_memory=pin)}
+    if workspace is None:
+        workspace = torch.empty(kvz_compress_host_workspace_size(B, G, n_c, n_in, d, ratio, m), dtype=torch.uint8,
+                                device="cuda")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    st = _stream(stream)
+    cst = _stream(copy_stream) if copy_stream is not None else st
+    _check("kvz_compress_host", lib().kvz_compress_host(
+        _ptr(Q), _ptr(K_ctx), _ptr(K_in), _ptr(V), B, G, n_c, n_in, d, float(scale), float(ratio), m,
+        _ptr(out["idx"]), out["idx"].numel(), _ptr(out["counts"]), _ptr(out["offsets"]), _ptr(out["K_out"]),
+        _ptr(out["V_out"]), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status), st, cst))
+    return out

@@ -314,3 +314,156 @@ kvz_status kvz_compact(const void* K, const void* V, int64_t B, int64_t n_c, int
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// End to end from host memory: one context's inputs are copied in by head
+// chunks on a copy stream, each chunk is scored as soon as it lands, then
+// selection, compaction and the copies of the results back to the host run
+// on the compute stream.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t kHostChunks = 8;   // head chunks the input copies are split into
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct HostPlan {
+  int64_t k, kept, chunk_heads;
+  size_t off_q, off_kc, off_ki, off_v, off_s, off_lse, lse_bytes, off_sel, sel_bytes, off_idx, off_cnt, off_off,
+      off_ko, off_vo, bytes;
+};
+
+bool host_plan(int64_t B, int G, int64_t n_c, int64_t n_in, int d, double ratio, int mode, HostPlan* p) {
+  if (B < 1 || G < 1 || n_c < 1 || n_in < 1 || (d != 64 && d != 128)) return false;
+  if (!(ratio >= 0.0 && ratio <= 1.0) || (mode != KVZ_PER_HEAD && mode != KVZ_GLOBAL)) return false;
+  if (B > 65535 || n_c > kMaxRows || n_in > kMaxRows || B * n_c >= (int64_t(1) << 32)) return false;
+  p->k = kvz_keep_count(mode == KVZ_GLOBAL ? B * n_c : n_c, ratio);
+  p->kept = mode == KVZ_GLOBAL ? p->k : B * p->k;
+  const int64_t nchunks = B < kHostChunks ? B : kHostChunks;
+  p->chunk_heads = (B + nchunks - 1) / nchunks;
+  const size_t row = static_cast<size_t>(d) * 2;
+  const size_t kept1 = static_cast<size_t>(p->kept > 0 ? p->kept : 1);
+  size_t o = 0;
+  p->off_q = o;   o = align256(o + static_cast<size_t>(B * G * n_in) * row);
+  p->off_kc = o;  o = align256(o + static_cast<size_t>(B * n_c) * row);
+  p->off_ki = o;  o = align256(o + static_cast<size_t>(B * n_in) * row);
+  p->off_v = o;   o = align256(o + static_cast<size_t>(B * n_c) * row);
+  p->off_s = o;   o = align256(o + static_cast<size_t>(B * n_c) * 4);
+  p->lse_bytes = kvz_score_workspace_size(p->chunk_heads, G, n_in, 0);
+  p->off_lse = o; o = align256(o + p->lse_bytes);
+  p->sel_bytes = kvz_select_workspace_size(B, n_c, mode);
+  p->off_sel = o; o = align256(o + p->sel_bytes);
+  p->off_idx = o; o = align256(o + kept1 * 4);
+  p->off_cnt = o; o = align256(o + static_cast<size_t>(B) * 4);
+  p->off_off = o; o = align256(o + static_cast<size_t>(B + 1) * 8);
+  p->off_ko = o;  o = align256(o + kept1 * row);
+  p->off_vo = o;  o = align256(o + kept1 * row);
+  p->bytes = o;
+  return true;
+}
+
+// Events of one call; released when the call returns (a recorded event may
+// be destroyed before it completes).
+struct CallEvents {
+  cudaEvent_t ev[kHostChunks + 2] = {};
+  int n = 0;
+  cudaError_t make(int count) {
+    for (; n < count; ++n) {
+      cudaError_t e = cudaEventCreateWithFlags(&ev[n], cudaEventDisableTiming);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
+  ~CallEvents() {
+    for (int i = 0; i < n; ++i) cudaEventDestroy(ev[i]);
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+size_t kvz_compress_host_workspace_size(int64_t B, int G, int64_t n_c, int64_t n_in, int d, double ratio,
+                                        int mode) {
+  HostPlan p;
+  return host_plan(B, G, n_c, n_in, d, ratio, mode, &p) ? p.bytes : 0;
+}
+
+kvz_status kvz_compress_host(const void* hQ, const void* hK_ctx, const void* hK_in, const void* hV, int64_t B,
+                             int G, int64_t n_c, int64_t n_in, int d, float scale, double ratio, int mode,
+                             int32_t* h_idx, int64_t idx_capacity, int32_t* h_counts, int64_t* h_offsets,
+                             void* hK_out, void* hV_out, void* workspace, size_t workspace_bytes,
+                             int32_t* d_status, cudaStream_t stream, cudaStream_t copy_stream) {
+  if (hQ == nullptr || hK_ctx == nullptr || hK_in == nullptr || hV == nullptr || h_counts == nullptr ||
+      h_offsets == nullptr)
+    return KVZ_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return KVZ_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale) || !(scale > 0.0f)) return KVZ_ERR_INVALID_ARG;
+  HostPlan p;
+  if (!host_plan(B, G, n_c, n_in, d, ratio, mode, &p)) return KVZ_ERR_INVALID_ARG;
+  if (idx_capacity < p.kept || (p.kept > 0 && (h_idx == nullptr || hK_out == nullptr || hV_out == nullptr)))
+    return KVZ_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < p.bytes) return KVZ_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return KVZ_ERR_ALIGNMENT;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* dQ = ws + p.off_q;
+  uint8_t* dKc = ws + p.off_kc;
+  uint8_t* dKi = ws + p.off_ki;
+  uint8_t* dV = ws + p.off_v;
+  float* dS = reinterpret_cast<float*>(ws + p.off_s);
+  int32_t* d_idx = reinterpret_cast<int32_t*>(ws + p.off_idx);
+  int32_t* d_cnt = reinterpret_cast<int32_t*>(ws + p.off_cnt);
+  int64_t* d_off = reinterpret_cast<int64_t*>(ws + p.off_off);
+  const size_t row = static_cast<size_t>(d) * 2;
+  const int64_t nchunks = (B + p.chunk_heads - 1) / p.chunk_heads;
+
+  CallEvents evs;
+  if (evs.make(static_cast<int>(nchunks) + 2) != cudaSuccess) return KVZ_ERR_CUDA;
+  cudaEvent_t ev_start = evs.ev[0], ev_v = evs.ev[1];
+  // the copies must not overwrite the workspace while earlier work on `stream` reads it
+  if (cudaEventRecord(ev_start, stream) != cudaSuccess || cudaStreamWaitEvent(copy_stream, ev_start, 0) != cudaSuccess)
+    return KVZ_ERR_CUDA;
+  auto h2d = [&](uint8_t* dst, const void* src, size_t off, size_t bytes) {
+    return cudaMemcpyAsync(dst + off, static_cast<const uint8_t*>(src) + off, bytes, cudaMemcpyHostToDevice,
+                           copy_stream);
+  };
+  for (int64_t c = 0; c < nchunks; ++c) {
+    const int64_t h0 = c * p.chunk_heads, nb = (h0 + p.chunk_heads <= B ? p.chunk_heads : B - h0);
+    if (h2d(dQ, hQ, static_cast<size_t>(h0 * G * n_in) * row, static_cast<size_t>(nb * G * n_in) * row) ||
+        h2d(dKc, hK_ctx, static_cast<size_t>(h0 * n_c) * row, static_cast<size_t>(nb * n_c) * row) ||
+        h2d(dKi, hK_in, static_cast<size_t>(h0 * n_in) * row, static_cast<size_t>(nb * n_in) * row) ||
+        cudaEventRecord(evs.ev[2 + c], copy_stream) != cudaSuccess)
+      return KVZ_ERR_CUDA;
+  }
+  if (h2d(dV, hV, 0, static_cast<size_t>(B * n_c) * row) || cudaEventRecord(ev_v, copy_stream) != cudaSuccess)
+    return KVZ_ERR_CUDA;
+
+  for (int64_t c = 0; c < nchunks; ++c) {
+    const int64_t h0 = c * p.chunk_heads, nb = (h0 + p.chunk_heads <= B ? p.chunk_heads : B - h0);
+    if (cudaStreamWaitEvent(stream, evs.ev[2 + c], 0) != cudaSuccess) return KVZ_ERR_CUDA;
+    kvz_status st = kvz_score(dQ + static_cast<size_t>(h0 * G * n_in) * row, dKc + static_cast<size_t>(h0 * n_c) * row,
+                              dKi + static_cast<size_t>(h0 * n_in) * row, nb, G, n_c, n_in, d, scale, 0,
+                              dS + h0 * n_c, ws + p.off_lse, p.lse_bytes, d_status, stream);
+    if (st != KVZ_OK) return st;
+  }
+  kvz_status st = kvz_select(dS, B, n_c, ratio, mode, d_idx, p.kept > 0 ? p.kept : 1, d_cnt, d_off,
+                             ws + p.off_sel, p.sel_bytes, d_status, stream);
+  if (st != KVZ_OK) return st;
+  if (cudaStreamWaitEvent(stream, ev_v, 0) != cudaSuccess) return KVZ_ERR_CUDA;
+  st = kvz_compact(dKc, dV, B, n_c, d, d_idx, d_cnt, d_off, nullptr, ws + p.off_ko, ws + p.off_vo, nullptr, 0,
+                   d_status, stream);
+  if (st != KVZ_OK) return st;
+  const size_t kept = static_cast<size_t>(p.kept);
+  if (cudaMemcpyAsync(h_counts, d_cnt, static_cast<size_t>(B) * 4, cudaMemcpyDeviceToHost, stream) ||
+      cudaMemcpyAsync(h_offsets, d_off, static_cast<size_t>(B + 1) * 8, cudaMemcpyDeviceToHost, stream))
+    return KVZ_ERR_CUDA;
+  if (kept > 0 &&
+      (cudaMemcpyAsync(h_idx, d_idx, kept * 4, cudaMemcpyDeviceToHost, stream) ||
+       cudaMemcpyAsync(hK_out, ws + p.off_ko, kept * row, cudaMemcpyDeviceToHost, stream) ||
+       cudaMemcpyAsync(hV_out, ws + p.off_vo, kept * row, cudaMemcpyDeviceToHost, stream)))
+    return KVZ_ERR_CUDA;
+  return KVZ_OK;
+}
+
+}  // extern "C"

@@ -135,3 +135,28 @@ def test_compact_rejections(lib):
     assert call(Ko_=K, Vo_=V, wsb=8) == WS
     assert lib.kvz_compact(vp(K), vp(V), B, n_c, d, None, vp(cnt), vp(off), None, vp(Ko), vp(Vo), None, 0,
                            None, None) == INVALID
+
+
+def test_compress_host_rejections(lib):
+    b = Bufs()
+    B, G, n_c, n_in, d = 2, 2, 1000, 1032, 128
+    hQ, hK, hKi, hV = (ctypes.create_string_buffer(16) for _ in range(4))   # never read: every call is rejected
+    hidx, hcnt, hoff, hko, hvo = (ctypes.create_string_buffer(16) for _ in range(5))
+    need = lib.kvz_compress_host_workspace_size(B, G, n_c, n_in, d, 0.3, 0)
+    assert need > 2 * (B * G * n_in + 2 * B * n_c + B * n_in) * d     # holds the device copies of the inputs
+    ws = b.get(need)
+    kept = B * 300
+
+    def call(d_=d, scale=0.1, ratio=0.3, mode=0, cap=kept, wsb=need, ws_=ws, q=hQ):
+        return lib.kvz_compress_host(q, hK, hKi, hV, B, G, n_c, n_in, d_, scale, ratio, mode, hidx, cap, hcnt, hoff,
+                                     hko, hvo, vp(ws_) if ws_ else None, wsb, None, None, None)
+
+    assert call(d_=96) == UNSUPPORTED
+    assert call(scale=0.0) == INVALID
+    assert call(ratio=1.5) == INVALID
+    assert call(mode=2) == INVALID
+    assert call(cap=kept - 1) == INVALID
+    assert call(q=None) == INVALID
+    assert call(wsb=need - 1) == WS
+    assert call(ws_=0) == WS
+    assert lib.kvz_compress_host_workspace_size(B, G, n_c, n_in, 96, 0.3, 0) == 0

@@ -283,3 +283,38 @@ def test_pipeline_selection_and_compaction_exact(name):
         oi, _, _ = orc.select(ref_S, w.ratio, w.mode)
         overlap = len(set(oi.tolist()) & set(ri.tolist())) / max(1, len(set(oi.tolist()) | set(ri.tolist())))
         assert overlap > 0.9
+
+
+# ---------------------------------------------------------------------------
+# End to end from host memory
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,G,n_c,n_prompt,d,ratio,mode,pinned", [
+    (1, 4, 256, 16, 64, 0.3, "per_head", True),
+    (11, 2, 700, 32, 128, 0.3, "per_head", True),     # 11 heads in chunks of 2 (the last chunk has 1)
+    (11, 2, 700, 32, 128, 0.2, "global", False),      # pageable host memory: correct, serialised
+    (3, 4, 2000, 40, 128, 0.0, "per_head", True),     # nothing kept
+])
+def test_compress_host_matches_device_path(B, G, n_c, n_prompt, d, ratio, mode, pinned):
+    x = _inputs(B, G, n_c, n_prompt, d, seed=B * 31 + n_c)
+    V = torch.randn((B, n_c, d), generator=torch.Generator(device="cuda").manual_seed(5), device="cuda")
+    V = V.to(torch.bfloat16)
+    host = {n: (t.cpu().pin_memory() if pinned else t.cpu()) for n, t in
+            (("Q", x["Q"]), ("K_ctx", x["K_ctx"]), ("K_in", x["K_in"]), ("V", V))}
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    copy_stream = torch.cuda.Stream()
+    out = kvz.kvz_compress_host(host["Q"], host["K_ctx"], host["K_in"], host["V"], ratio, mode, status=status,
+                                copy_stream=copy_stream)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    S = kvz.kvz_score(x["Q"], x["K_ctx"], x["K_in"])
+    idx, counts, offsets = kvz.kvz_select(S, ratio, mode)
+    total = int(offsets[-1].item())
+    Ko, Vo = kvz.kvz_compact(x["K_ctx"], V, idx, counts, offsets, out_rows=max(total, 1))
+    torch.cuda.synchronize()
+    assert torch.equal(out["counts"], counts.cpu()) and torch.equal(out["offsets"], offsets.cpu())
+    assert torch.equal(out["idx"][:total], idx.cpu()[:total])
+    assert torch.equal(out["K_out"][:total].view(torch.int16), Ko[:total].cpu().view(torch.int16))
+    assert torch.equal(out["V_out"][:total].view(torch.int16), Vo[:total].cpu().view(torch.int16))
+    # and the selection is the oracle's on these scores
+    ri, rc, ro = orc.select(S.cpu().numpy(), ratio, mode)
+    np.testing.assert_array_equal(out["idx"].numpy()[:total], ri)
