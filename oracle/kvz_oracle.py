@@ -40,6 +40,8 @@ __all__ = [
     "row_logits",
     "row_lse",
     "score",
+    "chunk_bounds",
+    "score_chunked",
     "keep_count",
     "select",
     "compact",
@@ -127,6 +129,54 @@ def score(Q, K_ctx, K_in, scale, rows=None, row_block=256):
         lse = m + np.log(np.sum(np.exp(Z - m), axis=2, keepdims=True))
         A_ctx = np.exp(Z[:, :, :n_c] - lse)                  # slice after softmax
         S = np.maximum(S, A_ctx.max(axis=(0, 1)))
+    return S
+
+
+# ---------------------------------------------------------------------------
+# Chunked scoring (KVzip §3.4 "technical challenges": chunk-based scoring)
+# ---------------------------------------------------------------------------
+def chunk_bounds(n_c, m):
+    """Context positions [c0, c1) of each chunk: fixed length m, the last one
+    shorter when m does not divide n_c."""
+    n_c, m = int(n_c), int(m)
+    if n_c < 1 or m < 1:
+        raise ValueError("n_c and m must be positive")
+    return [(c0, min(n_c, c0 + m)) for c0 in range(0, n_c, m)]
+
+
+def score_chunked(Q_chunks, K_ctx, K_in_chunks, scale, m):
+    """Chunked importance scores S[n_c] (KVzip §3.4).
+
+    The context is cut into chunks of m tokens.  Chunk t (positions [c0, c1),
+    m_t = c1 - c0 tokens) is appended to the repeat prompt and reconstructed
+    on its own: its input has n_in_t = n_prompt + m_t tokens with grouped
+    queries Q_chunks[t] [G, n_in_t, d] and input keys K_in_chunks[t]
+    [n_in_t, d], and its attention matrix is n_in_t x (m_t + n_in_t): the
+    rows see only the chunk's own m_t cache keys K_ctx[c0:c1] plus the input
+    keys (causally, own position included), and each row is normalised over
+    exactly those keys.  S on the chunk's positions is the max over (g, i) of
+    the rows' values on the chunk's cache keys.
+    """
+    K_ctx = np.asarray(K_ctx, dtype=np.float64)
+    bounds = chunk_bounds(K_ctx.shape[0], m)
+    if len(Q_chunks) != len(bounds) or len(K_in_chunks) != len(bounds):
+        raise ValueError("one Q and one K_in block per chunk")
+    S = np.zeros(K_ctx.shape[0], dtype=np.float64)
+    scale = float(scale)
+    for (c0, c1), Qt, Kit in zip(bounds, Q_chunks, K_in_chunks):
+        Qt = np.asarray(Qt, dtype=np.float64)
+        Kit = np.asarray(Kit, dtype=np.float64)
+        G, n_in, d = Qt.shape
+        if Kit.shape != (n_in, d) or n_in < c1 - c0:
+            raise ValueError("chunk inputs must be [G, n_prompt + m_t, d] and [n_prompt + m_t, d]")
+        keys = np.concatenate([K_ctx[c0:c1], Kit], axis=0)     # m_t cache keys, then the input keys
+        mt = c1 - c0
+        for g in range(G):
+            for i in range(n_in):
+                z = scale * (keys[: mt + i + 1] @ Qt[g, i])
+                zmax = np.max(z)
+                a = np.exp(z - zmax) / np.sum(np.exp(z - zmax))
+                S[c0:c1] = np.maximum(S[c0:c1], a[:mt])
     return S
 
 

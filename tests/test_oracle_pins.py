@@ -280,3 +280,94 @@ def test_compact_gathers_in_order():
     for b in range(B):
         np.testing.assert_array_equal(K2[b * n_c: b * n_c + counts[b]],
                                       K_out[offsets[b]:offsets[b + 1]])
+
+
+# --------------------------------------------------------------------------
+# Chunked scoring (KVzip §3.4): each chunk is reconstructed on its own, its
+# rows normalised over the chunk's m_t cache keys plus the visible input keys
+# --------------------------------------------------------------------------
+def _chunked_inputs(rng, G, n_c, n_prompt, m, d, scale_keys=1.0):
+    K_ctx = rng.standard_normal((n_c, d)) * scale_keys
+    Qs, Kis = [], []
+    for c0, c1 in orc.chunk_bounds(n_c, m):
+        n_in = n_prompt + (c1 - c0)
+        Qs.append(rng.standard_normal((G, n_in, d)))
+        Kis.append(rng.standard_normal((n_in, d)) * scale_keys)
+    return Qs, K_ctx, Kis
+
+
+def test_chunk_bounds():
+    assert orc.chunk_bounds(7, 3) == [(0, 3), (3, 6), (6, 7)]
+    assert orc.chunk_bounds(6, 3) == [(0, 3), (3, 6)]
+    assert orc.chunk_bounds(5, 8) == [(0, 5)]
+    assert orc.chunk_bounds(170000, 2048)[-1] == (169984, 170000)     # 83 full chunks and a 16-token tail
+
+
+@pytest.mark.parametrize("G,n_c,n_prompt,m,d", [(2, 10, 3, 4, 8), (1, 9, 0, 3, 4), (3, 20, 5, 7, 16)])
+def test_chunked_identical_keys_give_one_over_chunk_plus_one(G, n_c, n_prompt, m, d):
+    # every row of chunk t is uniform over its m_t + i + 1 visible keys, so the
+    # chunk's cache keys score 1 / (m_t + 1): the normaliser is the chunk's, not n_c
+    rng = np.random.default_rng(21)
+    v = rng.standard_normal(d)
+    Qs, _, Kis = _chunked_inputs(rng, G, n_c, n_prompt, m, d)
+    K_ctx = np.tile(v, (n_c, 1))
+    Kis = [np.tile(v, (k.shape[0], 1)) for k in Kis]
+    S = orc.score_chunked(Qs, K_ctx, Kis, 0.41, m)
+    want = np.concatenate([np.full(c1 - c0, 1.0 / (c1 - c0 + 1)) for c0, c1 in orc.chunk_bounds(n_c, m)])
+    np.testing.assert_allclose(S, want, rtol=1e-13)
+
+
+def test_chunked_single_key_chunks_are_two_way_softmaxes():
+    # m = 1, no prompt, G = 1: chunk j has one cache key k_j and one input row q_j
+    # that sees k_j and its own input key: S_j = e^{s k_j.q_j} / (e^{s k_j.q_j} + e^{s kin_j.q_j})
+    rng = np.random.default_rng(22)
+    n_c, d, s = 6, 5, 0.7
+    Qs, K_ctx, Kis = _chunked_inputs(rng, 1, n_c, 0, 1, d)
+    S = orc.score_chunked(Qs, K_ctx, Kis, s, 1)
+    for j in range(n_c):
+        a, b = s * K_ctx[j] @ Qs[j][0, 0], s * Kis[j][0] @ Qs[j][0, 0]
+        assert S[j] == pytest.approx(1.0 / (1.0 + math.exp(b - a)), rel=1e-14)
+
+
+def test_chunked_with_one_chunk_is_the_unchunked_score():
+    rng = np.random.default_rng(23)
+    G, n_c, n_prompt, d = 3, 17, 4, 8
+    Qs, K_ctx, Kis = _chunked_inputs(rng, G, n_c, n_prompt, 64, d)
+    assert len(Qs) == 1
+    np.testing.assert_allclose(orc.score_chunked(Qs, K_ctx, Kis, 0.3, 64), orc.score(Qs[0], K_ctx, Kis[0], 0.3),
+                               rtol=1e-13, atol=0)
+
+
+def test_chunked_scores_are_local_to_their_chunk():
+    rng = np.random.default_rng(24)
+    G, n_c, n_prompt, m, d = 2, 11, 3, 4, 8
+    Qs, K_ctx, Kis = _chunked_inputs(rng, G, n_c, n_prompt, m, d)
+    S0 = orc.score_chunked(Qs, K_ctx, Kis, 0.5, m)
+    Qs[1] = Qs[1] * -2.0                     # chunk 1 = positions [4, 8)
+    Kis[1] = Kis[1] + 1.0
+    S1 = orc.score_chunked(Qs, K_ctx, Kis, 0.5, m)
+    assert np.array_equal(S0[:4], S1[:4]) and np.array_equal(S0[8:], S1[8:])
+    assert not np.allclose(S0[4:8], S1[4:8])
+    assert np.all((S1 >= 0) & (S1 <= 1))
+
+
+def test_chunked_brute_force_mpmath():
+    # n_c = 7 in chunks of 3 (the last holds 1 key), 50-digit evaluation of
+    # the per-chunk softmax written out key by key
+    rng = np.random.default_rng(25)
+    G, n_c, n_prompt, m, d, scale = 2, 7, 2, 3, 4, 0.6
+    Qs, K_ctx, Kis = _chunked_inputs(rng, G, n_c, n_prompt, m, d)
+    S = orc.score_chunked(Qs, K_ctx, Kis, scale, m)
+    mpmath.mp.dps = 50
+    sc = mpmath.mpf(scale)
+    for (c0, c1), Qt, Kit in zip(orc.chunk_bounds(n_c, m), Qs, Kis):
+        keys = [list(map(mpmath.mpf, k)) for k in K_ctx[c0:c1]] + [list(map(mpmath.mpf, k)) for k in Kit]
+        mt = c1 - c0
+        for j in range(mt):
+            best = mpmath.mpf(0)
+            for g in range(G):
+                for i in range(Qt.shape[1]):
+                    q = list(map(mpmath.mpf, Qt[g, i]))
+                    w = [mpmath.e ** (sc * mpmath.fsum(a * b for a, b in zip(q, keys[u]))) for u in range(mt + i + 1)]
+                    best = max(best, w[j] / mpmath.fsum(w))
+            assert abs(S[c0 + j] - float(best)) <= 1e-13 * float(best)
