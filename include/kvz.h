@@ -240,6 +240,33 @@ kvz_status kvz_compact(const void* K, const void* V, int64_t B, int64_t n_c,
                        int32_t* d_status, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Chunked scoring (KVzip §3.4, "chunk-based scoring").                      */
+/*                                                                          */
+/* The context is cut into chunks of m tokens (the last one is n_c mod m     */
+/* tokens when m does not divide n_c).  Chunk t, context positions           */
+/* [c0, c1), m_t = c1 - c0, is appended to the repeat prompt and             */
+/* reconstructed on its own: its input has n_in_t = n_prompt + m_t tokens    */
+/* with their own grouped queries and input keys, and its rows see only the  */
+/* chunk's m_t cache keys K_ctx[c0:c1] plus the input keys (causally), each  */
+/* row normalised over exactly those keys: an n_in_t x (m_t + n_in_t)        */
+/* attention matrix per chunk.  S[c0 + j] is the max over (g, i) of chunk    */
+/* t's row values on its cache key j.  Cost is linear in n_c.                */
+/* Layout (bf16; T = n_c / m full chunks, m_last = n_c % m):                 */
+/*   Q         [B][T][G][n_prompt + m][d]       (NULL when T == 0)           */
+/*   Q_tail    [B][G][n_prompt + m_last][d]     (NULL when m_last == 0)      */
+/*   K_in      [B][T][n_prompt + m][d],  K_in_tail [B][n_prompt + m_last][d] */
+/*   K_ctx     [B][n_c][d];  S [B][n_c] fp32 (overwritten).                  */
+/* Workspace: kvz_score_chunked_workspace_size(...) bytes (per-row lse2).    */
+/* Limits as kvz_score; n_prompt >= 0, m >= 1.                               */
+/* ------------------------------------------------------------------------ */
+size_t kvz_score_chunked_workspace_size(int64_t B, int G, int64_t n_c, int64_t n_prompt, int64_t m);
+
+kvz_status kvz_score_chunked(const void* Q, const void* Q_tail, const void* K_ctx, const void* K_in,
+                             const void* K_in_tail, int64_t B, int G, int64_t n_c, int64_t n_prompt,
+                             int64_t m, int d, float scale, float* S, void* workspace,
+                             size_t workspace_bytes, int32_t* d_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* End to end from host memory.                                              */
 /*                                                                          */
 /* The whole path of one context (kvz_score, then kvz_select, then an        */

@@ -65,6 +65,9 @@ _SIGS = {
     "kvz_select": (_i32, [_vp, _i64, _i64, _f64, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
     "kvz_compact_workspace_size": (_sz, [_i64, _i64]),
     "kvz_compact": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "kvz_score_chunked_workspace_size": (_sz, [_i64, _i32, _i64, _i64, _i64]),
+    "kvz_score_chunked": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i64, _i64, _i64, _i32, _f32, _vp, _vp, _sz,
+                                 _vp, _vp]),
     "kvz_compress_host_workspace_size": (_sz, [_i64, _i32, _i64, _i64, _i32, _f64, _i32]),
     "kvz_compress_host": (_i32, [_vp, _vp, _vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _f64, _i32, _vp, _i64,
                                  _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp]),
@@ -317,3 +320,40 @@ def kvz_compress_host(Q, K_ctx, K_in, V, ratio: float, mode="per_head", scale: O
         _ptr(out["idx"]), out["idx"].numel(), _ptr(out["counts"]), _ptr(out["offsets"]), _ptr(out["K_out"]),
         _ptr(out["V_out"]), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status), st, cst))
     return out
+
+
+def kvz_score_chunked_workspace_size(B: int, G: int, n_c: int, n_prompt: int, m: int) -> int:
+    return lib().kvz_score_chunked_workspace_size(B, G, n_c, n_prompt, m)
+
+
+def kvz_score_chunked(Q, Q_tail, K_ctx, K_in, K_in_tail, m: int, scale: Optional[float] = None, S=None,
+                      workspace=None, status=None, stream=None):
+    """Chunked importance scores (KVzip §3.4); returns S [B, n_c] fp32.
+
+    Q [B, T, G, n_prompt+m, d] and K_in [B, T, n_prompt+m, d] hold the T full
+    chunks' inputs, Q_tail / K_in_tail the shorter last chunk's (None when m
+    divides n_c); K_ctx is [B, n_c, d]."""
+    _need_cuda(Q, Q_tail, K_ctx, K_in, K_in_tail, S, workspace, status)
+    B, n_c, d = K_ctx.shape
+    T, m_last = n_c // m, n_c % m
+    ref = Q if Q is not None else Q_tail
+    G = ref.shape[-3]
+    n_prompt = (Q.shape[-2] - m) if Q is not None else (Q_tail.shape[-2] - m_last)
+    if T > 0 and (Q is None or Q.shape != (B, T, G, n_prompt + m, d) or K_in is None
+                  or K_in.shape != (B, T, n_prompt + m, d)):
+        raise ValueError("kvz_score_chunked: Q must be [B, T, G, n_prompt+m, d] and K_in [B, T, n_prompt+m, d]")
+    if m_last > 0 and (Q_tail is None or Q_tail.shape != (B, G, n_prompt + m_last, d) or K_in_tail is None
+                       or K_in_tail.shape != (B, n_prompt + m_last, d)):
+        raise ValueError("kvz_score_chunked: Q_tail must be [B, G, n_prompt+m_last, d] and K_in_tail "
+                         "[B, n_prompt+m_last, d]")
+    if S is None:
+        S = torch.empty((B, n_c), dtype=torch.float32, device=K_ctx.device)
+    if workspace is None:
+        workspace = torch.empty(kvz_score_chunked_workspace_size(B, G, n_c, n_prompt, m), dtype=torch.uint8,
+                                device=K_ctx.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check("kvz_score_chunked", lib().kvz_score_chunked(
+        _ptr(Q), _ptr(Q_tail), _ptr(K_ctx), _ptr(K_in), _ptr(K_in_tail), B, G, n_c, n_prompt, m, d, float(scale),
+        _ptr(S), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)))
+    return S

@@ -171,8 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(a_full, kNumA * L::A_TILE);
       for (int a = 0; a < kNumA; ++a)
         for (int kb = 0; kb < L::KB; ++kb)
-          tma_load_3d(sA + a * L::A_TILE + kb * L::A_BLK, &tmKc, a_full, kb * 64,
-                      static_cast<int>(key0 + a * kKeys), b);
+          tma_load_4d(sA + a * L::A_TILE + kb * L::A_BLK, &tmKc, a_full, kb * 64,
+                      static_cast<int>(key0 + a * kKeys), b % p.T, b / p.T);
       for (int n = 0; n < ntile; ++n) {
         const int s = n % L::QST;
         const uint32_t use = static_cast<uint32_t>(n / L::QST);
@@ -300,7 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && j < p.n_c) {
       const float sj = exp2f(p.c2 * fmaxf(y0, y1));   // >= +0: its bit pattern orders like the value
-      atomicMax(reinterpret_cast<unsigned int*>(p.S + static_cast<int64_t>(b) * p.n_c + j), __float_as_uint(sj));
+      float* dst = p.S + static_cast<int64_t>(b / p.T) * p.ldS + static_cast<int64_t>(b % p.T) * p.s_block + j;
+      atomicMax(reinterpret_cast<unsigned int*>(dst), __float_as_uint(sj));
     }
   }
 

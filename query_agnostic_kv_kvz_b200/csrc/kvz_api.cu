@@ -49,6 +49,34 @@ bool make_map(CUtensorMap* m, const void* base, int64_t d, int64_t rows, int64_t
   return r == CUDA_SUCCESS;
 }
 
+// 4-D view [head][block][rows][d] of the context keys: `T` blocks of `rows`
+// keys per head, block b of head h starting at row h*head_stride +
+// b*block_stride.  Rows past `rows` read as zeros, so a block never sees the
+// next block's keys.
+bool make_ctx_map(CUtensorMap* m, const void* base, int64_t d, int64_t rows, int64_t T, int64_t heads,
+                  int64_t block_stride, int64_t head_stride) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(T),
+                        static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(block_stride * d * 2),
+                           static_cast<cuuint64_t>(head_stride * d * 2)};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Where the context keys of each problem live: T blocks per head (see
+// LseArgs); the plain score is T = 1 with both strides n_c.
+struct CtxGeom {
+  int T;
+  int64_t block_stride, head_stride;   // in rows
+};
+CtxGeom plain_geom(int64_t n_c) { return CtxGeom{1, n_c, n_c}; }
+
 float log2e_scale(float scale) { return static_cast<float>(static_cast<double>(scale) * 1.4426950408889634); }
 
 kvz_status check_score_common(const void* Q, const void* K_ctx, int64_t B, int G, int64_t n_c, int64_t n_in,
@@ -65,14 +93,16 @@ kvz_status check_score_common(const void* Q, const void* K_ctx, int64_t B, int G
 
 kvz_status run_lse(const void* Q, const void* K_ctx, const void* K_in, int64_t B, int G, int64_t n_c,
                    int64_t n_in, int d, float scale, int64_t i_begin, int64_t i_end, float* lse2, int64_t ld,
-                   int32_t* status, cudaStream_t stream) {
+                   int32_t* status, cudaStream_t stream, CtxGeom geom) {
   CUtensorMap tmQ, tmKc, tmKi;
-  if (!make_map(&tmQ, Q, d, n_in, B * G) || !make_map(&tmKc, K_ctx, d, n_c, B) ||
+  if (!make_map(&tmQ, Q, d, n_in, B * G) ||
+      !make_ctx_map(&tmKc, K_ctx, d, n_c, geom.T, B / geom.T, geom.block_stride, geom.head_stride) ||
       !make_map(&tmKi, K_in, d, n_in, B))
     return KVZ_ERR_CUDA;
   kvz::LseArgs a{};
   a.B = static_cast<int>(B);
   a.G = G;
+  a.T = geom.T;
   a.n_c = n_c;
   a.n_in = n_in;
   a.c2 = log2e_scale(scale);
@@ -87,12 +117,17 @@ kvz_status run_lse(const void* Q, const void* K_ctx, const void* K_in, int64_t B
 
 kvz_status run_colmax(const void* Q, const void* K_ctx, int64_t B, int G, int64_t n_c, int64_t n_in, int d,
                       float scale, int64_t i_begin, int64_t i_end, const float* lse2, int64_t ld, float* S,
-                      int32_t* status, cudaStream_t stream) {
+                      int32_t* status, cudaStream_t stream, CtxGeom geom, int64_t ldS, int64_t s_block) {
   CUtensorMap tmQ, tmKc;
-  if (!make_map(&tmQ, Q, d, n_in, B * G) || !make_map(&tmKc, K_ctx, d, n_c, B)) return KVZ_ERR_CUDA;
+  if (!make_map(&tmQ, Q, d, n_in, B * G) ||
+      !make_ctx_map(&tmKc, K_ctx, d, n_c, geom.T, B / geom.T, geom.block_stride, geom.head_stride))
+    return KVZ_ERR_CUDA;
   kvz::ColArgs a{};
   a.B = static_cast<int>(B);
   a.G = G;
+  a.T = geom.T;
+  a.ldS = ldS;
+  a.s_block = s_block;
   a.n_c = n_c;
   a.c2 = log2e_scale(scale);
   a.i_begin = i_begin;
@@ -140,7 +175,8 @@ kvz_status kvz_score_lse2(const void* Q, const void* K_ctx, const void* K_in, in
   if (!aligned(K_in, 16) || !aligned(lse2, 16) || ld_lse2 % 4 != 0) return KVZ_ERR_ALIGNMENT;
   if (i_begin < 0 || i_begin % 256 != 0 || i_end <= i_begin || i_end > n_in) return KVZ_ERR_INVALID_ARG;
   if (ld_lse2 < roundup(i_end - i_begin, 256)) return KVZ_ERR_INVALID_ARG;
-  return run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i_begin, i_end, lse2, ld_lse2, d_status, stream);
+  return run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i_begin, i_end, lse2, ld_lse2, d_status, stream,
+                 plain_geom(n_c));
 }
 
 kvz_status kvz_score_colmax(const void* Q, const void* K_ctx, int64_t B, int G, int64_t n_c, int64_t n_in, int d,
@@ -153,7 +189,8 @@ kvz_status kvz_score_colmax(const void* Q, const void* K_ctx, int64_t B, int G, 
   if (i_begin < 0 || i_begin % 256 != 0 || i_end <= i_begin || i_end > n_in) return KVZ_ERR_INVALID_ARG;
   if (ld_lse2 < roundup(i_end - i_begin, 256)) return KVZ_ERR_INVALID_ARG;
   if (!accumulate && kvz::launch_fill_f32(S, B * n_c, 0.0f, stream) != cudaSuccess) return KVZ_ERR_CUDA;
-  return run_colmax(Q, K_ctx, B, G, n_c, n_in, d, scale, i_begin, i_end, lse2, ld_lse2, S, d_status, stream);
+  return run_colmax(Q, K_ctx, B, G, n_c, n_in, d, scale, i_begin, i_end, lse2, ld_lse2, S, d_status, stream,
+                    plain_geom(n_c), n_c, n_c);
 }
 
 kvz_status kvz_score(const void* Q, const void* K_ctx, const void* K_in, int64_t B, int G, int64_t n_c,
@@ -173,9 +210,64 @@ kvz_status kvz_score(const void* Q, const void* K_ctx, const void* K_in, int64_t
   if (kvz::launch_fill_f32(S, B * n_c, 0.0f, stream) != cudaSuccess) return KVZ_ERR_CUDA;
   for (int64_t i0 = 0; i0 < n_in; i0 += chunk) {
     const int64_t i1 = i0 + chunk < n_in ? i0 + chunk : n_in;
-    st = run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, d_status, stream);
+    st = run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, d_status, stream, plain_geom(n_c));
     if (st != KVZ_OK) return st;
-    st = run_colmax(Q, K_ctx, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, S, d_status, stream);
+    st = run_colmax(Q, K_ctx, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, S, d_status, stream, plain_geom(n_c),
+                    n_c, n_c);
+    if (st != KVZ_OK) return st;
+  }
+  return KVZ_OK;
+}
+
+size_t kvz_score_chunked_workspace_size(int64_t B, int G, int64_t n_c, int64_t n_prompt, int64_t m) {
+  if (B < 1 || G < 1 || n_c < 1 || n_prompt < 0 || m < 1) return 0;
+  const int64_t T = n_c / m, m_last = n_c % m;
+  const int64_t full = T > 0 ? B * T * G * roundup(n_prompt + m, 256) * 4 : 0;
+  const int64_t tail = m_last > 0 ? B * G * roundup(n_prompt + m_last, 256) * 4 : 0;
+  return static_cast<size_t>(roundup(full > tail ? full : tail, 256));
+}
+
+kvz_status kvz_score_chunked(const void* Q, const void* Q_tail, const void* K_ctx, const void* K_in,
+                             const void* K_in_tail, int64_t B, int G, int64_t n_c, int64_t n_prompt, int64_t m,
+                             int d, float scale, float* S, void* workspace, size_t workspace_bytes,
+                             int32_t* d_status, cudaStream_t stream) {
+  if (K_ctx == nullptr || S == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return KVZ_ERR_UNSUPPORTED;
+  if (B < 1 || G < 1 || n_c < 1 || n_prompt < 0 || m < 1 || n_c > kMaxRows || n_prompt + m > kMaxRows)
+    return KVZ_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.0f)) return KVZ_ERR_INVALID_ARG;
+  const int64_t T = n_c / m, m_last = n_c % m;
+  if (T > 0 && (Q == nullptr || K_in == nullptr)) return KVZ_ERR_INVALID_ARG;
+  if (m_last > 0 && (Q_tail == nullptr || K_in_tail == nullptr)) return KVZ_ERR_INVALID_ARG;
+  if (B * T * static_cast<int64_t>(G) > 0x7FFFFFFF || B * static_cast<int64_t>(G) > 0x7FFFFFFF)
+    return KVZ_ERR_INVALID_ARG;
+  if (!aligned(K_ctx, 16) || !aligned(S, 4) || (Q && !aligned(Q, 16)) || (Q_tail && !aligned(Q_tail, 16)) ||
+      (K_in && !aligned(K_in, 16)) || (K_in_tail && !aligned(K_in_tail, 16)))
+    return KVZ_ERR_ALIGNMENT;
+  if (workspace == nullptr || workspace_bytes < kvz_score_chunked_workspace_size(B, G, n_c, n_prompt, m))
+    return KVZ_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return KVZ_ERR_ALIGNMENT;
+  float* lse2 = static_cast<float*>(workspace);
+  if (kvz::launch_fill_f32(S, B * n_c, 0.0f, stream) != cudaSuccess) return KVZ_ERR_CUDA;
+  if (T > 0) {
+    // the full chunks of every head as one batch of B*T problems
+    const int64_t n_in = n_prompt + m, ld = roundup(n_in, 256);
+    const CtxGeom geom{static_cast<int>(T), m, n_c};
+    kvz_status st = run_lse(Q, K_ctx, K_in, B * T, G, m, n_in, d, scale, 0, n_in, lse2, ld, d_status, stream, geom);
+    if (st != KVZ_OK) return st;
+    st = run_colmax(Q, K_ctx, B * T, G, m, n_in, d, scale, 0, n_in, lse2, ld, S, d_status, stream, geom, n_c, m);
+    if (st != KVZ_OK) return st;
+  }
+  if (m_last > 0) {
+    // the shorter last chunk of every head
+    const int64_t n_in = n_prompt + m_last, ld = roundup(n_in, 256);
+    const void* K_last = static_cast<const uint8_t*>(K_ctx) + T * m * d * 2;
+    const CtxGeom geom{1, m_last, n_c};
+    kvz_status st = run_lse(Q_tail, K_last, K_in_tail, B, G, m_last, n_in, d, scale, 0, n_in, lse2, ld, d_status,
+                            stream, geom);
+    if (st != KVZ_OK) return st;
+    st = run_colmax(Q_tail, K_last, B, G, m_last, n_in, d, scale, 0, n_in, lse2, ld, S + T * m, d_status, stream,
+                    geom, n_c, m_last);
     if (st != KVZ_OK) return st;
   }
   return KVZ_OK;
@@ -232,9 +324,10 @@ kvz_status kvz_score_noalloc(const void* Q, const void* K_ctx, const void* K_in,
   if (kvz::launch_fill_f32(S, B * n_c, 0.0f, stream) != cudaSuccess) return KVZ_ERR_CUDA;
   for (int64_t i0 = 0; i0 < n_in; i0 += chunk) {
     const int64_t i1 = i0 + chunk < n_in ? i0 + chunk : n_in;
-    st = run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, d_status, stream);
+    st = run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, d_status, stream, plain_geom(n_c));
     if (st != KVZ_OK) return st;
-    st = run_colmax(Q, K_ctx, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, S, d_status, stream);
+    st = run_colmax(Q, K_ctx, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, S, d_status, stream, plain_geom(n_c),
+                    n_c, n_c);
     if (st != KVZ_OK) return st;
   }
   return KVZ_OK;

@@ -11,8 +11,12 @@ namespace kvz {
 // Pass 1 (row log-sum-exp) arguments.  Rows i in [i_begin, i_end) are
 // computed; rows_pad = roundup(i_end - i_begin, 256) entries per (b, g) are
 // written at lse2[(b*G + g)*ld + (i - i_begin)], padding rows set to +inf.
+// A call scores B independent problems (query groups against context keys).
+// Problem p reads context-key block (p % T) of head (p / T): T = 1 for the
+// plain score, T = chunks per head for chunked scoring (the context-key map
+// is 4-D: columns, rows of a block, block, head).
 struct LseArgs {
-  int B, G;
+  int B, G, T;
   int64_t n_c, n_in;
   float c2;                 // scale * log2(e)
   int64_t i_begin, i_end, rows_pad, ld;
@@ -22,12 +26,13 @@ struct LseArgs {
 
 // Pass 2 (context-key column max) arguments; lse2 as pass 1 wrote it.
 struct ColArgs {
-  int B, G;
+  int B, G, T;
   int64_t n_c;
   float c2;
   int64_t i_begin, rows_pad, ld;
   const float* lse2;
-  float* S;
+  float* S;                 // problem p writes S[(p / T) * ldS + (p % T) * s_block + j], j < n_c
+  int64_t ldS, s_block;
   int n_kblk;               // key blocks per head (set by launch_colmax)
   int nsplit;               // row-tile ranges per (head, key block) (set by launch_colmax)
   int tiles_per_split;      // (set by launch_colmax)

@@ -148,11 +148,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t use = static_cast<uint32_t>(t / Lay::KST);
         if (!mbar_wait(&k_empty[s], (use & 1u) ^ 1u, abort_flag, p.status)) break;
         mbar_arrive_expect_tx(&k_full[s], Lay::TILE_BYTES);
-        const bool ctx = t < NC;
-        const CUtensorMap* m = ctx ? &tmKc : &tmKi;
-        const int row = ctx ? t * kTile : (t - NC) * kTile;
-        for (int kb = 0; kb < Lay::KB; ++kb)
-          tma_load_3d(sK + s * Lay::TILE_BYTES + kb * kSubBytes64, m, &k_full[s], kb * 64, row, b);
+        for (int kb = 0; kb < Lay::KB; ++kb) {
+          if (t < NC)   // context keys: block (b % T) of head (b / T)
+            tma_load_4d(sK + s * Lay::TILE_BYTES + kb * kSubBytes64, &tmKc, &k_full[s], kb * 64, t * kTile,
+                        b % p.T, b / p.T);
+          else
+            tma_load_3d(sK + s * Lay::TILE_BYTES + kb * kSubBytes64, &tmKi, &k_full[s], kb * 64,
+                        (t - NC) * kTile, b);
+        }
         issued = t + 1;
       }
     }

@@ -24,7 +24,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "layer_inputs", "synthetic_scores", "seed_for"]
+__all__ = ["Workload", "WORKLOADS", "layer_inputs", "chunked_inputs", "synthetic_scores", "seed_for"]
 
 
 @dataclass(frozen=True)
@@ -45,6 +45,7 @@ class Workload:
     in_place: bool = False        # compact K/V in place
     sinks: int = 0
     dup_frac: float = 0.0
+    chunk: int = 0                # context chunk length m of chunked scoring (0 = unchunked)
     extra: dict = field(default_factory=dict)
 
     def n_in(self, ctx: int = 0) -> int:
@@ -65,6 +66,9 @@ WORKLOADS = {
     "qwen14b_128k": Workload("qwen14b_128k", L=48, H=8, G=5, d=128, n_c=(131072,),
                              n_prompt=32, ratio=0.25, mode="per_head", key_scale=True,
                              row_chunk=4096, in_place=True),
+    # chunked scoring: 2K-token chunks of a 170K context (83 full chunks + 16)
+    "llama8b_170k_chunked": Workload("llama8b_170k_chunked", L=1, H=8, G=4, d=128, n_c=(170000,),
+                                     n_prompt=32, ratio=0.3, mode="per_head", key_scale=True, chunk=2048),
     "stress_ragged": Workload("stress_ragged", L=32, H=8, G=4, d=128,
                               n_c=(1000, 17000, 65537, 170000), n_prompt=32,
                               ratio=0.1, mode="global", key_scale=True,
@@ -160,3 +164,39 @@ def synthetic_scores(B: int, n_c: int, seed: int = 0, device="cpu",
         flat[pos[2 * k:3 * k]] = 1e-42          # subnormal
         flat[pos[3 * k:]] = -0.0                # equal to +0
     return S
+
+
+def chunked_inputs(workload: Workload, layer: int = 0, ctx: int = 0, seed: int = 0, device="cpu",
+                   heads: Optional[int] = None, n_c: Optional[int] = None, n_prompt: Optional[int] = None,
+                   G: Optional[int] = None, d: Optional[int] = None, m: Optional[int] = None):
+    """Inputs of chunked scoring for one layer (bf16): every context chunk of m
+    tokens is appended to the repeat prompt and has its own queries and input
+    keys.  Returns Q [H, T, G, n_prompt+m, d] and K_in [H, T, n_prompt+m, d]
+    for the T = n_c // m full chunks, Q_tail [H, G, n_prompt+m_last, d] and
+    K_in_tail [H, n_prompt+m_last, d] for the shorter last chunk (None when m
+    divides n_c), K_ctx and V [H, n_c, d].  Same distributions as
+    layer_inputs (N(0,1); the key-channel scale on every key)."""
+    H = workload.H if heads is None else heads
+    G = workload.G if G is None else G
+    d = workload.d if d is None else d
+    n_c = workload.n_c[ctx] if n_c is None else n_c
+    n_prompt = workload.n_prompt if n_prompt is None else n_prompt
+    m = workload.chunk if m is None else m
+    T, m_last = n_c // m, n_c % m
+    g = _gen(device, seed_for(workload, layer, ctx, seed))
+    f32 = torch.float32
+    Q = torch.randn((H, T, G, n_prompt + m, d), generator=g, device=device, dtype=f32)
+    K_in = torch.randn((H, T, n_prompt + m, d), generator=g, device=device, dtype=f32)
+    Q_tail = torch.randn((H, G, n_prompt + m_last, d), generator=g, device=device, dtype=f32) if m_last else None
+    K_in_tail = torch.randn((H, n_prompt + m_last, d), generator=g, device=device, dtype=f32) if m_last else None
+    K_ctx = torch.randn((H, n_c, d), generator=g, device=device, dtype=f32)
+    V = torch.randn((H, n_c, d), generator=g, device=device, dtype=f32)
+    if workload.key_scale:
+        sigma = torch.exp(0.5 * torch.randn((H, 1, d), generator=g, device=device, dtype=f32))
+        K_ctx.mul_(sigma)
+        K_in.mul_(sigma[:, None])
+        if K_in_tail is not None:
+            K_in_tail.mul_(sigma)
+    bf = lambda t: None if t is None else t.to(torch.bfloat16).contiguous()
+    return {"Q": bf(Q), "Q_tail": bf(Q_tail), "K_ctx": bf(K_ctx), "K_in": bf(K_in), "K_in_tail": bf(K_in_tail),
+            "V": bf(V), "m": m}

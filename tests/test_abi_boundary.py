@@ -160,3 +160,29 @@ def test_compress_host_rejections(lib):
     assert call(wsb=need - 1) == WS
     assert call(ws_=0) == WS
     assert lib.kvz_compress_host_workspace_size(B, G, n_c, n_in, 96, 0.3, 0) == 0
+
+
+def test_score_chunked_rejections(lib):
+    b = Bufs()
+    B, G, n_c, n_prompt, m, d = 2, 4, 700, 16, 256, 128
+    T, ml = n_c // m, n_c % m
+    Q, Qt = b.get(B * T * G * (n_prompt + m) * d * 2), b.get(B * G * (n_prompt + ml) * d * 2)
+    Kc = b.get(B * n_c * d * 2)
+    Ki, Kit = b.get(B * T * (n_prompt + m) * d * 2), b.get(B * (n_prompt + ml) * d * 2)
+    S = b.get(B * n_c * 4)
+    need = lib.kvz_score_chunked_workspace_size(B, G, n_c, n_prompt, m)
+    assert need == B * T * G * 512 * 4                     # the full chunks' rows, padded to 256, dominate
+    ws = b.get(need)
+
+    def call(q=Q, qt=Qt, d_=d, m_=m, wsb=need, scale=0.1):
+        return lib.kvz_score_chunked(vp(q) if q else None, vp(qt) if qt else None, vp(Kc), vp(Ki), vp(Kit), B, G,
+                                     n_c, n_prompt, m_, d_, scale, vp(S), vp(ws), wsb, None, None)
+
+    assert call(d_=96) == UNSUPPORTED
+    assert call(m_=0) == INVALID
+    assert call(q=0) == INVALID                  # full chunks exist but no Q
+    assert call(qt=0) == INVALID                 # a tail exists but no Q_tail
+    assert call(scale=float("nan")) == INVALID
+    assert call(wsb=need - 1) == WS
+    assert call(q=Q + 8) == ALIGN
+    assert lib.kvz_score_chunked_workspace_size(B, G, n_c, n_prompt, 0) == 0
