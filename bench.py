@@ -43,7 +43,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--workload", default=WORKLOAD,
-                    help="llama8b_layer (default, the headline), tiny, llama8b_stack, qwen14b_128k, stress_ragged")
+                    help="llama8b_layer (default, the headline), tiny, llama8b_stack, qwen14b_128k, stress_ragged, "
+                         "llama8b_170k_chunked")
     ap.add_argument("--layers", type=int, default=0,
                     help="run only the first L layers of the workload (a smaller case for profiling; "
                          "config.workload then names the truncation)")
@@ -143,9 +144,12 @@ def workload_numbers(w):
     B, G, d = w.B, w.G, w.d
     out = {"pairs_per_step": 0, "flops_pass1": 0, "flops_pass2": 0, "kept": 0, "select_bytes": 0}
     for c, n_c in enumerate(w.n_c):
-        n_in = w.n_in(c)
-        vis = B * G * (n_in * n_c + n_in * (n_in + 1) // 2)          # pass 1 pairs
-        ctx = B * G * n_in * n_c                                       # pass 2 pairs
+        # (context keys, input rows) of each independently scored block: the
+        # whole context, or each chunk with its own n_prompt + m_t input rows
+        blocks = [(n_c, w.n_in(c))] if not w.chunk else \
+            [(min(w.chunk, n_c - c0), w.n_prompt + min(w.chunk, n_c - c0)) for c0 in range(0, n_c, w.chunk)]
+        vis = sum(B * G * (ni * nk + ni * (ni + 1) // 2) for nk, ni in blocks)   # pass 1 pairs
+        ctx = sum(B * G * ni * nk for nk, ni in blocks)                          # pass 2 pairs
         kept = int(math.floor(w.ratio * B * n_c)) if w.mode == "global" else B * int(math.floor(w.ratio * n_c))
         out["pairs_per_step"] += B * n_c
         out["flops_pass1"] += 2 * d * vis
@@ -267,6 +271,13 @@ def main():
             for l in range(w.L):
                 Kl = c.K[l * H:(l + 1) * H]
                 Sl = c.S[l * H:(l + 1) * H]
+                if w.chunk:
+                    x = c.X[l]
+                    mark("sc")
+                    kvz.kvz_score_chunked(x["Q"], x["Q_tail"], Kl, x["K_in"], x["K_in_tail"], w.chunk, scale=scale,
+                                          S=Sl, workspace=c.chunk_ws, status=status, stream=stream)
+                    mark("end")
+                    continue
                 for (i0, i1) in c.chunks:
                     mark("p1")
                     kvz.kvz_score_lse2(c.Q[l], Kl, c.Kin[l], i_begin=i0, i_end=i1, scale=scale, lse2=c.lse2,
@@ -289,11 +300,12 @@ def main():
         return marks
 
     def phase_ms(marks):
-        acc = {"p1": 0.0, "p2": 0.0, "sel": 0.0, "cmp": 0.0}
+        # "sc": one chunked-score call (both passes); booked as pass 1, pass 2 = 0
+        acc = {"p1": 0.0, "p2": 0.0, "sel": 0.0, "cmp": 0.0, "sc": 0.0}
         for (tag, e0), (_, e1) in zip(marks, marks[1:]):
             if tag in acc:
                 acc[tag] += e0.elapsed_time(e1)
-        return [acc["p1"], acc["p2"], acc["sel"], acc["cmp"]]
+        return [acc["p1"] + acc["sc"], acc["p2"], acc["sel"], acc["cmp"]]
 
     # the headline workload always gets >= 3 warm-up steps; the large ones
     # (tens of seconds per step) take what the caller asks for
@@ -325,7 +337,7 @@ def main():
     # ---- end to end through the host-buffer C-ABI call (pinned buffers): every
     # step copies the inputs in and the results out inside the timed region
     e2e = None
-    if len(ctxs) == 1 and w.L == 1 and not w.in_place:
+    if len(ctxs) == 1 and w.L == 1 and not w.in_place and not w.chunk:
         c = ctxs[0]
         hx = {"Q": c.Q[0].cpu().pin_memory(), "K_ctx": c.K.cpu().pin_memory(), "K_in": c.Kin[0].cpu().pin_memory(),
               "V": c.V.cpu().pin_memory()}
@@ -371,14 +383,16 @@ def main():
     score_ms = lse_ms + col_ms
     fl1, fl2 = nums["flops_pass1"], nums["flops_pass2"]
     tf = lambda flops, ms: flops / (ms * 1e-3) / 1e12
-    n_p1 = sum(w.L * len(c.chunks) for c in ctxs)
+    n_p1 = sum(w.L * (c.score_launches if w.chunk else len(c.chunks)) for c in ctxs)
+    chunked = bool(w.chunk)
     roof = {
         "bound": "tensor",
-        "kernel": "lse_kernel (score pass 1: QK^T + online log-sum-exp)",
-        "achieved": tf(fl1, lse_ms),
+        "kernel": ("lse_kernel + colmax_kernel (chunked score call, both passes; executed FLOP)" if chunked else
+                   "lse_kernel (score pass 1: QK^T + online log-sum-exp)"),
+        "achieved": tf(fl1 + fl2, lse_ms) if chunked else tf(fl1, lse_ms),
         "peak": pk["bf16_tflops"],
         "unit": "TFLOP/s",
-        "frac": tf(fl1, lse_ms) / pk["bf16_tflops"],
+        "frac": (tf(fl1 + fl2, lse_ms) if chunked else tf(fl1, lse_ms)) / pk["bf16_tflops"],
         "traffic": recorded_traffic("lse_kernel") if w.name == WORKLOAD else None,
         "peak_source": "%s bf16 dense (burst)" % pk["source"],
         "algorithmic_flops_per_launch": fl1 / n_p1,
@@ -389,7 +403,8 @@ def main():
             "score_frac_executed": tf(fl1 + fl2, score_ms) / pk["bf16_tflops"],
             "score_tflops_algorithmic": tf(nums["flops_algorithmic"], score_ms),
             "score_frac_algorithmic": tf(nums["flops_algorithmic"], score_ms) / pk["bf16_tflops"],
-            "pass2_tflops": tf(fl2, col_ms), "pass2_frac": tf(fl2, col_ms) / pk["bf16_tflops"],
+            "pass2_tflops": tf(fl2, col_ms) if col_ms > 0 else None,
+            "pass2_frac": tf(fl2, col_ms) / pk["bf16_tflops"] if col_ms > 0 else None,
             "compact_bytes": nums["compact_bytes"],
             "compact_gbs": nums["compact_bytes"] / (cmp_ms * 1e-3) / 1e9,
             "compact_frac_hbm": nums["compact_bytes"] / (cmp_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
@@ -433,8 +448,19 @@ class Context:
         self.n_c, self.n_in = w.n_c[c], w.n_in(c)
         self.K = torch.empty((B, self.n_c, d), dtype=torch.bfloat16, device=dev)
         self.V = torch.empty((B, self.n_c, d), dtype=torch.bfloat16, device=dev)
-        self.Q, self.Kin = [], []
-        for l in range(L):
+        self.Q, self.Kin, self.X = [], [], []
+        if w.chunk:
+            # chunked scoring: every layer's per-chunk queries and input keys
+            for l in range(L):
+                x = synth.chunked_inputs(w, layer=l, ctx=c, seed=seed, device=dev)
+                self.K[l * H:(l + 1) * H].copy_(x.pop("K_ctx"))
+                self.V[l * H:(l + 1) * H].copy_(x.pop("V"))
+                self.X.append(x)
+            self.chunk_ws = torch.empty(kvz.kvz_score_chunked_workspace_size(H, G, self.n_c, w.n_prompt, w.chunk),
+                                        dtype=torch.uint8, device=dev)
+            n_full, tail = self.n_c // w.chunk, self.n_c % w.chunk
+            self.score_launches = (1 if n_full else 0) + (1 if tail else 0)     # lse launches per layer
+        for l in range(L if not w.chunk else 0):
             x = synth.layer_inputs(w, layer=l, ctx=c, seed=seed, device=dev)
             self.K[l * H:(l + 1) * H].copy_(x["K_ctx"])
             self.V[l * H:(l + 1) * H].copy_(x["V"])
@@ -457,9 +483,15 @@ class Context:
         if not w.in_place:
             self.K_out = torch.empty((cap, d), dtype=torch.bfloat16, device=dev)
             self.V_out = torch.empty((cap, d), dtype=torch.bfloat16, device=dev)
-        # lse (+ colmax, + S fill on the first chunk) per (layer, chunk); select 10; compact 1
-        # (in place: workspace fill, reader-run pre-pass, compaction)
-        self.launches = L * (2 * len(self.chunks) + 1) + 10 + (3 if w.in_place else 1)
+        # lse (+ colmax, + S fill on the first chunk) per (layer, chunk); select 10 (1 per head
+        # when one CTA per head does it); compact 1 (in place: workspace fill, reader-run
+        # pre-pass, compaction)
+        per_head_one = w.mode == "per_head" and (self.n_c <= 49152 or B >= 128)
+        sel = 1 if per_head_one else 10
+        if w.chunk:
+            self.launches = L * (2 * self.score_launches + 1) + sel + (3 if w.in_place else 1)
+        else:
+            self.launches = L * (2 * len(self.chunks) + 1) + sel + (3 if w.in_place else 1)
 
 
 if __name__ == "__main__":
