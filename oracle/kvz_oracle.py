@@ -44,6 +44,8 @@ __all__ = [
     "score_chunked",
     "keep_count",
     "select",
+    "head_scores",
+    "select_heads",
     "compact",
     "visible_pairs",
 ]
@@ -229,6 +231,36 @@ def select(S, ratio, mode):
     offsets = np.zeros(B + 1, dtype=np.int64)
     offsets[1:] = np.cumsum(counts)
     idx = (np.concatenate(per_head) if B else np.zeros(0)).astype(np.int32)
+    return idx, counts, offsets
+
+
+# ---------------------------------------------------------------------------
+# Context-independent head scores (KVzip §4.2 "context-independent eviction":
+# one static importance per head, the pair scores aggregated by a max along
+# the sequence) and head-level eviction
+# ---------------------------------------------------------------------------
+def head_scores(S):
+    """S_head[b] = max over the context positions j of S[b, j]."""
+    S = np.asarray(S)
+    if S.ndim != 2 or S.shape[1] < 1:
+        raise ValueError("S must be [B, n_c] with n_c >= 1")
+    return S.max(axis=1)
+
+
+def select_heads(S_head, ratio, n_c):
+    """Head-level eviction: keep the floor(ratio * B) heads with the highest
+    head score (ties to the lower head index); a kept head keeps all its n_c
+    pairs, an evicted head none.  Returns the selection in the same CSR form
+    as ``select`` (idx int32, counts int32 [B], offsets int64 [B+1])."""
+    S_head = np.asarray(S_head, dtype=np.float32)
+    B = S_head.shape[0]
+    order = np.argsort(-S_head, kind="stable")
+    kept = np.sort(order[: keep_count(B, ratio)])
+    counts = np.zeros(B, dtype=np.int32)
+    counts[kept] = int(n_c)
+    offsets = np.zeros(B + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    idx = np.tile(np.arange(int(n_c), dtype=np.int32), len(kept))
     return idx, counts, offsets
 
 

@@ -371,3 +371,47 @@ def test_chunked_brute_force_mpmath():
                     w = [mpmath.e ** (sc * mpmath.fsum(a * b for a, b in zip(q, keys[u]))) for u in range(mt + i + 1)]
                     best = max(best, w[j] / mpmath.fsum(w))
             assert abs(S[c0 + j] - float(best)) <= 1e-13 * float(best)
+
+
+# --------------------------------------------------------------------------
+# Head scores and head-level eviction (KVzip §4.2, context-independent)
+# --------------------------------------------------------------------------
+def test_head_score_is_attained_upper_bound():
+    rng = np.random.default_rng(31)
+    S = rng.random((6, 50)).astype(np.float32)
+    h = orc.head_scores(S)
+    for b in range(6):
+        assert np.all(S[b] <= h[b]) and h[b] in S[b]     # an upper bound that is attained: the max
+
+
+def test_head_scores_of_uniform_rows():
+    # identical keys: every score is 1/(n_c+1), so is every head score
+    rng = np.random.default_rng(32)
+    G, n_c, n_in, d = 2, 9, 12, 4
+    v = rng.standard_normal(d)
+    S = np.stack([orc.score(rng.standard_normal((G, n_in, d)), np.tile(v, (n_c, 1)), np.tile(v, (n_in, 1)), 0.5)
+                  for _ in range(3)])
+    np.testing.assert_allclose(orc.head_scores(S), 1.0 / (n_c + 1), rtol=1e-13)
+
+
+@pytest.mark.parametrize("B", [1, 2, 5, 7])
+def test_select_heads_exhaustive(B):
+    # every kept set of size k over a few score levels: the oracle's set is the
+    # one a brute-force search ranks first by (value desc, index asc)
+    rng = np.random.default_rng(33 + B)
+    n_c = 3
+    for trial in range(20):
+        S_head = rng.integers(0, 3, B).astype(np.float32) / 2
+        for ratio in (0.0, 0.3, 0.5, 1.0):
+            k = orc.keep_count(B, ratio)
+            # the kept set whose sorted (-score, index) list is lexicographically smallest
+            brute = None
+            for c in itertools.combinations(range(B), k):
+                keyv = sorted([(-float(S_head[i]), i) for i in c])
+                if brute is None or keyv < brute[0]:
+                    brute = (keyv, c)
+            idx, counts, offsets = orc.select_heads(S_head, ratio, n_c)
+            kept = [b for b in range(B) if counts[b] == n_c]
+            assert tuple(kept) == (brute[1] if brute else ())
+            assert set(counts.tolist()) <= {0, n_c} and offsets[-1] == k * n_c
+            assert np.array_equal(idx, np.tile(np.arange(n_c), k))
