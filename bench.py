@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--workload", default=WORKLOAD,
                     help="llama8b_layer (default, the headline), tiny, llama8b_stack, qwen14b_128k, stress_ragged, "
-                         "llama8b_170k_chunked")
+                         "llama8b_170k_chunked, llama8b_stack_heads")
     ap.add_argument("--layers", type=int, default=0,
                     help="run only the first L layers of the workload (a smaller case for profiling; "
                          "config.workload then names the truncation)")
@@ -150,12 +150,15 @@ def workload_numbers(w):
             [(min(w.chunk, n_c - c0), w.n_prompt + min(w.chunk, n_c - c0)) for c0 in range(0, n_c, w.chunk)]
         vis = sum(B * G * (ni * nk + ni * (ni + 1) // 2) for nk, ni in blocks)   # pass 1 pairs
         ctx = sum(B * G * ni * nk for nk, ni in blocks)                          # pass 2 pairs
-        kept = int(math.floor(w.ratio * B * n_c)) if w.mode == "global" else B * int(math.floor(w.ratio * n_c))
+        if w.mode == "heads":
+            kept = int(math.floor(w.ratio * B)) * n_c
+        else:
+            kept = int(math.floor(w.ratio * B * n_c)) if w.mode == "global" else B * int(math.floor(w.ratio * n_c))
         out["pairs_per_step"] += B * n_c
         out["flops_pass1"] += 2 * d * vis
         out["flops_pass2"] += 2 * d * ctx
         out["kept"] += kept
-        out["select_bytes"] += 5 * 4 * B * n_c
+        out["select_bytes"] += (1 if w.mode == "heads" else 5) * 4 * B * n_c
     out["flops_algorithmic"] = out["flops_pass1"]
     out["compact_bytes"] = out["kept"] * d * 2 * 2 * 2 + 4 * out["kept"]
     return out
@@ -287,8 +290,13 @@ def main():
                                          accumulate=i0 > 0, status=status, stream=stream)
                     mark("end")
             mark("sel")
-            kvz.kvz_select(c.S, w.ratio, w.mode, idx=c.idx, counts=c.counts, offsets=c.offsets,
-                           workspace=c.sel_ws, status=status, stream=stream)
+            if w.mode == "heads":
+                kvz.kvz_head_score(c.S, S_head=c.S_head, status=status, stream=stream)
+                kvz.kvz_select_heads(c.S_head, c.n_c, w.ratio, idx=c.idx, counts=c.counts, offsets=c.offsets,
+                                     workspace=c.sel_ws, status=status, stream=stream)
+            else:
+                kvz.kvz_select(c.S, w.ratio, w.mode, idx=c.idx, counts=c.counts, offsets=c.offsets,
+                               workspace=c.sel_ws, status=status, stream=stream)
             mark("cmp")
             if w.in_place:
                 kvz.kvz_compact(c.K, c.V, c.idx, c.counts, c.offsets, in_place=True, workspace=c.cmp_ws,
@@ -473,12 +481,18 @@ class Context:
         self.lse2 = torch.empty((H, G, self.ld), dtype=torch.float32, device=dev)
         self.S = torch.empty((B, self.n_c), dtype=torch.float32, device=dev)
         mode = kvz.GLOBAL if w.mode == "global" else kvz.PER_HEAD
-        k = kvz.kvz_keep_count(B * self.n_c if mode == kvz.GLOBAL else self.n_c, w.ratio)
-        cap = max(1, k if mode == kvz.GLOBAL else B * k)
+        if w.mode == "heads":
+            cap = max(1, kvz.kvz_keep_count(B, w.ratio) * self.n_c)
+            self.S_head = torch.empty(B, dtype=torch.float32, device=dev)
+            self.sel_ws = torch.empty(kvz.lib().kvz_select_heads_workspace_size(B), dtype=torch.uint8, device=dev)
+        else:
+            k = kvz.kvz_keep_count(B * self.n_c if mode == kvz.GLOBAL else self.n_c, w.ratio)
+            cap = max(1, k if mode == kvz.GLOBAL else B * k)
+            self.sel_ws = torch.empty(kvz.kvz_select_workspace_size(B, self.n_c, mode), dtype=torch.uint8,
+                                      device=dev)
         self.idx = torch.empty(cap, dtype=torch.int32, device=dev)
         self.counts = torch.empty(B, dtype=torch.int32, device=dev)
         self.offsets = torch.empty(B + 1, dtype=torch.int64, device=dev)
-        self.sel_ws = torch.empty(kvz.kvz_select_workspace_size(B, self.n_c, mode), dtype=torch.uint8, device=dev)
         self.cmp_ws = torch.empty(kvz.kvz_compact_workspace_size(B, self.n_c), dtype=torch.uint8, device=dev)
         if not w.in_place:
             self.K_out = torch.empty((cap, d), dtype=torch.bfloat16, device=dev)
@@ -487,7 +501,8 @@ class Context:
         # when one CTA per head does it); compact 1 (in place: workspace fill, reader-run
         # pre-pass, compaction)
         per_head_one = w.mode == "per_head" and (self.n_c <= 49152 or B >= 128)
-        sel = 1 if per_head_one else 10
+        # head level: fill + head max, one-segment selection (1 launch up to 49152 heads), csr + idx
+        sel = 1 if per_head_one else (5 if w.mode == "heads" else 10)
         if w.chunk:
             self.launches = L * (2 * self.score_launches + 1) + sel + (3 if w.in_place else 1)
         else:

@@ -204,6 +204,30 @@ kvz_status kvz_select(const float* S, int64_t B, int64_t n_c, double ratio,
                       int32_t* d_status, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Context-independent head scores and head-level eviction (KVzip §4.2,     */
+/* "context-independent eviction": one static importance per head, the pair  */
+/* scores aggregated by a max along the sequence).                           */
+/*                                                                          */
+/* kvz_head_score: S_head[b] = max_j S[b][j].  S [B][n_c] fp32 (>= 0),      */
+/*   S_head [B] fp32 (overwritten).  NaN or negative scores are reported    */
+/*   (KVZ_ERR_INVALID_SCORE) and counted as +0.                              */
+/* kvz_select_heads: keep the floor(ratio * B) heads with the highest head   */
+/*   score (ties to the lower head index); a kept head keeps all its n_c     */
+/*   pairs, an evicted head none.  Output in kvz_select's CSR form, ready    */
+/*   for kvz_compact: counts[b] in {0, n_c}, offsets [B+1], idx = 0..n_c-1   */
+/*   for each kept head in head order (capacity floor(ratio*B) * n_c).       */
+/*   Workspace: kvz_select_heads_workspace_size(B) bytes.  B <= 65535.       */
+/* ------------------------------------------------------------------------ */
+kvz_status kvz_head_score(const float* S, int64_t B, int64_t n_c, float* S_head, int32_t* d_status,
+                          cudaStream_t stream);
+
+size_t kvz_select_heads_workspace_size(int64_t B);
+
+kvz_status kvz_select_heads(const float* S_head, int64_t B, int64_t n_c, double ratio, int32_t* idx,
+                            int64_t idx_capacity, int32_t* counts, int64_t* offsets, void* workspace,
+                            size_t workspace_bytes, int32_t* d_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Compaction.                                                               */
 /*                                                                          */
 /* KVzip §2.1: the pruned cache K_p is a subset of the full cache K_c that   */

@@ -65,6 +65,9 @@ _SIGS = {
     "kvz_select": (_i32, [_vp, _i64, _i64, _f64, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
     "kvz_compact_workspace_size": (_sz, [_i64, _i64]),
     "kvz_compact": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "kvz_head_score": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
+    "kvz_select_heads_workspace_size": (_sz, [_i64]),
+    "kvz_select_heads": (_i32, [_vp, _i64, _i64, _f64, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
     "kvz_score_chunked_workspace_size": (_sz, [_i64, _i32, _i64, _i64, _i64]),
     "kvz_score_chunked": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i64, _i64, _i64, _i32, _f32, _vp, _vp, _sz,
                                  _vp, _vp]),
@@ -357,3 +360,35 @@ def kvz_score_chunked(Q, Q_tail, K_ctx, K_in, K_in_tail, m: int, scale: Optional
         _ptr(Q), _ptr(Q_tail), _ptr(K_ctx), _ptr(K_in), _ptr(K_in_tail), B, G, n_c, n_prompt, m, d, float(scale),
         _ptr(S), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)))
     return S
+
+
+def kvz_head_score(S, S_head=None, status=None, stream=None):
+    """Context-independent head scores (KVzip §4.2): S_head[b] = max_j S[b, j]."""
+    _need_cuda(S, S_head, status)
+    B, n_c = S.shape
+    if S_head is None:
+        S_head = torch.empty(B, dtype=torch.float32, device=S.device)
+    _check("kvz_head_score", lib().kvz_head_score(_ptr(S), B, n_c, _ptr(S_head), _ptr(status), _stream(stream)))
+    return S_head
+
+
+def kvz_select_heads(S_head, n_c: int, ratio: float, idx=None, counts=None, offsets=None, workspace=None,
+                     status=None, stream=None):
+    """Head-level eviction: keep the floor(ratio*B) best heads whole; returns
+    (idx, counts, offsets) in kvz_select's form, ready for kvz_compact."""
+    _need_cuda(S_head, idx, counts, offsets, workspace, status)
+    B = S_head.shape[0]
+    k = kvz_keep_count(B, ratio)
+    dev = S_head.device
+    if idx is None:
+        idx = torch.empty(max(1, k * n_c), dtype=torch.int32, device=dev)
+    if counts is None:
+        counts = torch.empty(B, dtype=torch.int32, device=dev)
+    if offsets is None:
+        offsets = torch.empty(B + 1, dtype=torch.int64, device=dev)
+    if workspace is None:
+        workspace = torch.empty(lib().kvz_select_heads_workspace_size(B), dtype=torch.uint8, device=dev)
+    _check("kvz_select_heads", lib().kvz_select_heads(
+        _ptr(S_head), B, n_c, float(ratio), _ptr(idx), idx.numel(), _ptr(counts), _ptr(offsets), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)))
+    return idx, counts, offsets

@@ -365,6 +365,45 @@ kvz_status kvz_select(const float* S, int64_t B, int64_t n_c, double ratio, int 
              : KVZ_ERR_CUDA;
 }
 
+kvz_status kvz_head_score(const float* S, int64_t B, int64_t n_c, float* S_head, int32_t* d_status,
+                          cudaStream_t stream) {
+  if (S == nullptr || S_head == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (B < 1 || B > 65535 || n_c < 1 || n_c > kMaxRows) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(S, 4) || !aligned(S_head, 4)) return KVZ_ERR_ALIGNMENT;
+  return kvz::launch_head_max(S, B, n_c, S_head, d_status, stream) == cudaSuccess ? KVZ_OK : KVZ_ERR_CUDA;
+}
+
+size_t kvz_select_heads_workspace_size(int64_t B) {
+  if (B < 1 || B > 65535) return 0;
+  const size_t sel = kvz_select_workspace_size(1, B, KVZ_PER_HEAD);
+  return ((sel + 255) & ~size_t(255)) + ((static_cast<size_t>(B) * 4 + 255) & ~size_t(255)) + 256;
+}
+
+kvz_status kvz_select_heads(const float* S_head, int64_t B, int64_t n_c, double ratio, int32_t* idx,
+                            int64_t idx_capacity, int32_t* counts, int64_t* offsets, void* workspace,
+                            size_t workspace_bytes, int32_t* d_status, cudaStream_t stream) {
+  if (S_head == nullptr || counts == nullptr || offsets == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (B < 1 || B > 65535 || n_c < 1 || n_c > kMaxRows) return KVZ_ERR_INVALID_ARG;
+  if (!(ratio >= 0.0 && ratio <= 1.0)) return KVZ_ERR_INVALID_ARG;
+  const int64_t k = kvz_keep_count(B, ratio);
+  if (idx_capacity < k * n_c || (k > 0 && idx == nullptr) || k * n_c > 0x7FFFFFFF) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(S_head, 4) || !aligned(counts, 4) || !aligned(offsets, 8) || (idx && !aligned(idx, 4)))
+    return KVZ_ERR_ALIGNMENT;
+  if (workspace == nullptr || workspace_bytes < kvz_select_heads_workspace_size(B)) return KVZ_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return KVZ_ERR_ALIGNMENT;
+  // the head scores as one segment of B scores: the kept heads, ascending
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t sel = (kvz_select_workspace_size(1, B, KVZ_PER_HEAD) + 255) & ~size_t(255);
+  int32_t* kept = reinterpret_cast<int32_t*>(ws + sel);
+  int32_t* cnt1 = reinterpret_cast<int32_t*>(ws + sel + ((static_cast<size_t>(B) * 4 + 255) & ~size_t(255)));
+  int64_t* off2 = reinterpret_cast<int64_t*>(cnt1 + 4);
+  kvz_status st = kvz_select(S_head, 1, B, ratio, KVZ_PER_HEAD, kept, k > 0 ? k : 1, cnt1, off2, ws, sel,
+                             d_status, stream);
+  if (st != KVZ_OK) return st;
+  return kvz::launch_head_expand(kept, k, B, n_c, idx, counts, offsets, stream) == cudaSuccess ? KVZ_OK
+                                                                                            : KVZ_ERR_CUDA;
+}
+
 size_t kvz_compact_workspace_size(int64_t B, int64_t n_c) {
   if (B < 1 || n_c < 1) return 0;
   return kvz::compact_workspace_bytes(B, n_c);

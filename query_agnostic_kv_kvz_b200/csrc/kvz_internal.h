@@ -45,6 +45,12 @@ cudaError_t launch_colmax(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc
                           cudaStream_t stream);
 cudaError_t launch_fill_f32(float* x, int64_t n, float v, cudaStream_t stream);
 
+// Head scores (segmented max of S) and the CSR form of a head-level selection.
+cudaError_t launch_head_max(const float* S, int64_t B, int64_t n_c, float* S_head, int32_t* status,
+                            cudaStream_t stream);
+cudaError_t launch_head_expand(const int32_t* kept, int64_t k, int64_t B, int64_t n_c, int32_t* idx,
+                               int32_t* counts, int64_t* offsets, cudaStream_t stream);
+
 // Selection.  Workspace layout is computed by select_workspace().
 struct SelWorkspace {
   size_t bytes;

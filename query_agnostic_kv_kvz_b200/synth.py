@@ -39,7 +39,7 @@ class Workload:
     n_c: Tuple[int, ...]          # one entry per context (ragged batches: several)
     n_prompt: int
     ratio: float
-    mode: str                     # "per_head" | "global"
+    mode: str                     # "per_head" | "global" | "heads" (head-level eviction)
     key_scale: bool = False       # per-channel log-normal key scale
     row_chunk: int = 0            # input rows per scoring pass (0 = all)
     in_place: bool = False        # compact K/V in place
@@ -66,6 +66,10 @@ WORKLOADS = {
     "qwen14b_128k": Workload("qwen14b_128k", L=48, H=8, G=5, d=128, n_c=(131072,),
                              n_prompt=32, ratio=0.25, mode="per_head", key_scale=True,
                              row_chunk=4096, in_place=True),
+    # head-level eviction: the 256 heads of the stack scored on an 8K context,
+    # the best half kept whole
+    "llama8b_stack_heads": Workload("llama8b_stack_heads", L=32, H=8, G=4, d=128, n_c=(8192,),
+                                    n_prompt=32, ratio=0.5, mode="heads", key_scale=True),
     # chunked scoring: 2K-token chunks of a 170K context (83 full chunks + 16)
     "llama8b_170k_chunked": Workload("llama8b_170k_chunked", L=1, H=8, G=4, d=128, n_c=(170000,),
                                      n_prompt=32, ratio=0.3, mode="per_head", key_scale=True, chunk=2048),

@@ -186,3 +186,23 @@ def test_score_chunked_rejections(lib):
     assert call(wsb=need - 1) == WS
     assert call(q=Q + 8) == ALIGN
     assert lib.kvz_score_chunked_workspace_size(B, G, n_c, n_prompt, 0) == 0
+
+
+def test_head_rejections(lib):
+    b = Bufs()
+    B, n_c = 8, 100
+    S, H = b.get(B * n_c * 4), b.get(B * 4)
+    idx, cnt, off = b.get(4 * n_c * 4), b.get(B * 4), b.get((B + 1) * 8)
+    need = lib.kvz_select_heads_workspace_size(B)
+    ws = b.get(need)
+    assert lib.kvz_head_score(vp(S), 0, n_c, vp(H), None, None) == INVALID
+    assert lib.kvz_head_score(vp(S + 2), B, n_c, vp(H), None, None) == ALIGN
+    assert lib.kvz_head_score(None, B, n_c, vp(H), None, None) == INVALID
+
+    def sel(ratio=0.5, cap=4 * n_c, wsb=need):
+        return lib.kvz_select_heads(vp(H), B, n_c, ratio, vp(idx), cap, vp(cnt), vp(off), vp(ws), wsb, None, None)
+
+    assert sel(ratio=1.2) == INVALID
+    assert sel(cap=4 * n_c - 1) == INVALID         # 4 heads of 100 rows each
+    assert sel(wsb=need - 1) == WS
+    assert lib.kvz_select_heads_workspace_size(70000) == 0
