@@ -46,6 +46,7 @@ __all__ = [
     "select",
     "head_scores",
     "select_heads",
+    "decode_attention",
     "compact",
     "visible_pairs",
 ]
@@ -262,6 +263,39 @@ def select_heads(S_head, ratio, n_c):
     offsets[1:] = np.cumsum(counts)
     idx = np.tile(np.arange(int(n_c), dtype=np.int32), len(kept))
     return idx, counts, offsets
+
+
+# ---------------------------------------------------------------------------
+# Decode attention over the pruned cache (KVzip §2.1: every later query reads
+# the pruned cache K_p, V_p in place of the full one)
+# ---------------------------------------------------------------------------
+def decode_attention(q, K_out, V_out, counts, offsets, scale):
+    """One decode step's attention for each KV head b over its kept rows.
+
+    q: [B, G, d] grouped queries of the new token; K_out, V_out: [rows, d],
+    head b's kept keys/values at rows offsets[b] .. offsets[b] + counts[b].
+    out[b, g] = sum_j softmax_j(scale * <q[b, g], k_j>) v_j; lse2[b, g] is the
+    base-2 log of the softmax denominator (scale folded in).  A head with no
+    kept rows gives out = 0 and lse2 = -inf.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    K_out = np.asarray(K_out, dtype=np.float64)
+    V_out = np.asarray(V_out, dtype=np.float64)
+    B, G, d = q.shape
+    out = np.zeros((B, G, d))
+    lse2 = np.full((B, G), -np.inf)
+    for b in range(B):
+        r0, n = int(offsets[b]), int(counts[b])
+        if n == 0:
+            continue
+        Kb, Vb = K_out[r0:r0 + n], V_out[r0:r0 + n]
+        for g in range(G):
+            z = float(scale) * (Kb @ q[b, g])
+            zm = np.max(z)
+            w = np.exp(z - zm)
+            out[b, g] = (w @ Vb) / np.sum(w)
+            lse2[b, g] = (zm + np.log(np.sum(w))) / math.log(2.0)
+    return out, lse2
 
 
 # ---------------------------------------------------------------------------

@@ -415,3 +415,52 @@ def test_select_heads_exhaustive(B):
             assert tuple(kept) == (brute[1] if brute else ())
             assert set(counts.tolist()) <= {0, n_c} and offsets[-1] == k * n_c
             assert np.array_equal(idx, np.tile(np.arange(n_c), k))
+
+
+# --------------------------------------------------------------------------
+# Decode attention over the pruned cache
+# --------------------------------------------------------------------------
+def _csr(counts):
+    offsets = np.zeros(len(counts) + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    return np.asarray(counts), offsets
+
+
+def test_decode_single_key_returns_its_value():
+    rng = np.random.default_rng(41)
+    counts, offsets = _csr([1, 1])
+    K, V = rng.standard_normal((2, 8)), rng.standard_normal((2, 8))
+    q = rng.standard_normal((2, 3, 8))
+    out, lse2 = orc.decode_attention(q, K, V, counts, offsets, 0.7)
+    for b in range(2):
+        np.testing.assert_allclose(out[b], np.tile(V[b], (3, 1)), rtol=1e-15)
+        np.testing.assert_allclose(lse2[b], 0.7 * (q[b] @ K[b]) / math.log(2), rtol=1e-13)
+
+
+def test_decode_identical_keys_average_the_values():
+    rng = np.random.default_rng(42)
+    counts, offsets = _csr([5, 0, 3])
+    v = rng.standard_normal(6)
+    K = np.tile(v, (8, 1))
+    V = rng.standard_normal((8, 6))
+    q = rng.standard_normal((3, 2, 6)) * 4
+    out, lse2 = orc.decode_attention(q, K, V, counts, offsets, 0.3)
+    np.testing.assert_allclose(out[0], np.tile(V[:5].mean(axis=0), (2, 1)), rtol=1e-12)
+    np.testing.assert_allclose(out[2], np.tile(V[5:].mean(axis=0), (2, 1)), rtol=1e-12)
+    assert np.all(out[1] == 0) and np.all(np.isneginf(lse2[1]))        # empty head
+
+
+def test_decode_on_the_kept_set_is_the_renormalised_full_softmax():
+    # attention over a subset equals the full-cache softmax restricted to the
+    # subset and renormalised (scipy softmax, an independent routine)
+    rng = np.random.default_rng(43)
+    n_c, d, G, s = 40, 16, 4, 0.25
+    K, V = rng.standard_normal((n_c, d)), rng.standard_normal((n_c, d))
+    q = rng.standard_normal((1, G, d))
+    keep = np.sort(rng.choice(n_c, 13, replace=False))
+    counts, offsets = _csr([len(keep)])
+    out, _ = orc.decode_attention(q, K[keep], V[keep], counts, offsets, s)
+    for g in range(G):
+        p = scipy.special.softmax(s * (K @ q[0, g]))
+        pk = p[keep] / p[keep].sum()
+        np.testing.assert_allclose(out[0, g], pk @ V[keep], rtol=1e-12, atol=1e-14)
