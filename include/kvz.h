@@ -264,6 +264,31 @@ kvz_status kvz_compact(const void* K, const void* V, int64_t B, int64_t n_c,
                        int32_t* d_status, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Decode attention over the pruned cache (KVzip §2.1: every later query     */
+/* reads the pruned cache in place of the full one).                         */
+/*                                                                          */
+/* One decode step for each KV head b with the G grouped queries of the new  */
+/* token: out[b][g] = sum_j softmax_j(scale * <q[b][g], k_j>) v_j over head  */
+/* b's kept rows j (rows offsets[b] .. offsets[b] + counts[b] of K_out and   */
+/* V_out, as kvz_compact packs them).  lse2[b][g] (optional) is the base-2   */
+/* log of the softmax denominator.  A head with counts[b] == 0 gives out = 0 */
+/* and lse2 = -inf.                                                          */
+/* Layout: q [B][G][d] bf16; K_out, V_out [n_rows][d] bf16; out [B][G][d]    */
+/* fp32; lse2 [B][G] fp32.  n_c bounds every counts[b] (it sizes the split   */
+/* of each head's rows over CTAs); a count outside [0, n_c] is reported      */
+/* (KVZ_ERR_INVALID_ARG in d_status) and that head is skipped.              */
+/* Limits: d in {64, 128}; 1 <= G <= 8 (else KVZ_ERR_UNSUPPORTED);          */
+/* B <= 65535.  Workspace: kvz_decode_workspace_size(B, G, n_c, d) bytes,    */
+/* 256-byte aligned (per-split partial results).                             */
+/* ------------------------------------------------------------------------ */
+size_t kvz_decode_workspace_size(int64_t B, int G, int64_t n_c, int d);
+
+kvz_status kvz_decode(const void* q, const void* K_out, const void* V_out, int64_t n_rows,
+                      const int32_t* counts, const int64_t* offsets, int64_t B, int G, int64_t n_c,
+                      int d, float scale, float* out, float* lse2, void* workspace,
+                      size_t workspace_bytes, int32_t* d_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Chunked scoring (KVzip §3.4, "chunk-based scoring").                      */
 /*                                                                          */
 /* The context is cut into chunks of m tokens (the last one is n_c mod m     */

@@ -65,6 +65,8 @@ _SIGS = {
     "kvz_select": (_i32, [_vp, _i64, _i64, _f64, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
     "kvz_compact_workspace_size": (_sz, [_i64, _i64]),
     "kvz_compact": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "kvz_decode_workspace_size": (_sz, [_i64, _i32, _i64, _i32]),
+    "kvz_decode": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _i64, _i32, _i64, _i32, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
     "kvz_head_score": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "kvz_select_heads_workspace_size": (_sz, [_i64]),
     "kvz_select_heads": (_i32, [_vp, _i64, _i64, _f64, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
@@ -392,3 +394,26 @@ def kvz_select_heads(S_head, n_c: int, ratio: float, idx=None, counts=None, offs
         _ptr(S_head), B, n_c, float(ratio), _ptr(idx), idx.numel(), _ptr(counts), _ptr(offsets), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)))
     return idx, counts, offsets
+
+
+def kvz_decode(q, K_out, V_out, counts, offsets, n_c: int, scale: Optional[float] = None, out=None, lse2=None,
+               workspace=None, status=None, stream=None):
+    """One decode step of attention over the pruned cache; returns (out [B, G, d]
+    fp32, lse2 [B, G] fp32).  q is bf16 [B, G, d]; K_out / V_out are the packed
+    [rows, d] caches kvz_compact writes; n_c bounds every head's count."""
+    _need_cuda(q, K_out, V_out, counts, offsets, out, lse2, workspace, status)
+    B, G, d = q.shape
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, G, d), dtype=torch.float32, device=dev)
+    if lse2 is None:
+        lse2 = torch.empty((B, G), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(lib().kvz_decode_workspace_size(B, G, n_c, d), dtype=torch.uint8, device=dev)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check("kvz_decode", lib().kvz_decode(
+        _ptr(q), _ptr(K_out), _ptr(V_out), K_out.shape[0], _ptr(counts), _ptr(offsets), B, G, n_c, d, float(scale),
+        _ptr(out), _ptr(lse2), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)))
+    return out, lse2

@@ -77,6 +77,21 @@ struct CtxGeom {
 };
 CtxGeom plain_geom(int64_t n_c) { return CtxGeom{1, n_c, n_c}; }
 
+// Rows [rows][d] of a packed cache read in 64-row x 64-column boxes (128-byte
+// swizzle) by the decode kernel.
+bool make_rows_map(CUtensorMap* m, const void* base, int64_t d, int64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(rows * d * 2)};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 float log2e_scale(float scale) { return static_cast<float>(static_cast<double>(scale) * 1.4426950408889634); }
 
 kvz_status check_score_common(const void* Q, const void* K_ctx, int64_t B, int G, int64_t n_c, int64_t n_in,
@@ -402,6 +417,49 @@ kvz_status kvz_select_heads(const float* S_head, int64_t B, int64_t n_c, double 
   if (st != KVZ_OK) return st;
   return kvz::launch_head_expand(kept, k, B, n_c, idx, counts, offsets, stream) == cudaSuccess ? KVZ_OK
                                                                                             : KVZ_ERR_CUDA;
+}
+
+size_t kvz_decode_workspace_size(int64_t B, int G, int64_t n_c, int d) {
+  if (B < 1 || B > 65535 || G < 1 || G > kvz::kDecGMax || n_c < 1 || (d != 64 && d != 128)) return 0;
+  int cps = 0, splits = 0;
+  kvz::decode_plan(B, n_c, &cps, &splits);
+  const size_t parts = static_cast<size_t>(B) * splits * G;
+  return ((parts * 8 + 255) & ~size_t(255)) + ((parts * d * 4 + 255) & ~size_t(255));
+}
+
+kvz_status kvz_decode(const void* q, const void* K_out, const void* V_out, int64_t n_rows, const int32_t* counts,
+                      const int64_t* offsets, int64_t B, int G, int64_t n_c, int d, float scale, float* out,
+                      float* lse2, void* workspace, size_t workspace_bytes, int32_t* d_status,
+                      cudaStream_t stream) {
+  if (q == nullptr || K_out == nullptr || V_out == nullptr || counts == nullptr || offsets == nullptr ||
+      out == nullptr)
+    return KVZ_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return KVZ_ERR_UNSUPPORTED;
+  if (G < 1 || G > kvz::kDecGMax) return KVZ_ERR_UNSUPPORTED;
+  if (B < 1 || B > 65535 || n_c < 1 || n_rows < 1 || n_rows > kMaxRows) return KVZ_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.0f)) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(K_out, 16) || !aligned(V_out, 16) || !aligned(q, 16) || !aligned(out, 16) || !aligned(counts, 4) ||
+      !aligned(offsets, 8) || (lse2 && !aligned(lse2, 4)))
+    return KVZ_ERR_ALIGNMENT;
+  const size_t need = kvz_decode_workspace_size(B, G, n_c, d);
+  if (workspace == nullptr || workspace_bytes < need) return KVZ_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return KVZ_ERR_ALIGNMENT;
+  CUtensorMap tmK, tmV;
+  if (!make_rows_map(&tmK, K_out, d, n_rows) || !make_rows_map(&tmV, V_out, d, n_rows)) return KVZ_ERR_CUDA;
+  kvz::DecArgs a{};
+  a.B = static_cast<int>(B);
+  a.G = G;
+  a.n_c = n_c;
+  a.c2 = log2e_scale(scale);
+  a.q = static_cast<const uint16_t*>(q);
+  a.counts = counts;
+  a.offsets = offsets;
+  kvz::decode_plan(B, n_c, &a.cps, &a.splits);
+  const size_t parts = static_cast<size_t>(B) * a.splits * G;
+  a.part_ml = static_cast<float2*>(workspace);
+  a.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((parts * 8 + 255) & ~size_t(255)));
+  a.status = d_status;
+  return kvz::launch_decode(d, tmK, tmV, a, out, lse2, stream) == cudaSuccess ? KVZ_OK : KVZ_ERR_CUDA;
 }
 
 size_t kvz_compact_workspace_size(int64_t B, int64_t n_c) {

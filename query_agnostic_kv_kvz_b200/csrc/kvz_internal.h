@@ -45,6 +45,25 @@ cudaError_t launch_colmax(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc
                           cudaStream_t stream);
 cudaError_t launch_fill_f32(float* x, int64_t n, float v, cudaStream_t stream);
 
+// Decode attention over the pruned cache (split-KV partials + combine).
+constexpr int kDecGMax = 8;                 // grouped queries per KV head
+struct DecArgs {
+  int B, G;
+  int64_t n_c;                              // upper bound of counts[b]
+  float c2;                                 // scale * log2(e)
+  const uint16_t* q;                        // bf16 [B][G][d]
+  const int32_t* counts;
+  const int64_t* offsets;
+  int cps;                                  // 64-key tiles per split
+  int splits;                               // splits per head (grid.x)
+  float2* part_ml;                          // [B][splits][G] (running max, sum), base 2
+  float* part_o;                            // [B][splits][G][d]
+  int32_t* status;
+};
+void decode_plan(int64_t B, int64_t n_c, int* cps, int* splits);
+cudaError_t launch_decode(int d, const CUtensorMap& tmK, const CUtensorMap& tmV, const DecArgs& a, float* out,
+                          float* lse2, cudaStream_t stream);
+
 // Head scores (segmented max of S) and the CSR form of a head-level selection.
 cudaError_t launch_head_max(const float* S, int64_t B, int64_t n_c, float* S_head, int32_t* status,
                             cudaStream_t stream);

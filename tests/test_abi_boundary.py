@@ -206,3 +206,25 @@ def test_head_rejections(lib):
     assert sel(cap=4 * n_c - 1) == INVALID         # 4 heads of 100 rows each
     assert sel(wsb=need - 1) == WS
     assert lib.kvz_select_heads_workspace_size(70000) == 0
+
+
+def test_decode_rejections(lib):
+    b = Bufs()
+    B, G, n_c, d = 2, 4, 500, 128
+    q, K, V = b.get(B * G * d * 2), b.get(B * n_c * d * 2), b.get(B * n_c * d * 2)
+    cnt, off = b.get(B * 4), b.get((B + 1) * 8)
+    out, lse = b.get(B * G * d * 4), b.get(B * G * 4)
+    need = lib.kvz_decode_workspace_size(B, G, n_c, d)
+    assert need > 0
+    ws = b.get(need)
+
+    def call(G_=G, d_=d, wsb=need, qq=q, scale=0.1):
+        return lib.kvz_decode(vp(qq), vp(K), vp(V), B * n_c, vp(cnt), vp(off), B, G_, n_c, d_, scale, vp(out),
+                              vp(lse), vp(ws), wsb, None, None)
+
+    assert call(d_=96) == UNSUPPORTED
+    assert call(G_=9) == UNSUPPORTED
+    assert call(scale=-1.0) == INVALID
+    assert call(wsb=need - 1) == WS
+    assert call(qq=q + 2) == ALIGN
+    assert lib.kvz_decode_workspace_size(B, 9, n_c, d) == 0
