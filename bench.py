@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD,
                     help="llama8b_layer (default, the headline), tiny, llama8b_stack, qwen14b_128k, stress_ragged, "
                          "llama8b_170k_chunked, llama8b_stack_heads")
+    ap.add_argument("--decode", action="store_true",
+                    help="also time one decode step of attention (G queries per KV head) over the pruned cache "
+                         "and over the full cache; adds a 'decode' object to the JSON line")
     ap.add_argument("--layers", type=int, default=0,
                     help="run only the first L layers of the workload (a smaller case for profiling; "
                          "config.workload then names the truncation)")
@@ -383,6 +386,55 @@ def main():
             raise RuntimeError("device status %d during e2e" % int(status.item()))
         e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
 
+    # ---- decode attention over the pruned cache vs the full cache (one step, all heads)
+    dec = None
+    if args.decode:
+        c = ctxs[0]
+        B = w.B
+        gq = torch.Generator(device=dev).manual_seed(11)
+        q = torch.randn((B, w.G, w.d), generator=gq, device=dev).to(torch.bfloat16)
+        if w.in_place:
+            Kd, Vd = c.K.view(B * c.n_c, w.d), c.V.view(B * c.n_c, w.d)
+            off_d = torch.arange(B + 1, dtype=torch.int64, device=dev) * c.n_c
+        else:
+            Kd, Vd, off_d = c.K_out, c.V_out, c.offsets
+        full_cnt = torch.full((B,), c.n_c, dtype=torch.int32, device=dev)
+        full_off = torch.arange(B + 1, dtype=torch.int64, device=dev) * c.n_c
+        Kf, Vf = c.K.view(B * c.n_c, w.d), c.V.view(B * c.n_c, w.d)
+        ws_d = torch.empty(kvz.lib().kvz_decode_workspace_size(B, w.G, c.n_c, w.d), dtype=torch.uint8, device=dev)
+        out_d = torch.empty((B, w.G, w.d), dtype=torch.float32, device=dev)
+        lse_d = torch.empty((B, w.G), dtype=torch.float32, device=dev)
+
+        def time_decode(K_, V_, cnt, off, iters=20):
+            for _ in range(3):
+                kvz.kvz_decode(q, K_, V_, cnt, off, c.n_c, scale=scale, out=out_d, lse2=lse_d, workspace=ws_d,
+                               status=status, stream=stream)
+            ts = []
+            for _ in range(iters):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                kvz.kvz_decode(q, K_, V_, cnt, off, c.n_c, scale=scale, out=out_d, lse2=lse_d, workspace=ws_d,
+                               status=status, stream=stream)
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                ts.append(e0.elapsed_time(e1))
+            return sorted(ts)[len(ts) // 2]
+
+        t_pruned = time_decode(Kd, Vd, c.counts, off_d)
+        t_full = time_decode(Kf, Vf, full_cnt, full_off)
+        if int(status.item()) != 0:
+            raise RuntimeError("device status %d during decode" % int(status.item()))
+        kept_rows = nums["kept"]
+        pk0 = peaks()
+        byt = kept_rows * w.d * 2 * 2
+        dec = {"ms": t_pruned, "bytes": byt, "gbs": byt / (t_pruned * 1e-3) / 1e9,
+               "frac_hbm": byt / (t_pruned * 1e-3) / 1e9 / pk0["hbm_gbs"],
+               "full_cache_ms": t_full, "full_cache_gbs": B * c.n_c * w.d * 4 / (t_full * 1e-3) / 1e9,
+               "speedup_vs_full_cache": t_full / t_pruned,
+               "what": "one decode step: %d KV heads x %d grouped queries over the pruned cache (%d kept rows) vs "
+                       "the full cache; median of 20, L2 flushed before each" % (B, w.G, kept_rows)}
+
     red = max_over_ranks([ms_step, e2e["ms"] if e2e else 0.0] + part_ms, device=dev)
     ms_step, e2e_ms, part_ms = red[0], red[1], red[2:]
 
@@ -427,6 +479,8 @@ def main():
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
+    if dec is not None:
+        line["decode"] = dec
     if e2e is not None:
         line["e2e"] = {"value": nums["pairs_per_step"] * world / (e2e_ms * 1e-3), "unit": UNIT,
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms}
