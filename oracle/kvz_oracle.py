@@ -47,6 +47,9 @@ __all__ = [
     "head_scores",
     "select_heads",
     "decode_attention",
+    "select_protected",
+    "quantize_rows",
+    "compact_quantized",
     "compact",
     "visible_pairs",
 ]
@@ -296,6 +299,68 @@ def decode_attention(q, K_out, V_out, counts, offsets, scale):
             out[b, g] = (w @ Vb) / np.sum(w)
             lse2[b, g] = (zm + np.log(np.sum(w))) / math.log(2.0)
     return out, lse2
+
+
+# ---------------------------------------------------------------------------
+# Protected prefix (KVzip §4.1: the initial system prompt's KV pairs are kept
+# intact) and int8 quantisation of the pruned cache (KVzip §4.2, "KV
+# quantization": KVzip composes with a quantised cache)
+# ---------------------------------------------------------------------------
+def select_protected(S, ratio, mode, n_protect):
+    """Selection with the first n_protect positions of every head always kept.
+
+    The ratio applies to the other positions: floor(ratio * (n_c - n_protect))
+    of them per head, or floor(ratio * B * (n_c - n_protect)) across all heads,
+    the highest scores first, ties to the lower flattened index (b, j).
+    Returns (idx, counts, offsets) as ``select``."""
+    S = np.asarray(S, dtype=np.float32)
+    B, n_c = S.shape
+    p = int(n_protect)
+    if not (0 <= p <= n_c):
+        raise ValueError("n_protect must lie in [0, n_c]")
+    rest = S[:, p:]
+    free = n_c - p
+    if mode == "per_head":
+        k = keep_count(free, ratio)
+        chosen = [np.argsort(-rest[b], kind="stable")[:k] + p for b in range(B)]
+    elif mode == "global":
+        k = keep_count(B * free, ratio)
+        order = np.argsort(-rest.reshape(-1), kind="stable")[:k]
+        heads, cols = order // max(free, 1), order % max(free, 1)
+        chosen = [cols[heads == b] + p for b in range(B)]
+    else:
+        raise ValueError("mode must be 'per_head' or 'global'")
+    per_head = [np.sort(np.concatenate([np.arange(p), c])).astype(np.int64) for c in chosen]
+    counts = np.array([len(x) for x in per_head], dtype=np.int32)
+    offsets = np.zeros(B + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    idx = np.concatenate(per_head).astype(np.int32) if B else np.zeros(0, np.int32)
+    return idx, counts, offsets
+
+
+def quantize_rows(X):
+    """Symmetric per-row int8 codes of X [rows, d] (float32 arithmetic).
+
+    absmax = max |x| of the row; scale = absmax / 127; code =
+    clip(rint(x * (127 / absmax)), -127, 127), rint rounding half to even.
+    The divisions and the product are single float32 operations, in this
+    order.  A row of zeros gets code 0 and scale 0."""
+    X = np.asarray(X, dtype=np.float32)
+    absmax = np.max(np.abs(X), axis=1)
+    scale = (absmax / np.float32(127.0)).astype(np.float32)
+    with np.errstate(divide="ignore"):
+        inv = np.where(absmax > 0, np.float32(127.0) / absmax, np.float32(0.0)).astype(np.float32)
+    codes = np.clip(np.rint((X * inv[:, None]).astype(np.float32)), -127, 127).astype(np.int8)
+    return codes, scale
+
+
+def compact_quantized(K_bits, V_bits, idx, counts, offsets):
+    """The packed pruned cache as int8 codes with one fp32 scale per row:
+    (Kq, K_scale, Vq, V_scale).  K_bits/V_bits are bf16 bit patterns."""
+    Kr, Vr = compact(K_bits, V_bits, idx, counts, offsets)
+    Kq, Ks = quantize_rows(bf16_bits_to_f64(Kr).astype(np.float32))
+    Vq, Vs = quantize_rows(bf16_bits_to_f64(Vr).astype(np.float32))
+    return Kq, Ks, Vq, Vs
 
 
 # ---------------------------------------------------------------------------

@@ -464,3 +464,64 @@ def test_decode_on_the_kept_set_is_the_renormalised_full_softmax():
         p = scipy.special.softmax(s * (K @ q[0, g]))
         pk = p[keep] / p[keep].sum()
         np.testing.assert_allclose(out[0, g], pk @ V[keep], rtol=1e-12, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Protected prefix and int8 rows
+# --------------------------------------------------------------------------
+def test_int8_rows_golden():
+    with open(os.path.join(os.path.dirname(__file__), "golden", "int8_row_quantization.json")) as f:
+        g = json.load(f)
+    codes, scales = orc.quantize_rows(np.array(g["rows"], dtype=np.float32))
+    assert codes.tolist() == g["codes"] and scales.tolist() == g["scales"]
+
+
+def test_int8_rows_properties():
+    rng = np.random.default_rng(51)
+    X = (rng.standard_normal((40, 128)) * rng.random((40, 1)) * 5).astype(np.float32)
+    X[3] = 0.0
+    codes, scales = orc.quantize_rows(X)
+    assert codes.dtype == np.int8 and codes[3].tolist() == [0] * 128 and scales[3] == 0
+    for r in range(40):
+        if r == 3:
+            continue
+        j = np.argmax(np.abs(X[r]))
+        assert abs(int(codes[r, j])) == 127                       # the largest magnitude maps to the end code
+        err = np.abs(X[r] - codes[r].astype(np.float64) * scales[r])
+        assert np.all(err <= 0.5 * scales[r] * (1 + 1e-5))        # round to nearest: half a step at most
+    np.testing.assert_array_equal(orc.quantize_rows(-X)[0], -codes)    # symmetric
+
+
+@pytest.mark.parametrize("mode", ["per_head", "global"])
+def test_select_protected_by_exhaustive_search(mode):
+    rng = np.random.default_rng(52 if mode == "per_head" else 53)
+    B, n_c, p = 2, 5, 2
+    for trial in range(30):
+        S = (rng.integers(0, 3, (B, n_c)) / 2).astype(np.float32)
+        for ratio in (0.0, 0.34, 0.5, 1.0):
+            idx, counts, offsets = orc.select_protected(S, ratio, mode, p)
+            kept = {(b, int(j)) for b in range(B) for j in idx[offsets[b]:offsets[b + 1]]}
+            assert all((b, j) in kept for b in range(B) for j in range(p))    # the prefix is always there
+            free = [(b, j) for b in range(B) for j in range(p, n_c)]
+            if mode == "per_head":
+                k = orc.keep_count(n_c - p, ratio)
+                groups = [[x for x in free if x[0] == b] for b in range(B)]
+            else:
+                k = orc.keep_count(B * (n_c - p), ratio)
+                groups = [free]
+            want = set()
+            for grp in groups:
+                # the k of the group ranked first by (score desc, flattened index asc)
+                best = min(itertools.combinations(grp, k), key=lambda c: sorted((-S[x], x) for x in c)) if k else ()
+                want |= set(best)
+            assert kept - {(b, j) for b in range(B) for j in range(p)} == want
+
+
+def test_select_protected_zero_prefix_is_select():
+    rng = np.random.default_rng(54)
+    S = rng.random((3, 40)).astype(np.float32)
+    for mode in ("per_head", "global"):
+        a = orc.select_protected(S, 0.3, mode, 0)
+        b_ = orc.select(S, 0.3, mode)
+        for x, y in zip(a, b_):
+            np.testing.assert_array_equal(x, y)
