@@ -228,6 +228,41 @@ kvz_status kvz_select_heads(const float* S_head, int64_t B, int64_t n_c, double 
                             size_t workspace_bytes, int32_t* d_status, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Selection with a protected prefix (KVzip §4.1: the initial system         */
+/* prompt's KV pairs are kept intact).                                       */
+/*                                                                          */
+/* As kvz_select, except that positions j < n_protect of every head are      */
+/* always kept and the ratio applies to the other positions: per head        */
+/* n_protect + floor(ratio * (n_c - n_protect)) kept; globally               */
+/* B * n_protect + floor(ratio * B * (n_c - n_protect)).  Ties among the     */
+/* unprotected positions go to the lower flattened index.  idx capacity as   */
+/* those totals (times B per head).  0 <= n_protect <= n_c; same workspace   */
+/* as kvz_select.                                                            */
+/* ------------------------------------------------------------------------ */
+kvz_status kvz_select_protected(const float* S, int64_t B, int64_t n_c, double ratio, int mode,
+                                int64_t n_protect, int32_t* idx, int64_t idx_capacity, int32_t* counts,
+                                int64_t* offsets, void* workspace, size_t workspace_bytes,
+                                int32_t* d_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Compaction into an int8 cache (KVzip §4.2, "KV quantization": the pruned  */
+/* cache composes with a quantised one).                                     */
+/*                                                                          */
+/* Out-of-place kvz_compact whose destination rows are symmetric int8 codes */
+/* with one fp32 scale per row: with a = max |x| over the row's d values,   */
+/* scale = a / 127 and code = rint(x * (127 / a)) clamped to [-127, 127]    */
+/* (round half to even; single IEEE float32 operations in that order); a    */
+/* row of zeros gets code 0 and scale 0.  x ~= code * scale.                */
+/* Layout: Kq, Vq [rows][d] int8 (16-byte aligned); K_scale, V_scale [rows] */
+/* fp32; row of head b's p-th kept key = (out_offsets ? out_offsets[b] :    */
+/* offsets[b]) + p.  Device-detected errors as kvz_compact.                 */
+/* ------------------------------------------------------------------------ */
+kvz_status kvz_compact_int8(const void* K, const void* V, int64_t B, int64_t n_c, int d,
+                            const int32_t* idx, const int32_t* counts, const int64_t* offsets,
+                            const int64_t* out_offsets, int8_t* Kq, int8_t* Vq, float* K_scale,
+                            float* V_scale, int32_t* d_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Compaction.                                                               */
 /*                                                                          */
 /* KVzip §2.1: the pruned cache K_p is a subset of the full cache K_c that   */

@@ -65,6 +65,8 @@ _SIGS = {
     "kvz_select": (_i32, [_vp, _i64, _i64, _f64, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
     "kvz_compact_workspace_size": (_sz, [_i64, _i64]),
     "kvz_compact": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "kvz_select_protected": (_i32, [_vp, _i64, _i64, _f64, _i32, _i64, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "kvz_compact_int8": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "kvz_decode_workspace_size": (_sz, [_i64, _i32, _i64, _i32]),
     "kvz_decode": (_i32, [_vp, _vp, _vp, _i64, _vp, _vp, _i64, _i32, _i64, _i32, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
     "kvz_head_score": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
@@ -417,3 +419,46 @@ def kvz_decode(q, K_out, V_out, counts, offsets, n_c: int, scale: Optional[float
         _ptr(out), _ptr(lse2), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
         _stream(stream)))
     return out, lse2
+
+
+def kvz_select_protected(S, ratio: float, mode="per_head", n_protect: int = 0, idx=None, counts=None, offsets=None,
+                         workspace=None, status=None, stream=None):
+    """kvz_select with the first n_protect positions of every head always
+    kept (KVzip §4.1 system prompt); the ratio applies to the rest."""
+    _need_cuda(S, idx, counts, offsets, workspace, status)
+    B, n_c = S.shape
+    m = _mode(mode)
+    free = n_c - n_protect
+    k = (B * n_protect + kvz_keep_count(B * free, ratio)) if m == GLOBAL else (n_protect + kvz_keep_count(free, ratio))
+    cap = k if m == GLOBAL else B * k
+    dev = S.device
+    if idx is None:
+        idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+    if counts is None:
+        counts = torch.empty(B, dtype=torch.int32, device=dev)
+    if offsets is None:
+        offsets = torch.empty(B + 1, dtype=torch.int64, device=dev)
+    if workspace is None:
+        workspace = torch.empty(kvz_select_workspace_size(B, n_c, m), dtype=torch.uint8, device=dev)
+    _check("kvz_select_protected", lib().kvz_select_protected(
+        _ptr(S), B, n_c, float(ratio), m, int(n_protect), _ptr(idx), idx.numel(), _ptr(counts), _ptr(offsets),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)))
+    return idx, counts, offsets
+
+
+def kvz_compact_int8(K, V, idx, counts, offsets, out_offsets=None, out_rows: Optional[int] = None, Kq=None, Vq=None,
+                     K_scale=None, V_scale=None, status=None, stream=None):
+    """Out-of-place compaction into int8 codes with one fp32 scale per row
+    (KVzip §4.2 KV quantisation); returns (Kq, K_scale, Vq, V_scale)."""
+    _need_cuda(K, V, idx, counts, offsets, out_offsets, Kq, Vq, K_scale, V_scale, status)
+    B, n_c, d = K.shape
+    rows = B * n_c if out_rows is None else int(out_rows)
+    dev = K.device
+    Kq = torch.empty((rows, d), dtype=torch.int8, device=dev) if Kq is None else Kq
+    Vq = torch.empty((rows, d), dtype=torch.int8, device=dev) if Vq is None else Vq
+    K_scale = torch.empty(rows, dtype=torch.float32, device=dev) if K_scale is None else K_scale
+    V_scale = torch.empty(rows, dtype=torch.float32, device=dev) if V_scale is None else V_scale
+    _check("kvz_compact_int8", lib().kvz_compact_int8(
+        _ptr(K), _ptr(V), B, n_c, d, _ptr(idx), _ptr(counts), _ptr(offsets), _ptr(out_offsets), _ptr(Kq), _ptr(Vq),
+        _ptr(K_scale), _ptr(V_scale), _ptr(status), _stream(stream)))
+    return Kq, K_scale, Vq, V_scale

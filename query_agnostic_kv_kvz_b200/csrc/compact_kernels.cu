@@ -140,6 +140,114 @@ __global__ void __launch_bounds__(kGatherThreads)
   }
 }
 
+// Out of place into int8 (KVzip analysis report, §4.2 "KV quantization": the
+// pruned cache composes with a quantised one).  Symmetric per-row codes: with
+// a = max |x| over the row, scale = a / 127 and code = rint(x * (127 / a)),
+// clamped to [-127, 127]; a row of zeros has code 0 and scale 0.  The two
+// divisions and the product are single IEEE float32 operations (no fused or
+// approximate forms), so the codes are reproducible to the bit.  A row is
+// read by vpr threads (16 bytes each); its absmax comes from a shuffle
+// reduction over them.  HBM-bound: 4d bytes read, 2d + 8 written per row.
+constexpr int kQuantThreads = 256;
+constexpr int kQuantUnroll = 4;
+
+__device__ __forceinline__ void quant8(const int4& w, float inv, int8_t* dst) {
+  const uint32_t u[4] = {static_cast<uint32_t>(w.x), static_cast<uint32_t>(w.y), static_cast<uint32_t>(w.z),
+                         static_cast<uint32_t>(w.w)};
+  uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const uint32_t h = (u[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu;
+    const float x = __uint_as_float(h << 16);
+    int q = __float2int_rn(__fmul_rn(x, inv));
+    q = q > 127 ? 127 : (q < -127 ? -127 : q);
+    packed[e >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << ((e & 3) * 8);
+  }
+  *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+}
+
+__device__ __forceinline__ float absmax8(const int4& w) {
+  const uint32_t u[4] = {static_cast<uint32_t>(w.x), static_cast<uint32_t>(w.y), static_cast<uint32_t>(w.z),
+                         static_cast<uint32_t>(w.w)};
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = fmaxf(m, fabsf(__uint_as_float(u[i] << 16)));
+    m = fmaxf(m, fabsf(__uint_as_float(u[i] & 0xFFFF0000u)));
+  }
+  return m;
+}
+
+__global__ void __launch_bounds__(kQuantThreads)
+    compact_int8_kernel(const int4* __restrict__ K, const int4* __restrict__ V, int64_t B, int64_t n_c, int vpr,
+                        const int32_t* __restrict__ idx, const int64_t* __restrict__ offsets,
+                        const int64_t* __restrict__ out_offsets, int8_t* __restrict__ Kq, int8_t* __restrict__ Vq,
+                        float* __restrict__ Ks, float* __restrict__ Vs, int32_t* status) {
+  __shared__ int64_t s_head;
+  const int64_t total = offsets[B];
+  const int rows_per_step = kQuantThreads / vpr;
+  const int rows_per_blk = rows_per_step * kQuantUnroll;
+  const int my_row = threadIdx.x / vpr;
+  const int vec = threadIdx.x % vpr;
+  for (int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_blk; r0 < total;
+       r0 += static_cast<int64_t>(gridDim.x) * rows_per_blk) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int64_t lo = 0, hi = B - 1;                                 // largest b with offsets[b] <= r0
+      while (lo < hi) {
+        const int64_t mid = (lo + hi + 1) >> 1;
+        if (offsets[mid] <= r0) lo = mid; else hi = mid - 1;
+      }
+      s_head = lo;
+    }
+    __syncthreads();
+    int64_t hb = s_head;
+    int4 kv[kQuantUnroll], vv[kQuantUnroll];
+    int64_t dst[kQuantUnroll];
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const int64_t slot = r0 + u * rows_per_step + my_row;
+      dst[u] = -1;
+      kv[u] = vv[u] = make_int4(0, 0, 0, 0);
+      if (slot < total) {
+        while (hb + 1 < B && offsets[hb + 1] <= slot) ++hb;
+        const int64_t j = idx[slot];
+        if (j < 0 || j >= n_c) {
+          report_err(status, KVZ_ERR_INVALID_ARG);
+        } else {
+          const int64_t src = (hb * n_c + j) * vpr + vec;
+          const int64_t base = out_offsets != nullptr ? out_offsets[hb] : offsets[hb];
+          dst[u] = base + (slot - offsets[hb]);
+          kv[u] = ld_stream(K + src);
+          vv[u] = ld_stream(V + src);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      // the vpr threads of a row are consecutive lanes of one warp
+      float ak = absmax8(kv[u]), av = absmax8(vv[u]);
+#pragma unroll
+      for (int o2 = 1; o2 < 16; o2 <<= 1) {
+        if (o2 < vpr) {
+          ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, o2));
+          av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, o2));
+        }
+      }
+      if (dst[u] >= 0) {
+        const float ik = ak > 0.0f ? __fdiv_rn(127.0f, ak) : 0.0f;
+        const float iv = av > 0.0f ? __fdiv_rn(127.0f, av) : 0.0f;
+        quant8(kv[u], ik, Kq + dst[u] * vpr * 8 + vec * 8);
+        quant8(vv[u], iv, Vq + dst[u] * vpr * 8 + vec * 8);
+        if (vec == 0) {
+          Ks[dst[u]] = __fdiv_rn(ak, 127.0f);
+          Vs[dst[u]] = __fdiv_rn(av, 127.0f);
+        }
+      }
+    }
+  }
+}
+
 // Dependencies of in-place compaction.  Slot chunk c (slots [cC, (c+1)C))
 // writes rows [cC, (c+1)C).  Because idx ascends within a head, the slots
 // whose source rows lie in that range form one contiguous run
@@ -354,6 +462,20 @@ cudaError_t launch_compact_gather(const void* K, const void* V, int64_t B, int64
   compact_gather_kernel<<<static_cast<unsigned>(blocks), kGatherThreads, 0, stream>>>(
       static_cast<const int4*>(K), static_cast<const int4*>(V), B, n_c, vpr, idx, offsets, out_offsets,
       static_cast<int4*>(K_out), static_cast<int4*>(V_out), status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compact_int8(const void* K, const void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
+                                const int64_t* offsets, const int64_t* out_offsets, int8_t* Kq, int8_t* Vq,
+                                float* K_scale, float* V_scale, int32_t* status, cudaStream_t stream) {
+  const int vpr = d / 8;
+  const int rows_per_blk = (kQuantThreads / vpr) * kQuantUnroll;
+  int64_t blocks = (B * n_c + rows_per_blk - 1) / rows_per_blk;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  if (blocks < 1) blocks = 1;
+  compact_int8_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
+      static_cast<const int4*>(K), static_cast<const int4*>(V), B, n_c, vpr, idx, offsets, out_offsets, Kq, Vq,
+      K_scale, V_scale, status);
   return cudaGetLastError();
 }
 

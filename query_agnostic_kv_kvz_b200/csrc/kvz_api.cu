@@ -374,8 +374,34 @@ kvz_status kvz_select(const float* S, int64_t B, int64_t n_c, double ratio, int 
   const kvz::SelWorkspace lay = kvz::select_workspace(B, n_c, mode);
   if (workspace == nullptr || workspace_bytes < lay.bytes) return KVZ_ERR_WORKSPACE;
   if (!aligned(workspace, 16)) return KVZ_ERR_ALIGNMENT;
-  return kvz::launch_select(S, B, n_c, mode, k, idx, counts, offsets, workspace, lay, d_status, stream) ==
+  return kvz::launch_select(S, B, n_c, 0, mode, k, idx, counts, offsets, workspace, lay, d_status, stream) ==
                  cudaSuccess
+             ? KVZ_OK
+             : KVZ_ERR_CUDA;
+}
+
+kvz_status kvz_select_protected(const float* S, int64_t B, int64_t n_c, double ratio, int mode, int64_t n_protect,
+                                int32_t* idx, int64_t idx_capacity, int32_t* counts, int64_t* offsets,
+                                void* workspace, size_t workspace_bytes, int32_t* d_status, cudaStream_t stream) {
+  if (S == nullptr || counts == nullptr || offsets == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (mode != KVZ_PER_HEAD && mode != KVZ_GLOBAL) return KVZ_ERR_INVALID_ARG;
+  if (B < 1 || B > 65535 || n_c < 1 || n_c > kMaxRows) return KVZ_ERR_INVALID_ARG;
+  if (B * n_c >= (int64_t(1) << 32)) return KVZ_ERR_INVALID_ARG;
+  if (!(ratio >= 0.0 && ratio <= 1.0) || n_protect < 0 || n_protect > n_c) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(S, 4) || !aligned(counts, 4) || !aligned(offsets, 8) || (idx && !aligned(idx, 4)))
+    return KVZ_ERR_ALIGNMENT;
+  // the protected positions rank above every score, so keeping them plus the
+  // ratio's share of the rest is a top-k of k = protected + share
+  const int64_t free = n_c - n_protect;
+  const int64_t k = mode == KVZ_GLOBAL ? B * n_protect + kvz_keep_count(B * free, ratio)
+                                       : n_protect + kvz_keep_count(free, ratio);
+  const int64_t need = mode == KVZ_GLOBAL ? k : B * k;
+  if (idx_capacity < need || (need > 0 && idx == nullptr)) return KVZ_ERR_INVALID_ARG;
+  const kvz::SelWorkspace lay = kvz::select_workspace(B, n_c, mode);
+  if (workspace == nullptr || workspace_bytes < lay.bytes) return KVZ_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return KVZ_ERR_ALIGNMENT;
+  return kvz::launch_select(S, B, n_c, n_protect, mode, k, idx, counts, offsets, workspace, lay, d_status,
+                            stream) == cudaSuccess
              ? KVZ_OK
              : KVZ_ERR_CUDA;
 }
@@ -460,6 +486,24 @@ kvz_status kvz_decode(const void* q, const void* K_out, const void* V_out, int64
   a.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((parts * 8 + 255) & ~size_t(255)));
   a.status = d_status;
   return kvz::launch_decode(d, tmK, tmV, a, out, lse2, stream) == cudaSuccess ? KVZ_OK : KVZ_ERR_CUDA;
+}
+
+kvz_status kvz_compact_int8(const void* K, const void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
+                            const int32_t* counts, const int64_t* offsets, const int64_t* out_offsets, int8_t* Kq,
+                            int8_t* Vq, float* K_scale, float* V_scale, int32_t* d_status, cudaStream_t stream) {
+  if (K == nullptr || V == nullptr || idx == nullptr || counts == nullptr || offsets == nullptr || Kq == nullptr ||
+      Vq == nullptr || K_scale == nullptr || V_scale == nullptr)
+    return KVZ_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return KVZ_ERR_UNSUPPORTED;
+  if (B < 1 || B > 0x7FFFFFFF / 8 || n_c < 1 || n_c > kMaxRows) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(K, 16) || !aligned(V, 16) || !aligned(Kq, 16) || !aligned(Vq, 16) || !aligned(K_scale, 4) ||
+      !aligned(V_scale, 4) || !aligned(idx, 4) || !aligned(counts, 4) || !aligned(offsets, 8) ||
+      (out_offsets && !aligned(out_offsets, 8)))
+    return KVZ_ERR_ALIGNMENT;
+  return kvz::launch_compact_int8(K, V, B, n_c, d, idx, offsets, out_offsets, Kq, Vq, K_scale, V_scale, d_status,
+                                  stream) == cudaSuccess
+             ? KVZ_OK
+             : KVZ_ERR_CUDA;
 }
 
 size_t kvz_compact_workspace_size(int64_t B, int64_t n_c) {

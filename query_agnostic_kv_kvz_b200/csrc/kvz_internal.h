@@ -76,8 +76,8 @@ struct SelWorkspace {
   size_t off_state, off_hist, off_cg, off_ce, off_eqb, off_cbase, off_head_eq, off_head_base;
 };
 SelWorkspace select_workspace(int64_t B, int64_t n_c, int mode);
-cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int mode, int64_t k, int32_t* idx,
-                          int32_t* counts, int64_t* offsets, void* ws, const SelWorkspace& lay,
+cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int64_t n_protect, int mode, int64_t k,
+                          int32_t* idx, int32_t* counts, int64_t* offsets, void* ws, const SelWorkspace& lay,
                           int32_t* status, cudaStream_t stream);
 
 // Compaction.
@@ -90,5 +90,9 @@ cudaError_t launch_compact_inplace(void* K, void* V, int64_t B, int64_t n_c, int
                                    const int32_t* counts, const int64_t* offsets, uint32_t* ws, int32_t* status,
                                    cudaStream_t stream);
 size_t compact_workspace_bytes(int64_t B, int64_t n_c);
+// Out-of-place compaction into int8 codes with one fp32 scale per row.
+cudaError_t launch_compact_int8(const void* K, const void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
+                                const int64_t* offsets, const int64_t* out_offsets, int8_t* Kq, int8_t* Vq,
+                                float* K_scale, float* V_scale, int32_t* status, cudaStream_t stream);
 
 }  // namespace kvz

@@ -50,6 +50,12 @@ __device__ __forceinline__ uint32_t score_key(float s, int32_t* status) {
   return u;
 }
 
+// Key of position j of a head: the first n_protect positions rank above
+// every score (their key exceeds +inf's pattern), the rest as score_key.
+__device__ __forceinline__ uint32_t select_key(const float* src, int64_t j, int64_t n_protect, int32_t* status) {
+  return j < n_protect ? 0xFFFFFFFFu : score_key(__ldg(src + j), status);
+}
+
 __device__ __forceinline__ int digit_shift(int pass) { return pass == 0 ? 21 : (pass == 1 ? 10 : 0); }
 __device__ __forceinline__ uint32_t digit_mask(int pass) { return pass == 2 ? 0x3FFu : 0x7FFu; }
 
@@ -102,8 +108,9 @@ __global__ void sel_init(SelState* st, int nseg, unsigned long long k, uint32_t*
 }
 
 // Histogram of the current digit over keys that match the prefix.
-__global__ void __launch_bounds__(kSelThreads) sel_hist(const float* S, int64_t n_c, int mode, int pass,
-                                                        const SelState* st, uint32_t* hist, int32_t* status) {
+__global__ void __launch_bounds__(kSelThreads) sel_hist(const float* S, int64_t n_c, int64_t n_protect, int mode,
+                                                        int pass, const SelState* st, uint32_t* hist,
+                                                        int32_t* status) {
   __shared__ uint32_t h[kBins];
   const int b = blockIdx.y;
   const int seg = mode == KVZ_GLOBAL ? 0 : b;
@@ -118,7 +125,7 @@ __global__ void __launch_bounds__(kSelThreads) sel_hist(const float* S, int64_t 
   const uint32_t dm = digit_mask(pass);
   int32_t* st_ptr = pass == 0 ? status : nullptr;
   for (int e = threadIdx.x; e < lim; e += kSelThreads) {
-    const uint32_t key = score_key(__ldg(src + e), st_ptr);
+    const uint32_t key = select_key(src - c0, c0 + e, n_protect, st_ptr);
     if ((key & s.mask) == s.prefix) atomicAdd(&h[(key >> sh) & dm], 1u);
   }
   __syncthreads();
@@ -165,8 +172,9 @@ __global__ void __launch_bounds__(1024) sel_pick(int pass, SelState* st, uint32_
 }
 
 // Per chunk: number of keys above T and equal to T.
-__global__ void __launch_bounds__(kSelThreads) sel_count(const float* S, int64_t n_c, int mode, int nchunk,
-                                                         const SelState* st, uint32_t* cg, uint32_t* ce) {
+__global__ void __launch_bounds__(kSelThreads) sel_count(const float* S, int64_t n_c, int64_t n_protect, int mode,
+                                                         int nchunk, const SelState* st, uint32_t* cg,
+                                                         uint32_t* ce) {
   __shared__ unsigned long long wbuf[32];
   const int b = blockIdx.y;
   const int seg = mode == KVZ_GLOBAL ? 0 : b;
@@ -176,7 +184,7 @@ __global__ void __launch_bounds__(kSelThreads) sel_count(const float* S, int64_t
   const float* src = S + static_cast<int64_t>(b) * n_c + c0;
   uint32_t gt = 0u, eq = 0u;
   for (int e = threadIdx.x; e < lim; e += kSelThreads) {
-    const uint32_t key = score_key(__ldg(src + e), nullptr);
+    const uint32_t key = select_key(src - c0, c0 + e, n_protect, nullptr);
     gt += key > T ? 1u : 0u;
     eq += key == T ? 1u : 0u;
   }
@@ -253,10 +261,10 @@ __global__ void __launch_bounds__(1024) sel_scan(int64_t B, int nchunk, int mode
 }
 
 // Per chunk: write the kept positions in ascending order.
-__global__ void __launch_bounds__(kSelThreads) sel_write(const float* S, int64_t n_c, int mode, int nchunk,
-                                                         const SelState* st, const unsigned long long* eqb,
-                                                         const uint32_t* cbase, const int64_t* offsets,
-                                                         int32_t* idx) {
+__global__ void __launch_bounds__(kSelThreads) sel_write(const float* S, int64_t n_c, int64_t n_protect, int mode,
+                                                         int nchunk, const SelState* st,
+                                                         const unsigned long long* eqb, const uint32_t* cbase,
+                                                         const int64_t* offsets, int32_t* idx) {
   __shared__ uint32_t wbuf[32];
   const int b = blockIdx.y;
   const int seg = mode == KVZ_GLOBAL ? 0 : b;
@@ -274,7 +282,7 @@ __global__ void __launch_bounds__(kSelThreads) sel_write(const float* S, int64_t
 #pragma unroll
   for (int it = 0; it < kSelItems; ++it) {
     const int l = l0 + it;
-    key[it] = l < lim ? score_key(__ldg(src + l), nullptr) : 0u;
+    key[it] = l < lim ? select_key(src - c0, c0 + l, n_protect, nullptr) : 0u;
     neq += (l < lim && key[it] == T) ? 1u : 0u;
   }
   const uint32_t eq_incl = block_inclusive_sum<uint32_t>(neq, wbuf);
@@ -314,8 +322,9 @@ constexpr int64_t kHeadStageMax = 49152;                 // scores staged in sha
 
 template <bool STAGED>
 __global__ void __launch_bounds__(kHeadThreads) sel_head_kernel(const float* S, int64_t B, int64_t n_c,
-                                                                int64_t k, int32_t* idx, int32_t* counts,
-                                                                int64_t* offsets, int32_t* status) {
+                                                                int64_t n_protect, int64_t k, int32_t* idx,
+                                                                int32_t* counts, int64_t* offsets,
+                                                                int32_t* status) {
   extern __shared__ uint32_t skey[];                     // STAGED: the head's keys
   __shared__ uint32_t hist[kBins];
   __shared__ unsigned long long wbuf[32];
@@ -334,7 +343,7 @@ __global__ void __launch_bounds__(kHeadThreads) sel_head_kernel(const float* S, 
     s_eq = 0ull;
   }
   if (k == 0) return;
-  auto key_at = [&](int64_t j) -> uint32_t { return STAGED ? skey[j] : score_key(__ldg(src + j), nullptr); };
+  auto key_at = [&](int64_t j) -> uint32_t { return STAGED ? skey[j] : select_key(src, j, n_protect, nullptr); };
 
   for (int pass = 0; pass < 3; ++pass) {
     for (int e = threadIdx.x; e < kBins; e += kHeadThreads) hist[e] = 0u;
@@ -345,7 +354,7 @@ __global__ void __launch_bounds__(kHeadThreads) sel_head_kernel(const float* S, 
     for (int64_t j = threadIdx.x; j < n_c; j += kHeadThreads) {
       uint32_t key;
       if (pass == 0) {
-        key = score_key(__ldg(src + j), status);
+        key = select_key(src, j, n_protect, status);
         if (STAGED) skey[j] = key;
       } else {
         key = key_at(j);
@@ -445,8 +454,8 @@ SelWorkspace select_workspace(int64_t B, int64_t n_c, int mode) {
   return w;
 }
 
-cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int mode, int64_t k, int32_t* idx,
-                          int32_t* counts, int64_t* offsets, void* ws, const SelWorkspace& lay,
+cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int64_t n_protect, int mode, int64_t k,
+                          int32_t* idx, int32_t* counts, int64_t* offsets, void* ws, const SelWorkspace& lay,
                           int32_t* status, cudaStream_t stream) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   SelState* st = reinterpret_cast<SelState*>(base + lay.off_state);
@@ -463,11 +472,11 @@ cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int mode, int6
       cudaError_t e = cudaFuncSetAttribute(sel_head_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(kHeadStageMax * 4));
       if (e != cudaSuccess) return e;
-      sel_head_kernel<true><<<static_cast<unsigned>(B), kHeadThreads, smem, stream>>>(S, B, n_c, k, idx, counts,
-                                                                                    offsets, status);
+      sel_head_kernel<true><<<static_cast<unsigned>(B), kHeadThreads, smem, stream>>>(S, B, n_c, n_protect, k, idx,
+                                                                                    counts, offsets, status);
     } else {
-      sel_head_kernel<false><<<static_cast<unsigned>(B), kHeadThreads, 0, stream>>>(S, B, n_c, k, idx, counts,
-                                                                                   offsets, status);
+      sel_head_kernel<false><<<static_cast<unsigned>(B), kHeadThreads, 0, stream>>>(S, B, n_c, n_protect, k, idx,
+                                                                                   counts, offsets, status);
     }
     return cudaGetLastError();
   }
@@ -478,12 +487,12 @@ cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int mode, int6
   if (init_blocks > 1184) init_blocks = 1184;
   sel_init<<<static_cast<unsigned>(init_blocks), 256, 0, stream>>>(st, nseg, static_cast<unsigned long long>(k), hist);
   for (int pass = 0; pass < 3; ++pass) {
-    sel_hist<<<grid, kSelThreads, 0, stream>>>(S, n_c, mode, pass, st, hist, status);
+    sel_hist<<<grid, kSelThreads, 0, stream>>>(S, n_c, n_protect, mode, pass, st, hist, status);
     sel_pick<<<nseg, 1024, 0, stream>>>(pass, st, hist);
   }
-  sel_count<<<grid, kSelThreads, 0, stream>>>(S, n_c, mode, nchunk, st, cg, ce);
+  sel_count<<<grid, kSelThreads, 0, stream>>>(S, n_c, n_protect, mode, nchunk, st, cg, ce);
   sel_scan<<<1, 1024, 0, stream>>>(B, nchunk, mode, st, cg, ce, eqb, cbase, head_eq, head_base, counts, offsets);
-  sel_write<<<grid, kSelThreads, 0, stream>>>(S, n_c, mode, nchunk, st, eqb, cbase, offsets, idx);
+  sel_write<<<grid, kSelThreads, 0, stream>>>(S, n_c, n_protect, mode, nchunk, st, eqb, cbase, offsets, idx);
   return cudaGetLastError();
 }
 

@@ -228,3 +228,23 @@ def test_decode_rejections(lib):
     assert call(wsb=need - 1) == WS
     assert call(qq=q + 2) == ALIGN
     assert lib.kvz_decode_workspace_size(B, 9, n_c, d) == 0
+
+
+def test_protect_and_int8_rejections(lib):
+    b = Bufs()
+    B, n_c, d = 2, 256, 128
+    S = b.get(B * n_c * 4)
+    idx, cnt, off = b.get(B * n_c * 4), b.get(B * 4), b.get((B + 1) * 8)
+    wsn = lib.kvz_select_workspace_size(B, n_c, 0)
+    ws = b.get(wsn)
+    sel = lambda p, cap=B * n_c: lib.kvz_select_protected(vp(S), B, n_c, 0.3, 0, p, vp(idx), cap, vp(cnt), vp(off),
+                                                        vp(ws), wsn, None, None)
+    assert sel(-1) == INVALID
+    assert sel(n_c + 1) == INVALID
+    assert sel(10, cap=B * (10 + 73) - 1) == INVALID      # per head: 10 + floor(0.3 * 246) = 83
+    K, V = b.get(B * n_c * d * 2), b.get(B * n_c * d * 2)
+    Kq, Vq, Ks, Vs = b.get(B * n_c * d), b.get(B * n_c * d), b.get(B * n_c * 4), b.get(B * n_c * 4)
+    q8 = lambda d_=d, kq=Kq: lib.kvz_compact_int8(vp(K), vp(V), B, n_c, d_, vp(idx), vp(cnt), vp(off), None, vp(kq),
+                                                 vp(Vq), vp(Ks), vp(Vs), None, None)
+    assert q8(d_=96) == UNSUPPORTED
+    assert q8(kq=Kq + 8) == ALIGN
