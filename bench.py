@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--workload", default=WORKLOAD,
                     help="llama8b_layer (default, the headline), tiny, llama8b_stack, qwen14b_128k, stress_ragged, "
-                         "llama8b_170k_chunked, llama8b_stack_heads")
+                         "llama8b_170k_chunked, llama8b_stack_heads, llama8b_stack_int8")
     ap.add_argument("--decode", action="store_true",
                     help="also time one decode step of attention (G queries per KV head) over the pruned cache "
                          "and over the full cache; adds a 'decode' object to the JSON line")
@@ -153,17 +153,23 @@ def workload_numbers(w):
             [(min(w.chunk, n_c - c0), w.n_prompt + min(w.chunk, n_c - c0)) for c0 in range(0, n_c, w.chunk)]
         vis = sum(B * G * (ni * nk + ni * (ni + 1) // 2) for nk, ni in blocks)   # pass 1 pairs
         ctx = sum(B * G * ni * nk for nk, ni in blocks)                          # pass 2 pairs
+        P, free = w.n_protect, n_c - w.n_protect
         if w.mode == "heads":
             kept = int(math.floor(w.ratio * B)) * n_c
+        elif w.mode == "global":
+            kept = B * P + int(math.floor(w.ratio * B * free))
         else:
-            kept = int(math.floor(w.ratio * B * n_c)) if w.mode == "global" else B * int(math.floor(w.ratio * n_c))
+            kept = B * (P + int(math.floor(w.ratio * free)))
         out["pairs_per_step"] += B * n_c
         out["flops_pass1"] += 2 * d * vis
         out["flops_pass2"] += 2 * d * ctx
         out["kept"] += kept
         out["select_bytes"] += (1 if w.mode == "heads" else 5) * 4 * B * n_c
     out["flops_algorithmic"] = out["flops_pass1"]
-    out["compact_bytes"] = out["kept"] * d * 2 * 2 * 2 + 4 * out["kept"]
+    if w.quant:   # bf16 K, V read; int8 K, V and two fp32 scales written; idx read
+        out["compact_bytes"] = out["kept"] * (d * 2 * 2 + d * 2 + 8) + 4 * out["kept"]
+    else:
+        out["compact_bytes"] = out["kept"] * d * 2 * 2 * 2 + 4 * out["kept"]
     return out
 
 
@@ -297,11 +303,17 @@ def main():
                 kvz.kvz_head_score(c.S, S_head=c.S_head, status=status, stream=stream)
                 kvz.kvz_select_heads(c.S_head, c.n_c, w.ratio, idx=c.idx, counts=c.counts, offsets=c.offsets,
                                      workspace=c.sel_ws, status=status, stream=stream)
+            elif w.n_protect:
+                kvz.kvz_select_protected(c.S, w.ratio, w.mode, w.n_protect, idx=c.idx, counts=c.counts,
+                                         offsets=c.offsets, workspace=c.sel_ws, status=status, stream=stream)
             else:
                 kvz.kvz_select(c.S, w.ratio, w.mode, idx=c.idx, counts=c.counts, offsets=c.offsets,
                                workspace=c.sel_ws, status=status, stream=stream)
             mark("cmp")
-            if w.in_place:
+            if w.quant:
+                kvz.kvz_compact_int8(c.K, c.V, c.idx, c.counts, c.offsets, Kq=c.Kq, Vq=c.Vq, K_scale=c.Ks,
+                                     V_scale=c.Vs, status=status, stream=stream)
+            elif w.in_place:
                 kvz.kvz_compact(c.K, c.V, c.idx, c.counts, c.offsets, in_place=True, workspace=c.cmp_ws,
                                 status=status, stream=stream)
             else:
@@ -348,7 +360,7 @@ def main():
     # ---- end to end through the host-buffer C-ABI call (pinned buffers): every
     # step copies the inputs in and the results out inside the timed region
     e2e = None
-    if len(ctxs) == 1 and w.L == 1 and not w.in_place and not w.chunk:
+    if len(ctxs) == 1 and w.L == 1 and not w.in_place and not w.chunk and not w.quant and not w.n_protect:
         c = ctxs[0]
         hx = {"Q": c.Q[0].cpu().pin_memory(), "K_ctx": c.K.cpu().pin_memory(), "K_in": c.Kin[0].cpu().pin_memory(),
               "V": c.V.cpu().pin_memory()}
@@ -388,7 +400,7 @@ def main():
 
     # ---- decode attention over the pruned cache vs the full cache (one step, all heads)
     dec = None
-    if args.decode:
+    if args.decode and not w.quant:
         c = ctxs[0]
         B = w.B
         gq = torch.Generator(device=dev).manual_seed(11)
@@ -540,15 +552,23 @@ class Context:
             self.S_head = torch.empty(B, dtype=torch.float32, device=dev)
             self.sel_ws = torch.empty(kvz.lib().kvz_select_heads_workspace_size(B), dtype=torch.uint8, device=dev)
         else:
-            k = kvz.kvz_keep_count(B * self.n_c if mode == kvz.GLOBAL else self.n_c, w.ratio)
-            cap = max(1, k if mode == kvz.GLOBAL else B * k)
+            free = self.n_c - w.n_protect
+            if mode == kvz.GLOBAL:
+                cap = max(1, B * w.n_protect + kvz.kvz_keep_count(B * free, w.ratio))
+            else:
+                cap = max(1, B * (w.n_protect + kvz.kvz_keep_count(free, w.ratio)))
             self.sel_ws = torch.empty(kvz.kvz_select_workspace_size(B, self.n_c, mode), dtype=torch.uint8,
                                       device=dev)
         self.idx = torch.empty(cap, dtype=torch.int32, device=dev)
         self.counts = torch.empty(B, dtype=torch.int32, device=dev)
         self.offsets = torch.empty(B + 1, dtype=torch.int64, device=dev)
         self.cmp_ws = torch.empty(kvz.kvz_compact_workspace_size(B, self.n_c), dtype=torch.uint8, device=dev)
-        if not w.in_place:
+        if w.quant:
+            self.Kq = torch.empty((cap, d), dtype=torch.int8, device=dev)
+            self.Vq = torch.empty((cap, d), dtype=torch.int8, device=dev)
+            self.Ks = torch.empty(cap, dtype=torch.float32, device=dev)
+            self.Vs = torch.empty(cap, dtype=torch.float32, device=dev)
+        elif not w.in_place:
             self.K_out = torch.empty((cap, d), dtype=torch.bfloat16, device=dev)
             self.V_out = torch.empty((cap, d), dtype=torch.bfloat16, device=dev)
         # lse (+ colmax, + S fill on the first chunk) per (layer, chunk); select 10 (1 per head

@@ -46,6 +46,8 @@ class Workload:
     sinks: int = 0
     dup_frac: float = 0.0
     chunk: int = 0                # context chunk length m of chunked scoring (0 = unchunked)
+    n_protect: int = 0            # leading positions of every head always kept (system prompt)
+    quant: bool = False           # compact into an int8 cache with per-row scales
     extra: dict = field(default_factory=dict)
 
     def n_in(self, ctx: int = 0) -> int:
@@ -70,6 +72,10 @@ WORKLOADS = {
     # the best half kept whole
     "llama8b_stack_heads": Workload("llama8b_stack_heads", L=32, H=8, G=4, d=128, n_c=(8192,),
                                     n_prompt=32, ratio=0.5, mode="heads", key_scale=True),
+    # a 64-token system prompt kept intact, the rest compacted into int8
+    "llama8b_stack_int8": Workload("llama8b_stack_int8", L=32, H=8, G=4, d=128, n_c=(32768,),
+                                   n_prompt=32, ratio=0.3, mode="global", key_scale=True,
+                                   n_protect=64, quant=True),
     # chunked scoring: 2K-token chunks of a 170K context (83 full chunks + 16)
     "llama8b_170k_chunked": Workload("llama8b_170k_chunked", L=1, H=8, G=4, d=128, n_c=(170000,),
                                      n_prompt=32, ratio=0.3, mode="per_head", key_scale=True, chunk=2048),
