@@ -417,13 +417,17 @@ def main():
         out_d = torch.empty((B, w.G, w.d), dtype=torch.float32, device=dev)
         lse_d = torch.empty((B, w.G), dtype=torch.float32, device=dev)
 
-        def time_decode(K_, V_, cnt, off, iters=20):
+        def time_decode(K_, V_, cnt, off, nbytes, iters=20):
+            # a cache over twice the L2 evicts itself between steps (the timing
+            # rules' "inputs larger than L2"); smaller ones get the write flush
+            big = nbytes > 2 * (126 << 20)
             for _ in range(3):
                 kvz.kvz_decode(q, K_, V_, cnt, off, c.n_c, scale=scale, out=out_d, lse2=lse_d, workspace=ws_d,
                                status=status, stream=stream)
             ts = []
             for _ in range(iters):
-                flush.zero_()
+                if not big:
+                    flush.zero_()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 kvz.kvz_decode(q, K_, V_, cnt, off, c.n_c, scale=scale, out=out_d, lse2=lse_d, workspace=ws_d,
@@ -433,19 +437,21 @@ def main():
                 ts.append(e0.elapsed_time(e1))
             return sorted(ts)[len(ts) // 2]
 
-        t_pruned = time_decode(Kd, Vd, c.counts, off_d)
-        t_full = time_decode(Kf, Vf, full_cnt, full_off)
+        kept_rows = nums["kept"]
+        byt = kept_rows * w.d * 2 * 2
+        byt_full = B * c.n_c * w.d * 4
+        t_pruned = time_decode(Kd, Vd, c.counts, off_d, byt)
+        t_full = time_decode(Kf, Vf, full_cnt, full_off, byt_full)
         if int(status.item()) != 0:
             raise RuntimeError("device status %d during decode" % int(status.item()))
-        kept_rows = nums["kept"]
         pk0 = peaks()
-        byt = kept_rows * w.d * 2 * 2
         dec = {"ms": t_pruned, "bytes": byt, "gbs": byt / (t_pruned * 1e-3) / 1e9,
                "frac_hbm": byt / (t_pruned * 1e-3) / 1e9 / pk0["hbm_gbs"],
                "full_cache_ms": t_full, "full_cache_gbs": B * c.n_c * w.d * 4 / (t_full * 1e-3) / 1e9,
                "speedup_vs_full_cache": t_full / t_pruned,
                "what": "one decode step: %d KV heads x %d grouped queries over the pruned cache (%d kept rows) vs "
-                       "the full cache; median of 20, L2 flushed before each" % (B, w.G, kept_rows)}
+                       "the full cache; median of 20; caches over 2x L2 unflushed (larger than L2), smaller ones "
+                       "after a 256 MB write flush" % (B, w.G, kept_rows)}
 
     red = max_over_ranks([ms_step, e2e["ms"] if e2e else 0.0] + part_ms, device=dev)
     ms_step, e2e_ms, part_ms = red[0], red[1], red[2:]

@@ -151,31 +151,33 @@ __global__ void __launch_bounds__(kGatherThreads)
 constexpr int kQuantThreads = 256;
 constexpr int kQuantUnroll = 4;
 
+// Codes of 8 bf16 values.  v = x * inv is one IEEE product; adding 1.5 * 2^23
+// then rounds v to the nearest integer (ties to even, |v| < 2^22) and leaves
+// that integer in the low bits of the sum's pattern, so the code is its low
+// byte.  |x| <= a gives |v| <= 127 (1 + 2^-24)^2 < 127.5: the code never
+// leaves [-127, 127].
 __device__ __forceinline__ void quant8(const int4& w, float inv, int8_t* dst) {
+  constexpr float kRound = 12582912.0f;                       // 1.5 * 2^23
   const uint32_t u[4] = {static_cast<uint32_t>(w.x), static_cast<uint32_t>(w.y), static_cast<uint32_t>(w.z),
                          static_cast<uint32_t>(w.w)};
-  uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const uint32_t h = (u[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu;
-    const float x = __uint_as_float(h << 16);
-    int q = __float2int_rn(__fmul_rn(x, inv));
-    q = q > 127 ? 127 : (q < -127 ? -127 : q);
-    packed[e >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << ((e & 3) * 8);
-  }
-  *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-}
-
-__device__ __forceinline__ float absmax8(const int4& w) {
-  const uint32_t u[4] = {static_cast<uint32_t>(w.x), static_cast<uint32_t>(w.y), static_cast<uint32_t>(w.z),
-                         static_cast<uint32_t>(w.w)};
-  float m = 0.0f;
+  uint32_t c[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    m = fmaxf(m, fabsf(__uint_as_float(u[i] << 16)));
-    m = fmaxf(m, fabsf(__uint_as_float(u[i] & 0xFFFF0000u)));
+    c[2 * i] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(u[i] << 16), inv), kRound));
+    c[2 * i + 1] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(u[i] & 0xFFFF0000u), inv), kRound));
   }
-  return m;
+  const uint32_t lo = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410);
+  *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+}
+
+// max |x| of 8 bf16 values: magnitude patterns (sign cleared) order like the
+// magnitudes, so two-lane 16-bit integer maxima find it.
+__device__ __forceinline__ float absmax8(const int4& w) {
+  const uint32_t m = __vmaxu2(__vmaxu2(static_cast<uint32_t>(w.x) & 0x7FFF7FFFu, static_cast<uint32_t>(w.y) & 0x7FFF7FFFu),
+                              __vmaxu2(static_cast<uint32_t>(w.z) & 0x7FFF7FFFu, static_cast<uint32_t>(w.w) & 0x7FFF7FFFu));
+  const uint32_t h = (m >> 16) > (m & 0xFFFFu) ? (m >> 16) : (m & 0xFFFFu);
+  return __uint_as_float(h << 16);
 }
 
 __global__ void __launch_bounds__(kQuantThreads)

@@ -7,7 +7,7 @@
 // kept row).  Split-KV: a CTA takes a contiguous run of 64-key tiles of one
 // head, brought in by TMA (three-stage ring, 128-byte swizzle, read back with
 // ldmatrix), keeps a running (max, sum, output) per query and writes it as a
-// partial; decode_combine_kernel merges the partials of each (head, query).
+// partial; the CTA that finishes a head's last split merges its partials.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -77,6 +77,40 @@ __device__ __forceinline__ uint32_t tile_chunk(uint32_t tile, int key, int dim) 
   return tile + (dim / 64) * DecLay<D>::BLK + key * 128 + ((((dim % 64) / 8) ^ (key & 7)) * 16);
 }
 
+// Merge the partials of head b: out = sum_s o_s 2^(m_s - M) / L with
+// L = sum_s l_s 2^(m_s - M), M = max_s m_s.  Run by the CTA that finishes the
+// head's last split; the splits' partials are read from L2.
+template <int D>
+__device__ void combine_head(const DecArgs& p, int b, int nsp, float* out, float* lse2, float* s_w) {
+  const int G = p.G;
+  const int64_t base = static_cast<int64_t>(b) * p.splits;
+  __shared__ float s_M[kDecGMax], s_L[kDecGMax];
+  if (threadIdx.x < G) {
+    const int g = threadIdx.x;
+    float M = -INFINITY;
+    for (int s = 0; s < nsp; ++s) M = fmaxf(M, __ldcg(&p.part_ml[(base + s) * G + g]).x);
+    float Ls = 0.0f;
+    for (int s = 0; s < nsp; ++s) {
+      const float2 ml = __ldcg(&p.part_ml[(base + s) * G + g]);
+      const float wgt = exp2f(ml.x - M);
+      s_w[s * kDecGMax + g] = wgt;
+      Ls += ml.y * wgt;
+    }
+    s_M[g] = M;
+    s_L[g] = Ls;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < G * D; e += kDecThreads) {
+    const int g = e / D;
+    float acc = 0.0f;
+#pragma unroll 8
+    for (int s = 0; s < nsp; ++s) acc = fmaf(__ldcg(&p.part_o[((base + s) * G) * D + e]), s_w[s * kDecGMax + g], acc);
+    out[static_cast<int64_t>(b) * G * D + e] = acc / s_L[g];
+  }
+  if (threadIdx.x < G && lse2 != nullptr)
+    lse2[static_cast<int64_t>(b) * G + threadIdx.x] = s_M[threadIdx.x] + log2f(s_L[threadIdx.x]);
+}
+
 // Split-KV decode on the tensor cores (mma.sync m16n8k16, bf16 -> fp32): the
 // G <= 8 queries of a KV head are the rows of the MMA (padded to 16), which
 // is below the 64-row minimum of tcgen05; the kernel is HBM-bound and the
@@ -87,7 +121,7 @@ __device__ __forceinline__ uint32_t tile_chunk(uint32_t tile, int key, int dim) 
 template <int D>
 __global__ void __launch_bounds__(kDecThreads)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                        DecArgs p) {
+                        DecArgs p, float* out, float* lse2) {
   using L = DecLay<D>;
   constexpr int KS = D / 16;                                  // k-steps of Q K^T
   constexpr int NT = D / 8;                                   // n-tiles of P V
@@ -113,7 +147,11 @@ __global__ void __launch_bounds__(kDecThreads)
   const int cps = (ntile + p.splits - 1) / p.splits;          // this head's tiles spread over all its splits
   const int t0 = sp * cps;
   const int n = min(ntile, t0 + cps) - t0;                    // tiles of this split
-  if (n <= 0) return;                                         // uniform: the combine skips it
+  if (ntile == 0 && sp == 0) {                                // no kept rows: output 0, lse -inf
+    for (int e = tid; e < G * D; e += kDecThreads) out[static_cast<int64_t>(b) * G * D + e] = 0.0f;
+    if (tid < G && lse2 != nullptr) lse2[static_cast<int64_t>(b) * G + tid] = -INFINITY;
+  }
+  if (n <= 0) return;                                         // uniform: no partial from this split
 
   if (tid == 0) {
     for (int s = 0; s < kDecStages; ++s) mbar_init(&full[s], 1);
@@ -257,47 +295,18 @@ __global__ void __launch_bounds__(kDecThreads)
     p.part_o[(part * G + g) * D + dd] = acc;
     if (dd == 0) p.part_ml[part * G + g] = make_float2(M, Ls);
   }
-}
-
-// Merge the partials of each (head, query): out = sum_s o_s 2^(m_s - M) / L,
-// L = sum_s l_s 2^(m_s - M), M = max_s m_s.  The splits' weights are staged
-// in shared memory once; each thread then sums its outputs over the splits
-// with independent loads.
-template <int D>
-__global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(DecArgs p, float* out, float* lse2) {
-  __shared__ float s_w[kDecMaxSplits * kDecGMax];          // 2^(m_s - M) / L per (split, query)
-  __shared__ float s_M[kDecGMax], s_L[kDecGMax];
-  const int b = blockIdx.x;
-  const int count = p.counts[b];
-  const int ntile = (count >= 0 && count <= p.n_c) ? (count + kDecKeys - 1) / kDecKeys : 0;
-  const int cps = (ntile + p.splits - 1) / p.splits;
-  const int nsp = cps > 0 ? (ntile + cps - 1) / cps : 0;     // splits that had tiles
-  const int G = p.G;
-  const int64_t base = static_cast<int64_t>(b) * p.splits;
-  if (threadIdx.x < G) {
-    const int g = threadIdx.x;
-    float M = -INFINITY;
-    for (int s = 0; s < nsp; ++s) M = fmaxf(M, p.part_ml[(base + s) * G + g].x);
-    float Ls = 0.0f;
-    for (int s = 0; s < nsp; ++s) {
-      const float2 ml = p.part_ml[(base + s) * G + g];
-      const float w = exp2f(ml.x - M);
-      s_w[s * kDecGMax + g] = w;
-      Ls += ml.y * w;
-    }
-    s_M[g] = M;
-    s_L[g] = Ls;
-  }
+  // ---- the CTA that finishes the head's last split merges all of them
+  __shared__ int s_last;
+  __threadfence();                                            // this partial before the count
   __syncthreads();
-  for (int e = threadIdx.x; e < G * D; e += kDecThreads) {
-    const int g = e / D;
-    float acc = 0.0f;
-#pragma unroll 4
-    for (int s = 0; s < nsp; ++s) acc = fmaf(p.part_o[((base + s) * G) * D + e], s_w[s * kDecGMax + g], acc);
-    out[static_cast<int64_t>(b) * G * D + e] = nsp > 0 ? acc / s_L[g] : 0.0f;
+  const int nsp = (ntile + cps - 1) / cps;                    // splits of this head that have tiles
+  if (tid == 0) s_last = atomicAdd(&p.done[b], 1u) == static_cast<unsigned>(nsp - 1);
+  __syncthreads();
+  if (s_last) {
+    __threadfence();                                          // the other splits' partials before reading them
+    __syncthreads();
+    combine_head<D>(p, b, nsp, out, lse2, reinterpret_cast<float*>(smem));   // weights over the idle stages
   }
-  if (threadIdx.x < G && lse2 != nullptr)
-    lse2[static_cast<int64_t>(b) * G + threadIdx.x] = nsp > 0 ? s_M[threadIdx.x] + log2f(s_L[threadIdx.x]) : -INFINITY;
 }
 
 }  // namespace
@@ -320,12 +329,13 @@ void decode_plan(int64_t B, int64_t n_c, int* cps, int* splits) {
 namespace {
 
 template <int D>
-cudaError_t launch_split(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecArgs& a, cudaStream_t stream) {
+cudaError_t launch_split(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecArgs& a, float* out, float* lse2,
+                         cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        DecLay<D>::SMEM);
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>(a.splits), static_cast<unsigned>(a.B));
-  decode_split_kernel<D><<<grid, kDecThreads, DecLay<D>::SMEM, stream>>>(tmK, tmV, a);
+  decode_split_kernel<D><<<grid, kDecThreads, DecLay<D>::SMEM, stream>>>(tmK, tmV, a, out, lse2);
   return cudaGetLastError();
 }
 
@@ -333,13 +343,11 @@ cudaError_t launch_split(const CUtensorMap& tmK, const CUtensorMap& tmV, const D
 
 cudaError_t launch_decode(int d, const CUtensorMap& tmK, const CUtensorMap& tmV, const DecArgs& a, float* out,
                           float* lse2, cudaStream_t stream) {
-  cudaError_t e = d == 128 ? launch_split<128>(tmK, tmV, a, stream) : launch_split<64>(tmK, tmV, a, stream);
+  // per-head counts of finished splits start at zero (all-zero bits)
+  cudaError_t e = launch_fill_f32(reinterpret_cast<float*>(a.done), a.B, 0.0f, stream);
   if (e != cudaSuccess) return e;
-  if (d == 128)
-    decode_combine_kernel<128><<<static_cast<unsigned>(a.B), kDecThreads, 0, stream>>>(a, out, lse2);
-  else
-    decode_combine_kernel<64><<<static_cast<unsigned>(a.B), kDecThreads, 0, stream>>>(a, out, lse2);
-  return cudaGetLastError();
+  return d == 128 ? launch_split<128>(tmK, tmV, a, out, lse2, stream)
+                  : launch_split<64>(tmK, tmV, a, out, lse2, stream);
 }
 
 }  // namespace kvz

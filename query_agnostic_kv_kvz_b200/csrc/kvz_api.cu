@@ -450,7 +450,8 @@ size_t kvz_decode_workspace_size(int64_t B, int G, int64_t n_c, int d) {
   int cps = 0, splits = 0;
   kvz::decode_plan(B, n_c, &cps, &splits);
   const size_t parts = static_cast<size_t>(B) * splits * G;
-  return ((parts * 8 + 255) & ~size_t(255)) + ((parts * d * 4 + 255) & ~size_t(255));
+  return ((parts * 8 + 255) & ~size_t(255)) + ((parts * d * 4 + 255) & ~size_t(255)) +
+         ((static_cast<size_t>(B) * 4 + 255) & ~size_t(255));
 }
 
 kvz_status kvz_decode(const void* q, const void* K_out, const void* V_out, int64_t n_rows, const int32_t* counts,
@@ -484,6 +485,7 @@ kvz_status kvz_decode(const void* q, const void* K_out, const void* V_out, int64
   const size_t parts = static_cast<size_t>(B) * a.splits * G;
   a.part_ml = static_cast<float2*>(workspace);
   a.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((parts * 8 + 255) & ~size_t(255)));
+  a.done = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(a.part_o) + ((parts * d * 4 + 255) & ~size_t(255)));
   a.status = d_status;
   return kvz::launch_decode(d, tmK, tmV, a, out, lse2, stream) == cudaSuccess ? KVZ_OK : KVZ_ERR_CUDA;
 }

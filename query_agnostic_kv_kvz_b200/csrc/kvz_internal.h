@@ -58,6 +58,7 @@ struct DecArgs {
   int splits;                               // splits per head (grid.x)
   float2* part_ml;                          // [B][splits][G] (running max, sum), base 2
   float* part_o;                            // [B][splits][G][d]
+  unsigned* done;                           // [B] splits finished per head (zeroed by the launcher)
   int32_t* status;
 };
 void decode_plan(int64_t B, int64_t n_c, int* cps, int* splits);
