@@ -332,11 +332,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <typename K>
-cudaError_t set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-}
-
 }  // namespace
 
 cudaError_t launch_colmax(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, const ColArgs& args,
@@ -359,11 +354,11 @@ cudaError_t launch_colmax(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc
   a.tiles_per_split = static_cast<int>(tps);
   cudaError_t e;
   if (d == 128) {
-    e = set_smem(colmax_kernel<128>, Lay<128>::SMEM);
+    e = smem_limit_once<colmax_kernel<128>>(Lay<128>::SMEM);
     if (e != cudaSuccess) return e;
     colmax_kernel<128><<<static_cast<unsigned>(grid), kThreads, Lay<128>::SMEM, stream>>>(tmQ, tmKc, a);
   } else {
-    e = set_smem(colmax_kernel<64>, Lay<64>::SMEM);
+    e = smem_limit_once<colmax_kernel<64>>(Lay<64>::SMEM);
     if (e != cudaSuccess) return e;
     colmax_kernel<64><<<static_cast<unsigned>(grid), kThreads, Lay<64>::SMEM, stream>>>(tmQ, tmKc, a);
   }

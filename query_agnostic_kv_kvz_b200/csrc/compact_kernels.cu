@@ -180,70 +180,87 @@ __device__ __forceinline__ float absmax8(const int4& w) {
   return __uint_as_float(h << 16);
 }
 
+// Work unit = (head b, block of rows_per_blk slots of that head): the head is
+// known without a search, and units past a head's count leave at once.
 __global__ void __launch_bounds__(kQuantThreads)
     compact_int8_kernel(const int4* __restrict__ K, const int4* __restrict__ V, int64_t B, int64_t n_c, int vpr,
-                        const int32_t* __restrict__ idx, const int64_t* __restrict__ offsets,
-                        const int64_t* __restrict__ out_offsets, int8_t* __restrict__ Kq, int8_t* __restrict__ Vq,
-                        float* __restrict__ Ks, float* __restrict__ Vs, int32_t* status) {
-  __shared__ int64_t s_head;
-  const int64_t total = offsets[B];
+                        const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
+                        const int64_t* __restrict__ offsets, const int64_t* __restrict__ out_offsets,
+                        int8_t* __restrict__ Kq, int8_t* __restrict__ Vq, float* __restrict__ Ks,
+                        float* __restrict__ Vs, int32_t* status) {
   const int rows_per_step = kQuantThreads / vpr;
   const int rows_per_blk = rows_per_step * kQuantUnroll;
+  const int64_t blocks_per_head = (n_c + rows_per_blk - 1) / rows_per_blk;
   const int my_row = threadIdx.x / vpr;
   const int vec = threadIdx.x % vpr;
-  for (int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_blk; r0 < total;
-       r0 += static_cast<int64_t>(gridDim.x) * rows_per_blk) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int64_t lo = 0, hi = B - 1;                                 // largest b with offsets[b] <= r0
-      while (lo < hi) {
-        const int64_t mid = (lo + hi + 1) >> 1;
-        if (offsets[mid] <= r0) lo = mid; else hi = mid - 1;
-      }
-      s_head = lo;
+  for (int64_t unit = blockIdx.x; unit < B * blocks_per_head; unit += gridDim.x) {
+    const int64_t hb = unit / blocks_per_head;
+    const int64_t p0 = (unit % blocks_per_head) * rows_per_blk;        // first slot within the head
+    const int64_t cnt = counts[hb];
+    if (cnt < 0 || cnt > n_c) {                                        // not a selection's count
+      if (p0 == 0 && threadIdx.x == 0) report_err(status, KVZ_ERR_INVALID_ARG);
+      continue;
     }
-    __syncthreads();
-    int64_t hb = s_head;
+    if (p0 >= cnt) continue;                                           // uniform for the CTA
+    const int64_t in0 = offsets[hb];
+    const int64_t out0 = out_offsets != nullptr ? out_offsets[hb] : in0;
     int4 kv[kQuantUnroll], vv[kQuantUnroll];
     int64_t dst[kQuantUnroll];
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
-      const int64_t slot = r0 + u * rows_per_step + my_row;
+      const int64_t pp = p0 + u * rows_per_step + my_row;
       dst[u] = -1;
       kv[u] = vv[u] = make_int4(0, 0, 0, 0);
-      if (slot < total) {
-        while (hb + 1 < B && offsets[hb + 1] <= slot) ++hb;
-        const int64_t j = idx[slot];
+      if (pp < cnt) {
+        const int64_t j = idx[in0 + pp];
         if (j < 0 || j >= n_c) {
           report_err(status, KVZ_ERR_INVALID_ARG);
         } else {
           const int64_t src = (hb * n_c + j) * vpr + vec;
-          const int64_t base = out_offsets != nullptr ? out_offsets[hb] : offsets[hb];
-          dst[u] = base + (slot - offsets[hb]);
+          dst[u] = out0 + pp;
           kv[u] = ld_stream(K + src);
           vv[u] = ld_stream(V + src);
         }
       }
     }
+    // absmax of each row (K and V): its vpr threads are consecutive lanes
+    float ak[kQuantUnroll], av[kQuantUnroll];
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
-      // the vpr threads of a row are consecutive lanes of one warp
-      float ak = absmax8(kv[u]), av = absmax8(vv[u]);
+      ak[u] = absmax8(kv[u]);
+      av[u] = absmax8(vv[u]);
 #pragma unroll
       for (int o2 = 1; o2 < 16; o2 <<= 1) {
         if (o2 < vpr) {
-          ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, o2));
-          av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, o2));
+          ak[u] = fmaxf(ak[u], __shfl_xor_sync(0xffffffffu, ak[u], o2));
+          av[u] = fmaxf(av[u], __shfl_xor_sync(0xffffffffu, av[u], o2));
         }
       }
+    }
+    // the 2 * kQuantUnroll divisions of a row run in parallel, one per lane of
+    // its group (lane 2u takes K of row u, lane 2u+1 V), and come back by shuffle
+    static_assert(2 * kQuantUnroll <= 8, "a row group (8 or 16 lanes) holds every division");
+    float a = 0.0f;
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      if (vec == 2 * u) a = ak[u];
+      if (vec == 2 * u + 1) a = av[u];
+    }
+    const float inv = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+    const float scl = __fdiv_rn(a, 127.0f);
+    const int group = (threadIdx.x & 31) & ~(vpr - 1);        // first lane of this row's group
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+      const float ik = __shfl_sync(0xffffffffu, inv, group + 2 * u);
+      const float iv = __shfl_sync(0xffffffffu, inv, group + 2 * u + 1);
+      const float sk = __shfl_sync(0xffffffffu, scl, group + 2 * u);
+      const float sv = __shfl_sync(0xffffffffu, scl, group + 2 * u + 1);
       if (dst[u] >= 0) {
-        const float ik = ak > 0.0f ? __fdiv_rn(127.0f, ak) : 0.0f;
-        const float iv = av > 0.0f ? __fdiv_rn(127.0f, av) : 0.0f;
         quant8(kv[u], ik, Kq + dst[u] * vpr * 8 + vec * 8);
         quant8(vv[u], iv, Vq + dst[u] * vpr * 8 + vec * 8);
         if (vec == 0) {
-          Ks[dst[u]] = __fdiv_rn(ak, 127.0f);
-          Vs[dst[u]] = __fdiv_rn(av, 127.0f);
+          Ks[dst[u]] = sk;
+          Vs[dst[u]] = sv;
         }
       }
     }
@@ -468,16 +485,17 @@ cudaError_t launch_compact_gather(const void* K, const void* V, int64_t B, int64
 }
 
 cudaError_t launch_compact_int8(const void* K, const void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
-                                const int64_t* offsets, const int64_t* out_offsets, int8_t* Kq, int8_t* Vq,
-                                float* K_scale, float* V_scale, int32_t* status, cudaStream_t stream) {
+                                const int32_t* counts, const int64_t* offsets, const int64_t* out_offsets,
+                                int8_t* Kq, int8_t* Vq, float* K_scale, float* V_scale, int32_t* status,
+                                cudaStream_t stream) {
   const int vpr = d / 8;
   const int rows_per_blk = (kQuantThreads / vpr) * kQuantUnroll;
-  int64_t blocks = (B * n_c + rows_per_blk - 1) / rows_per_blk;
+  int64_t blocks = B * ((n_c + rows_per_blk - 1) / rows_per_blk);
   if (blocks > 148 * 8) blocks = 148 * 8;
   if (blocks < 1) blocks = 1;
   compact_int8_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-      static_cast<const int4*>(K), static_cast<const int4*>(V), B, n_c, vpr, idx, offsets, out_offsets, Kq, Vq,
-      K_scale, V_scale, status);
+      static_cast<const int4*>(K), static_cast<const int4*>(V), B, n_c, vpr, idx, counts, offsets, out_offsets, Kq,
+      Vq, K_scale, V_scale, status);
   return cudaGetLastError();
 }
 

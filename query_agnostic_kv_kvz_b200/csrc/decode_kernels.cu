@@ -331,8 +331,7 @@ namespace {
 template <int D>
 cudaError_t launch_split(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecArgs& a, float* out, float* lse2,
                          cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       DecLay<D>::SMEM);
+  cudaError_t e = smem_limit_once<decode_split_kernel<D>>(DecLay<D>::SMEM);
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>(a.splits), static_cast<unsigned>(a.B));
   decode_split_kernel<D><<<grid, kDecThreads, DecLay<D>::SMEM, stream>>>(tmK, tmV, a, out, lse2);

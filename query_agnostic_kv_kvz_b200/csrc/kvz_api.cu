@@ -502,8 +502,8 @@ kvz_status kvz_compact_int8(const void* K, const void* V, int64_t B, int64_t n_c
       !aligned(V_scale, 4) || !aligned(idx, 4) || !aligned(counts, 4) || !aligned(offsets, 8) ||
       (out_offsets && !aligned(out_offsets, 8)))
     return KVZ_ERR_ALIGNMENT;
-  return kvz::launch_compact_int8(K, V, B, n_c, d, idx, offsets, out_offsets, Kq, Vq, K_scale, V_scale, d_status,
-                                  stream) == cudaSuccess
+  return kvz::launch_compact_int8(K, V, B, n_c, d, idx, counts, offsets, out_offsets, Kq, Vq, K_scale, V_scale,
+                                  d_status, stream) == cudaSuccess
              ? KVZ_OK
              : KVZ_ERR_CUDA;
 }

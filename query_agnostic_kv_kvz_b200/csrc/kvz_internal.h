@@ -4,9 +4,26 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 namespace kvz {
+
+// Raise a kernel's dynamic shared-memory limit once per device (the launch
+// paths call this before every launch; the attribute call itself is a host
+// round trip worth skipping).  `bytes` is a constant of the kernel.
+template <auto Kernel>
+cudaError_t smem_limit_once(int bytes) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit != 0) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Pass 1 (row log-sum-exp) arguments.  Rows i in [i_begin, i_end) are
 // computed; rows_pad = roundup(i_end - i_begin, 256) entries per (b, g) are
@@ -93,7 +110,8 @@ cudaError_t launch_compact_inplace(void* K, void* V, int64_t B, int64_t n_c, int
 size_t compact_workspace_bytes(int64_t B, int64_t n_c);
 // Out-of-place compaction into int8 codes with one fp32 scale per row.
 cudaError_t launch_compact_int8(const void* K, const void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
-                                const int64_t* offsets, const int64_t* out_offsets, int8_t* Kq, int8_t* Vq,
-                                float* K_scale, float* V_scale, int32_t* status, cudaStream_t stream);
+                                const int32_t* counts, const int64_t* offsets, const int64_t* out_offsets,
+                                int8_t* Kq, int8_t* Vq, float* K_scale, float* V_scale, int32_t* status,
+                                cudaStream_t stream);
 
 }  // namespace kvz

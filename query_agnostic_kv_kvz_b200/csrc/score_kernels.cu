@@ -325,11 +325,6 @@ __global__ void fill_f32_kernel(float* x, int64_t n, float v) {
     x[e] = v;
 }
 
-template <typename K>
-cudaError_t set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-}
-
 }  // namespace
 
 cudaError_t launch_lse(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, const CUtensorMap& tmKi,
@@ -339,11 +334,11 @@ cudaError_t launch_lse(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, c
   if (grid <= 0 || grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
   cudaError_t e;
   if (d == 128) {
-    e = set_smem(lse_kernel<128>, LseLayout<128>::SMEM);
+    e = smem_limit_once<lse_kernel<128>>(LseLayout<128>::SMEM);
     if (e != cudaSuccess) return e;
     lse_kernel<128><<<static_cast<unsigned>(grid), kThreads, LseLayout<128>::SMEM, stream>>>(tmQ, tmKc, tmKi, a);
   } else {
-    e = set_smem(lse_kernel<64>, LseLayout<64>::SMEM);
+    e = smem_limit_once<lse_kernel<64>>(LseLayout<64>::SMEM);
     if (e != cudaSuccess) return e;
     lse_kernel<64><<<static_cast<unsigned>(grid), kThreads, LseLayout<64>::SMEM, stream>>>(tmQ, tmKc, tmKi, a);
   }

@@ -469,8 +469,7 @@ cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int64_t n_prot
   if (mode == KVZ_PER_HEAD && (n_c <= kHeadStageMax || B >= 128)) {
     if (n_c <= kHeadStageMax) {
       const int smem = static_cast<int>(n_c * 4);
-      cudaError_t e = cudaFuncSetAttribute(sel_head_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(kHeadStageMax * 4));
+      cudaError_t e = smem_limit_once<sel_head_kernel<true>>(static_cast<int>(kHeadStageMax * 4));
       if (e != cudaSuccess) return e;
       sel_head_kernel<true><<<static_cast<unsigned>(B), kHeadThreads, smem, stream>>>(S, B, n_c, n_protect, k, idx,
                                                                                     counts, offsets, status);
