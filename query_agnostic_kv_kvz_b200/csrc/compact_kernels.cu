@@ -149,7 +149,6 @@ __global__ void __launch_bounds__(kGatherThreads)
 // read by vpr threads (16 bytes each); its absmax comes from a shuffle
 // reduction over them.  HBM-bound: 4d bytes read, 2d + 8 written per row.
 constexpr int kQuantThreads = 256;
-constexpr int kQuantUnroll = 4;
 
 // Codes of 8 bf16 values.  v = x * inv is one IEEE product; adding 1.5 * 2^23
 // then rounds v to the nearest integer (ties to even, |v| < 2^22) and leaves
@@ -180,91 +179,161 @@ __device__ __forceinline__ float absmax8(const int4& w) {
   return __uint_as_float(h << 16);
 }
 
-// Work unit = (head b, block of rows_per_blk slots of that head): the head is
-// known without a search, and units past a head's count leave at once.
+// Work unit = (head b, block of 64 slots of that head): the head is known
+// without a search, and units past a head's count are skipped.  A CTA walks
+// its units with a two-stage shared-memory ring: the rows of its next unit
+// are in flight (cp.async) while the current one is quantised, and the
+// source indices of the unit after that are fetched a step earlier still, so
+// the bytes in flight do not depend on registers or on the compute phase.
+constexpr int kQuantRows = 64;                                  // slots per unit
+constexpr int kQuantStageBytes = 2 * kQuantRows * 256;          // K and V rows of a unit at d = 128
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 __global__ void __launch_bounds__(kQuantThreads)
     compact_int8_kernel(const int4* __restrict__ K, const int4* __restrict__ V, int64_t B, int64_t n_c, int vpr,
                         const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
                         const int64_t* __restrict__ offsets, const int64_t* __restrict__ out_offsets,
                         int8_t* __restrict__ Kq, int8_t* __restrict__ Vq, float* __restrict__ Ks,
                         float* __restrict__ Vs, int32_t* status) {
+  extern __shared__ int4 qstage[];                              // [2][K rows | V rows] of a unit
+  constexpr int kPer = kQuantRows / (kQuantThreads / 16);       // rows per thread (4 at d=128, 2 at d=64)
   const int rows_per_step = kQuantThreads / vpr;
-  const int rows_per_blk = rows_per_step * kQuantUnroll;
-  const int64_t blocks_per_head = (n_c + rows_per_blk - 1) / rows_per_blk;
+  const int per = kQuantRows / rows_per_step;                   // rows of a unit per thread
+  const int64_t bph = (n_c + kQuantRows - 1) / kQuantRows;      // units per head
+  const int64_t nunits = B * bph;
   const int my_row = threadIdx.x / vpr;
   const int vec = threadIdx.x % vpr;
-  for (int64_t unit = blockIdx.x; unit < B * blocks_per_head; unit += gridDim.x) {
-    const int64_t hb = unit / blocks_per_head;
-    const int64_t p0 = (unit % blocks_per_head) * rows_per_blk;        // first slot within the head
-    const int64_t cnt = counts[hb];
-    if (cnt < 0 || cnt > n_c) {                                        // not a selection's count
-      if (p0 == 0 && threadIdx.x == 0) report_err(status, KVZ_ERR_INVALID_ARG);
-      continue;
+  const int tensor_vec = kQuantRows * vpr;
+
+  // next unit of this CTA at or after u that has slots (nunits when none)
+  auto next_active = [&](int64_t u) -> int64_t {
+    for (; u < nunits; u += gridDim.x) {
+      const int64_t cnt = counts[u / bph];
+      if (cnt < 0 || cnt > n_c) {
+        if ((u % bph) == 0 && threadIdx.x == 0) report_err(status, KVZ_ERR_INVALID_ARG);
+        continue;
+      }
+      if ((u % bph) * kQuantRows < cnt) return u;
     }
-    if (p0 >= cnt) continue;                                           // uniform for the CTA
-    const int64_t in0 = offsets[hb];
-    const int64_t out0 = out_offsets != nullptr ? out_offsets[hb] : in0;
-    int4 kv[kQuantUnroll], vv[kQuantUnroll];
-    int64_t dst[kQuantUnroll];
+    return nunits;
+  };
+  // source row of each of this thread's slots in unit u (-1: no slot there)
+  auto fetch_src = [&](int64_t u, int32_t (&src)[kPer]) {
 #pragma unroll
-    for (int u = 0; u < kQuantUnroll; ++u) {
-      const int64_t pp = p0 + u * rows_per_step + my_row;
-      dst[u] = -1;
-      kv[u] = vv[u] = make_int4(0, 0, 0, 0);
-      if (pp < cnt) {
-        const int64_t j = idx[in0 + pp];
-        if (j < 0 || j >= n_c) {
-          report_err(status, KVZ_ERR_INVALID_ARG);
-        } else {
-          const int64_t src = (hb * n_c + j) * vpr + vec;
-          dst[u] = out0 + pp;
-          kv[u] = ld_stream(K + src);
-          vv[u] = ld_stream(V + src);
+    for (int k = 0; k < kPer; ++k) src[k] = -1;
+    if (u >= nunits) return;
+    const int64_t hb = u / bph, p0 = (u % bph) * kQuantRows, cnt = counts[hb], in0 = offsets[hb];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int64_t pp = p0 + my_row + k * rows_per_step;
+      if (k < per && pp < cnt) src[k] = idx[in0 + pp];
+    }
+  };
+  auto issue = [&](int64_t u, int st, const int32_t (&src)[kPer]) {
+    if (u < nunits) {
+      const int64_t hb = u / bph;
+      int4* sk = qstage + st * 2 * tensor_vec;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int64_t j = src[k];
+        if (k < per && j >= 0 && j < n_c) {
+          const int r = my_row + k * rows_per_step;
+          cp_async16(sk + r * vpr + vec, K + (hb * n_c + j) * vpr + vec);
+          cp_async16(sk + tensor_vec + r * vpr + vec, V + (hb * n_c + j) * vpr + vec);
         }
       }
     }
-    // absmax of each row (K and V): its vpr threads are consecutive lanes
-    float ak[kQuantUnroll], av[kQuantUnroll];
+    cp_async_commit();
+  };
+
+  int32_t src_cur[kPer], src_nxt[kPer];
+  int64_t u = next_active(blockIdx.x);
+  fetch_src(u, src_cur);
+  issue(u, 0, src_cur);
+  int64_t un = next_active(u + gridDim.x);
+  fetch_src(un, src_nxt);
+  int st = 0;
+  while (u < nunits) {
+    issue(un, st ^ 1, src_nxt);                                   // the next unit's rows go in flight
+    const int64_t unn = next_active(un + gridDim.x);
+    int32_t src_nn[kPer];
+    fetch_src(unn, src_nn);                                       // and the indices of the one after
+    cp_async_wait1();                                             // this thread's rows of unit u
+    __syncthreads();                                              // everyone's
+    const int64_t hb = u / bph, p0 = (u % bph) * kQuantRows;
+    const int64_t cnt = counts[hb];
+    const int64_t out0 = (out_offsets != nullptr ? out_offsets[hb] : offsets[hb]) + p0;
+    const int4* sk = qstage + st * 2 * tensor_vec;
+    // absmax of each row (K and V) over its vpr lanes
+    float ak[kPer], av[kPer];
+    int4 kv[kPer], vv[kPer];
 #pragma unroll
-    for (int u = 0; u < kQuantUnroll; ++u) {
-      ak[u] = absmax8(kv[u]);
-      av[u] = absmax8(vv[u]);
+    for (int k = 0; k < kPer; ++k) {
+      const int r = my_row + k * rows_per_step;
+      kv[k] = vv[k] = make_int4(0, 0, 0, 0);
+      if (k < per) {
+        kv[k] = sk[r * vpr + vec];
+        vv[k] = sk[tensor_vec + r * vpr + vec];
+      }
+      ak[k] = absmax8(kv[k]);
+      av[k] = absmax8(vv[k]);
 #pragma unroll
       for (int o2 = 1; o2 < 16; o2 <<= 1) {
         if (o2 < vpr) {
-          ak[u] = fmaxf(ak[u], __shfl_xor_sync(0xffffffffu, ak[u], o2));
-          av[u] = fmaxf(av[u], __shfl_xor_sync(0xffffffffu, av[u], o2));
+          ak[k] = fmaxf(ak[k], __shfl_xor_sync(0xffffffffu, ak[k], o2));
+          av[k] = fmaxf(av[k], __shfl_xor_sync(0xffffffffu, av[k], o2));
         }
       }
     }
-    // the 2 * kQuantUnroll divisions of a row run in parallel, one per lane of
-    // its group (lane 2u takes K of row u, lane 2u+1 V), and come back by shuffle
-    static_assert(2 * kQuantUnroll <= 8, "a row group (8 or 16 lanes) holds every division");
+    // the row divisions run in parallel, one per lane of the row's group
     float a = 0.0f;
 #pragma unroll
-    for (int u = 0; u < kQuantUnroll; ++u) {
-      if (vec == 2 * u) a = ak[u];
-      if (vec == 2 * u + 1) a = av[u];
+    for (int k = 0; k < kPer; ++k) {
+      if (vec == 2 * k) a = ak[k];
+      if (vec == 2 * k + 1) a = av[k];
     }
     const float inv = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
     const float scl = __fdiv_rn(a, 127.0f);
-    const int group = (threadIdx.x & 31) & ~(vpr - 1);        // first lane of this row's group
+    const int group = (threadIdx.x & 31) & ~(vpr - 1);
 #pragma unroll
-    for (int u = 0; u < kQuantUnroll; ++u) {
-      const float ik = __shfl_sync(0xffffffffu, inv, group + 2 * u);
-      const float iv = __shfl_sync(0xffffffffu, inv, group + 2 * u + 1);
-      const float sk = __shfl_sync(0xffffffffu, scl, group + 2 * u);
-      const float sv = __shfl_sync(0xffffffffu, scl, group + 2 * u + 1);
-      if (dst[u] >= 0) {
-        quant8(kv[u], ik, Kq + dst[u] * vpr * 8 + vec * 8);
-        quant8(vv[u], iv, Vq + dst[u] * vpr * 8 + vec * 8);
+    for (int k = 0; k < kPer; ++k) {
+      const float ik = __shfl_sync(0xffffffffu, inv, group + 2 * k);
+      const float iv = __shfl_sync(0xffffffffu, inv, group + 2 * k + 1);
+      const float sk2 = __shfl_sync(0xffffffffu, scl, group + 2 * k);
+      const float sv2 = __shfl_sync(0xffffffffu, scl, group + 2 * k + 1);
+      const int r = my_row + k * rows_per_step;
+      if (k < per && p0 + r < cnt && src_cur[k] >= 0 && src_cur[k] < n_c) {
+        const int64_t dst = out0 + r;
+        quant8(kv[k], ik, Kq + dst * vpr * 8 + vec * 8);
+        quant8(vv[k], iv, Vq + dst * vpr * 8 + vec * 8);
         if (vec == 0) {
-          Ks[dst[u]] = sk;
-          Vs[dst[u]] = sv;
+          Ks[dst] = sk2;
+          Vs[dst] = sv2;
         }
+      } else if (k < per && p0 + r < cnt && vec == 0) {
+        report_err(status, KVZ_ERR_INVALID_ARG);                  // idx out of [0, n_c)
       }
     }
+    __syncthreads();                                              // stage st is free again
+    u = un;
+    un = unn;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      src_cur[k] = src_nxt[k];
+      src_nxt[k] = src_nn[k];
+    }
+    st ^= 1;
   }
+  cp_async_wait0();
 }
 
 // Dependencies of in-place compaction.  Slot chunk c (slots [cC, (c+1)C))
@@ -489,11 +558,13 @@ cudaError_t launch_compact_int8(const void* K, const void* V, int64_t B, int64_t
                                 int8_t* Kq, int8_t* Vq, float* K_scale, float* V_scale, int32_t* status,
                                 cudaStream_t stream) {
   const int vpr = d / 8;
-  const int rows_per_blk = (kQuantThreads / vpr) * kQuantUnroll;
-  int64_t blocks = B * ((n_c + rows_per_blk - 1) / rows_per_blk);
-  if (blocks > 148 * 8) blocks = 148 * 8;
+  const int smem = 2 * 2 * kQuantRows * vpr * 16;               // two stages of a unit's K and V rows
+  cudaError_t e = smem_limit_once<compact_int8_kernel>(kQuantStageBytes * 2);
+  if (e != cudaSuccess) return e;
+  int64_t blocks = B * ((n_c + kQuantRows - 1) / kQuantRows);
+  if (blocks > 148 * 3) blocks = 148 * 3;                       // three CTAs per SM (64 KB each at d = 128)
   if (blocks < 1) blocks = 1;
-  compact_int8_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
+  compact_int8_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, smem, stream>>>(
       static_cast<const int4*>(K), static_cast<const int4*>(V), B, n_c, vpr, idx, counts, offsets, out_offsets, Kq,
       Vq, K_scale, V_scale, status);
   return cudaGetLastError();
