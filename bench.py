@@ -196,7 +196,7 @@ def oracle_head_time(x, w, head):
         threads = len(os.sched_getaffinity(0))
     except Exception:
         threads = os.cpu_count() or 1
-    return dt, threads
+    return dt, threads, idx
 
 
 # ---------------------------------------------------------------------------
@@ -242,7 +242,7 @@ def main():
         times = []
         threads = 1
         for s in range(steps):
-            dt, threads = oracle_head_time(x, w, s % w.B)
+            dt, threads, _ = oracle_head_time(x, w, s % w.B)
             times.append(dt)
         per_head = sum(times) / len(times)
         value = w.n_c[0] / per_head
@@ -514,10 +514,18 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline and w.name == WORKLOAD:
         c = ctxs[0]
         x0 = {"Q": c.Q[0], "K_ctx": c.K[: w.H], "K_in": c.Kin[0], "V": c.V[: w.H]}
-        dt, threads = oracle_head_time(x0, w, 0)
+        dt, threads, oracle_idx = oracle_head_time(x0, w, 0)
         line["cpu_baseline"] = {"value": c.n_c / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": "head 0 of the %d-head layer: fp64 score + select + compact "
                                           "(%.1f s)" % (w.B, dt)}
+        # index-set overlap of the GPU's kept keys with the oracle's selection
+        # from its own fp64 scores (reported, not gated: a top-k over scores
+        # that agree within the tolerance may still differ at the threshold)
+        o0, o1 = int(c.offsets[0].item()), int(c.offsets[1].item())
+        gpu_set = set(c.idx[o0:o1].cpu().tolist())
+        ora_set = set(int(v) for v in oracle_idx)
+        line["selection_overlap"] = {"head": 0, "jaccard": len(gpu_set & ora_set) / max(1, len(gpu_set | ora_set)),
+                                     "kept": len(ora_set)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
