@@ -309,12 +309,14 @@ kvz_status kvz_compact(const void* K, const void* V, int64_t B, int64_t n_c,
 /* log of the softmax denominator.  A head with counts[b] == 0 gives out = 0 */
 /* and lse2 = -inf.                                                          */
 /* Layout: q [B][G][d] bf16; K_out, V_out [n_rows][d] bf16; out [B][G][d]    */
-/* fp32; lse2 [B][G] fp32.  n_c bounds every counts[b] (it sizes the split   */
-/* of each head's rows over CTAs); a count outside [0, n_c] is reported      */
-/* (KVZ_ERR_INVALID_ARG in d_status) and that head is skipped.              */
+/* fp32; lse2 [B][G] fp32.  n_c bounds every counts[b]; a count outside     */
+/* [0, n_c] is reported (KVZ_ERR_INVALID_ARG in d_status) and that head is   */
+/* skipped.  The rows are split over CTAs on the device from the counts, at  */
+/* the same number of rows per CTA for every head, so uneven heads (global   */
+/* selection) cost no more than even ones.                                  */
 /* Limits: d in {64, 128}; 1 <= G <= 8 (else KVZ_ERR_UNSUPPORTED);          */
 /* B <= 65535.  Workspace: kvz_decode_workspace_size(B, G, n_c, d) bytes,    */
-/* 256-byte aligned (per-split partial results).                             */
+/* 256-byte aligned (the work list and per-split partial results).           */
 /* ------------------------------------------------------------------------ */
 size_t kvz_decode_workspace_size(int64_t B, int G, int64_t n_c, int d);
 

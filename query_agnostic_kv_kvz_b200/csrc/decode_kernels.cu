@@ -24,7 +24,7 @@ namespace {
 constexpr int kDecThreads = 128;            // 4 warps; warp w owns keys [16w, 16w+16) of every tile
 constexpr int kDecKeys = 64;                 // keys per tile (TMA box rows)
 constexpr int kDecStages = 3;
-constexpr int kDecMaxSplits = 256;           // splits per head (shared-memory weights in the combine)
+constexpr int kDecMaxSplits = 256;           // splits per head (two merge levels of 16)
 constexpr int kDecWarps = kDecThreads / 32;
 
 template <int D>
@@ -77,38 +77,92 @@ __device__ __forceinline__ uint32_t tile_chunk(uint32_t tile, int key, int dim) 
   return tile + (dim / 64) * DecLay<D>::BLK + key * 128 + ((((dim % 64) / 8) ^ (key & 7)) * 16);
 }
 
-// Merge the partials of head b: out = sum_s o_s 2^(m_s - M) / L with
-// L = sum_s l_s 2^(m_s - M), M = max_s m_s.  Run by the CTA that finishes the
-// head's last split; the splits' partials are read from L2.
+// Splits are merged by a two-level tree: the last CTA to finish in each group
+// of kDecGroup consecutive splits of a head merges that group, and the last
+// group merger merges the groups.  A merge loads all its partials at once, so
+// it costs about one L2 round trip per level, whatever the head's split count.
+constexpr int kDecGroup = 16;
+static_assert(kDecGroup * kDecGroup >= kDecMaxSplits, "two levels cover every head");
+static_assert(kDecGMax * kDecGroup == kDecThreads, "one thread per (query, partial) in a merge");
+
+// True in every thread of the CTA that arrives last of `total` at `counter`.
+// Each arriving CTA's writes are ordered before its count; the last one
+// orders the count before its reads of the others' writes.
+__device__ __forceinline__ bool last_arrival(unsigned* counter, int total) {
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(counter, 1u) == static_cast<unsigned>(total - 1);
+  __syncthreads();
+  const bool last = s_last != 0;
+  if (last) __threadfence();
+  return last;
+}
+
+// Merge cnt <= kDecGroup partials (slots first, first + stride, ...), each a
+// (max m_s, sum l_s, output o_s) with o_s relative to m_s, base 2:
+// M = max_s m_s, L = sum_s l_s 2^(m_s - M), O = sum_s o_s 2^(m_s - M).
+// final: out[b] = O / L and lse2[b] = M + log2 L; else (M, L, O) replaces
+// the partial in slot `first` (each thread reads its own elements of that
+// slot before writing them).
 template <int D>
-__device__ void combine_head(const DecArgs& p, int b, int nsp, float* out, float* lse2, float* s_w) {
-  const int G = p.G;
-  const int64_t base = static_cast<int64_t>(b) * p.splits;
+__device__ void merge_partials(const DecArgs& p, int64_t first, int stride, int cnt, bool final, int b, float* out,
+                               float* lse2) {
+  __shared__ float s_w[kDecGroup * kDecGMax];
   __shared__ float s_M[kDecGMax], s_L[kDecGMax];
-  if (threadIdx.x < G) {
-    const int g = threadIdx.x;
-    float M = -INFINITY;
-    for (int s = 0; s < nsp; ++s) M = fmaxf(M, __ldcg(&p.part_ml[(base + s) * G + g]).x);
-    float Ls = 0.0f;
-    for (int s = 0; s < nsp; ++s) {
-      const float2 ml = __ldcg(&p.part_ml[(base + s) * G + g]);
-      const float wgt = exp2f(ml.x - M);
-      s_w[s * kDecGMax + g] = wgt;
-      Ls += ml.y * wgt;
+  const int G = p.G, tid = threadIdx.x;
+  {
+    const int g = tid / kDecGroup, j = tid % kDecGroup;       // 16-lane group per query
+    const bool on = g < G && j < cnt;
+    float2 ml = make_float2(-INFINITY, 0.0f);
+    if (on) ml = __ldcg(&p.part_ml[(first + static_cast<int64_t>(j) * stride) * G + g]);
+    float M = ml.x;
+#pragma unroll
+    for (int o = kDecGroup / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w = on ? exp2f(ml.x - M) : 0.0f;               // m_s is finite for every written partial
+    float Ls = ml.y * w;
+#pragma unroll
+    for (int o = kDecGroup / 2; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+    if (g < G) {
+      s_w[j * kDecGMax + g] = w;
+      if (j == 0) {
+        s_M[g] = M;
+        s_L[g] = Ls;
+      }
     }
-    s_M[g] = M;
-    s_L[g] = Ls;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < G * D; e += kDecThreads) {
-    const int g = e / D;
-    float acc = 0.0f;
-#pragma unroll 8
-    for (int s = 0; s < nsp; ++s) acc = fmaf(__ldcg(&p.part_o[((base + s) * G) * D + e]), s_w[s * kDecGMax + g], acc);
-    out[static_cast<int64_t>(b) * G * D + e] = acc / s_L[g];
+  const int E4 = G * D / 4;
+  for (int e4 = tid; e4 < E4; e4 += kDecThreads) {
+    const int g = (4 * e4) / D;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int j = 0; j < kDecGroup; ++j) {
+      if (j < cnt) {
+        const float4 v =
+            __ldcg(reinterpret_cast<const float4*>(p.part_o + (first + static_cast<int64_t>(j) * stride) * G * D) + e4);
+        const float w = s_w[j * kDecGMax + g];
+        acc.x = fmaf(v.x, w, acc.x);
+        acc.y = fmaf(v.y, w, acc.y);
+        acc.z = fmaf(v.z, w, acc.z);
+        acc.w = fmaf(v.w, w, acc.w);
+      }
+    }
+    if (final) {
+      const float Lg = s_L[g];
+      reinterpret_cast<float4*>(out + static_cast<int64_t>(b) * G * D)[e4] =
+          make_float4(acc.x / Lg, acc.y / Lg, acc.z / Lg, acc.w / Lg);
+    } else {
+      reinterpret_cast<float4*>(p.part_o + first * G * D)[e4] = acc;
+    }
   }
-  if (threadIdx.x < G && lse2 != nullptr)
-    lse2[static_cast<int64_t>(b) * G + threadIdx.x] = s_M[threadIdx.x] + log2f(s_L[threadIdx.x]);
+  if (tid < G) {
+    if (final) {
+      if (lse2 != nullptr) lse2[static_cast<int64_t>(b) * G + tid] = s_M[tid] + log2f(s_L[tid]);
+    } else {
+      p.part_ml[first * G + tid] = make_float2(s_M[tid], s_L[tid]);
+    }
+  }
 }
 
 // Split-KV decode on the tensor cores (mma.sync m16n8k16, bf16 -> fp32): the
@@ -134,33 +188,14 @@ __global__ void __launch_bounds__(kDecThreads)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(full + kDecStages);
 
-  const int b = blockIdx.y, sp = blockIdx.x;
+  const DecItem it = p.items[blockIdx.x];
+  const int n = it.n;                                         // tiles of this split
+  if (n <= 0) return;                                         // uniform: no work in this item
+  const int b = it.b, sp = it.sp, t0 = it.t0, count = it.count;
+  const int64_t off = it.off;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = p.G;
-  const int count = p.counts[b];
-  const int64_t off = p.offsets[b];
-  if (count < 0 || count > p.n_c) {                           // the splits cover n_c keys at most
-    if (sp == 0 && tid == 0 && p.status != nullptr) atomicCAS(p.status, 0, KVZ_ERR_INVALID_ARG);
-    return;
-  }
-  const int ntile = (count + kDecKeys - 1) / kDecKeys;
-  const int cps = (ntile + p.splits - 1) / p.splits;          // this head's tiles spread over all its splits
-  const int t0 = sp * cps;
-  const int n = min(ntile, t0 + cps) - t0;                    // tiles of this split
-  if (ntile == 0 && sp == 0) {                                // no kept rows: output 0, lse -inf
-    for (int e = tid; e < G * D; e += kDecThreads) out[static_cast<int64_t>(b) * G * D + e] = 0.0f;
-    if (tid < G && lse2 != nullptr) lse2[static_cast<int64_t>(b) * G + tid] = -INFINITY;
-  }
-  if (n <= 0) return;                                         // uniform: no partial from this split
 
-  if (tid == 0) {
-    for (int s = 0; s < kDecStages; ++s) mbar_init(&full[s], 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  for (int e = tid; e < 8 * D; e += kDecThreads)
-    sQ[e] = e / D < G ? p.q[static_cast<int64_t>(b) * G * D + e] : uint16_t(0);
-  __syncthreads();
   auto issue = [&](int i) {
     const int s = i % kDecStages;
     mbar_arrive_expect_tx(&full[s], L::STAGE);
@@ -171,11 +206,20 @@ __global__ void __launch_bounds__(kDecThreads)
       tma_load_3d(st + L::TILE + kb * L::BLK, &tmV, &full[s], kb * 64, row, 0);
     }
   };
-  if (tid == 0) {
+  if (tid == 0) {                                             // the first tiles are in flight during the Q load
+    for (int s = 0; s < kDecStages; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
     for (int i = 0; i < n && i < kDecStages; ++i) issue(i);
   }
+  for (int e = tid; e < D; e += kDecThreads) {                // 8 rows of 16-byte chunks; rows >= G zero
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if ((e * 8) / D < G) v = reinterpret_cast<const uint4*>(p.q + static_cast<int64_t>(b) * G * D)[e];
+    reinterpret_cast<uint4*>(sQ)[e] = v;
+  }
+  __syncthreads();
 
   // A fragments of Q (rows = queries; rows 8..15 are padding and stay zero):
   // this thread's row r = lane/4, columns 2c, 2c+1 and 2c+8, 2c+9 of each k-step.
@@ -277,7 +321,8 @@ __global__ void __launch_bounds__(kDecThreads)
     sO[(warp * 8 + r) * D + nt * 8 + 2 * c + 1] = o[nt][1];
   }
   __syncthreads();
-  const int64_t part = static_cast<int64_t>(b) * p.splits + sp;
+  const int64_t part = blockIdx.x;
+  const bool single = it.nsp == 1;                            // the split is the whole head: final output
   for (int e = tid; e < G * D; e += kDecThreads) {
     const int g = e / D, dd = e % D;
     float M = -INFINITY;
@@ -292,49 +337,153 @@ __global__ void __launch_bounds__(kDecThreads)
       Ls += sL[w2 * 8 + g] * wgt;
       acc += sO[(w2 * 8 + g) * D + dd] * wgt;
     }
-    p.part_o[(part * G + g) * D + dd] = acc;
-    if (dd == 0) p.part_ml[part * G + g] = make_float2(M, Ls);
+    if (single) {
+      out[(static_cast<int64_t>(b) * G + g) * D + dd] = acc / Ls;
+      if (dd == 0 && lse2 != nullptr) lse2[static_cast<int64_t>(b) * G + g] = M + log2f(Ls);
+    } else {
+      p.part_o[(part * G + g) * D + dd] = acc;
+      if (dd == 0) p.part_ml[part * G + g] = make_float2(M, Ls);
+    }
   }
-  // ---- the CTA that finishes the head's last split merges all of them
-  __shared__ int s_last;
-  __threadfence();                                            // this partial before the count
-  __syncthreads();
-  const int nsp = (ntile + cps - 1) / cps;                    // splits of this head that have tiles
-  if (tid == 0) s_last = atomicAdd(&p.done[b], 1u) == static_cast<unsigned>(nsp - 1);
-  __syncthreads();
-  if (s_last) {
-    __threadfence();                                          // the other splits' partials before reading them
-    __syncthreads();
-    combine_head<D>(p, b, nsp, out, lse2, reinterpret_cast<float*>(smem));   // weights over the idle stages
-  }
+  if (single) return;
+  // ---- merge tree: groups of kDecGroup consecutive splits, then the groups
+  const int64_t base = part - sp;                             // the head's first split
+  const int grp = sp / kDecGroup;
+  const int ngrp = (it.nsp + kDecGroup - 1) / kDecGroup;
+  const int64_t gfirst = base + static_cast<int64_t>(grp) * kDecGroup;
+  if (!last_arrival(&p.gdone[gfirst], min(kDecGroup, it.nsp - grp * kDecGroup))) return;
+  merge_partials<D>(p, gfirst, 1, min(kDecGroup, it.nsp - grp * kDecGroup), ngrp == 1, b, out, lse2);
+  if (ngrp == 1) return;
+  if (!last_arrival(&p.done[b], ngrp)) return;
+  merge_partials<D>(p, base, kDecGroup, ngrp, true, b, out, lse2);
 }
 
 }  // namespace
 
-// Splits per head: about two waves of two CTAs per SM over all heads, at
-// most one split per 64-key tile of the longest possible head and at most
-// kDecMaxSplits (each head's tiles are spread over its splits on the device,
-// from its own count).
-void decode_plan(int64_t B, int64_t n_c, int* cps, int* splits) {
-  const int64_t max_tiles = (n_c + kDecKeys - 1) / kDecKeys;
-  const int64_t target = 148 * 2 * 2;
-  int64_t sp = (target + B - 1) / B;
-  if (sp > max_tiles) sp = max_tiles;
-  if (sp > kDecMaxSplits) sp = kDecMaxSplits;
-  if (sp < 1) sp = 1;
-  *splits = static_cast<int>(sp);
-  *cps = static_cast<int>((max_tiles + sp - 1) / sp);
+namespace {
+
+constexpr int kPlanThreads = 1024;
+
+// Block-wide sums of one value per thread (kPlanThreads threads).
+__device__ long long plan_sum(long long v, long long* s_red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  long long t = 0;
+  for (int w = 0; w < kPlanThreads / 32; ++w) t += s_red[w];
+  return t;
 }
 
-namespace {
+// Tiles of head h, or -1 for a count outside [0, n_c].
+__device__ int plan_tiles(const DecArgs& p, int h) {
+  const int c = p.counts[h];
+  return (c < 0 || c > p.n_c) ? -1 : (c + kDecKeys - 1) / kDecKeys;
+}
+
+// The decode work list (one CTA).  Every split of every head takes the same
+// number of 64-key tiles, cps, so the CTAs carry equal work whatever the
+// heads' counts (a global selection leaves them uneven).  cps is the
+// smallest value that fits all tiles into about kDecWave CTAs and gives no
+// head more than kDecMaxSplits splits.  Then sum_b ceil(tiles_b / cps) <=
+// kDecWave + B items, the grid size.  Heads with no kept rows are written
+// here (out = 0, lse2 = -inf); the finished-split counters are zeroed.
+template <int D>
+__global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecArgs p, float* out, float* lse2) {
+  __shared__ long long s_red[kPlanThreads / 32];
+  __shared__ int s_scan[kPlanThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  long long tot = 0, mx = 0;
+  for (int h = tid; h < p.B; h += kPlanThreads) {
+    const int t = plan_tiles(p, h);
+    if (t > 0) {
+      tot += t;
+      mx = max(mx, static_cast<long long>(t));
+    }
+  }
+  tot = plan_sum(tot, s_red);
+  long long m = mx;
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __syncthreads();
+  if (lane == 0) s_red[warp] = m;
+  __syncthreads();
+  for (int w = 0; w < kPlanThreads / 32; ++w) mx = max(mx, s_red[w]);
+  long long cps = (tot + kDecWave - 1) / kDecWave;
+  cps = max(cps, (mx + kDecMaxSplits - 1) / kDecMaxSplits);
+  cps = max(cps, 1ll);
+
+  const int c32 = static_cast<int>(cps);                      // <= ceil(n_c / 64)
+  __shared__ int s_base[kPlanThreads], s_nsp[kPlanThreads], s_t[kPlanThreads];
+
+  // exclusive scan of the heads' split counts, kPlanThreads heads at a time;
+  // then one warp per head writes the head's items, a lane per split
+  int carry = 0;
+  for (int h0 = 0; h0 < p.B; h0 += kPlanThreads) {
+    const int h = h0 + tid;
+    const int t = h < p.B ? plan_tiles(p, h) : 0;
+    const int nsp = t > 0 ? (t + c32 - 1) / c32 : 0;
+    int inc = nsp;                                            // inclusive scan in the warp
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    __syncthreads();                                          // the previous chunk's shared arrays are read
+    if (lane == 31) s_scan[warp] = inc;
+    __syncthreads();
+    int before = carry;
+    for (int w = 0; w < warp; ++w) before += s_scan[w];
+    int chunk = 0;
+    for (int w = 0; w < kPlanThreads / 32; ++w) chunk += s_scan[w];
+    s_base[tid] = before + inc - nsp;
+    s_nsp[tid] = nsp;
+    s_t[tid] = t;
+    if (h < p.B) {
+      p.done[h] = 0u;
+      if (t < 0 && p.status != nullptr) atomicCAS(p.status, 0, KVZ_ERR_INVALID_ARG);
+    }
+    __syncthreads();
+    const int nh = min(kPlanThreads, p.B - h0);
+    for (int hh = warp; hh < nh; hh += kPlanThreads / 32) {
+      const int hb = h0 + hh, th = s_t[hh], nb = s_nsp[hh], base = s_base[hh];
+      if (th == 0) {                                          // no kept rows: out = 0, lse2 = -inf
+        for (int e = lane; e < p.G * D; e += 32) out[static_cast<int64_t>(hb) * p.G * D + e] = 0.0f;
+        if (lse2 != nullptr && lane < p.G) lse2[static_cast<int64_t>(hb) * p.G + lane] = -INFINITY;
+      }
+      if (nb <= 0) continue;
+      const int cnt = p.counts[hb];
+      const long long offb = p.offsets[hb];
+      for (int sp = lane; sp < nb && base + sp < p.n_items; sp += 32) {   // the bound always holds; a guard
+        DecItem it;
+        it.b = hb;
+        it.sp = sp;
+        it.t0 = sp * c32;
+        it.n = min(c32, th - sp * c32);
+        it.count = cnt;
+        it.nsp = nb;
+        it.off = offb;
+        p.items[base + sp] = it;
+      }
+    }
+    carry += chunk;
+  }
+  for (int i = tid; i < p.n_items; i += kPlanThreads) p.gdone[i] = 0u;   // group counters
+  // the items past the last split do nothing
+  for (int i = carry + tid; i < p.n_items; i += kPlanThreads) {
+    DecItem it{};
+    it.b = -1;
+    p.items[i] = it;
+  }
+}
 
 template <int D>
 cudaError_t launch_split(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecArgs& a, float* out, float* lse2,
                          cudaStream_t stream) {
-  cudaError_t e = smem_limit_once<decode_split_kernel<D>>(DecLay<D>::SMEM);
+  decode_plan_kernel<D><<<1, kPlanThreads, 0, stream>>>(a, out, lse2);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(a.splits), static_cast<unsigned>(a.B));
-  decode_split_kernel<D><<<grid, kDecThreads, DecLay<D>::SMEM, stream>>>(tmK, tmV, a, out, lse2);
+  e = smem_limit_once<decode_split_kernel<D>>(DecLay<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  decode_split_kernel<D><<<a.n_items, kDecThreads, DecLay<D>::SMEM, stream>>>(tmK, tmV, a, out, lse2);
   return cudaGetLastError();
 }
 
@@ -342,9 +491,6 @@ cudaError_t launch_split(const CUtensorMap& tmK, const CUtensorMap& tmV, const D
 
 cudaError_t launch_decode(int d, const CUtensorMap& tmK, const CUtensorMap& tmV, const DecArgs& a, float* out,
                           float* lse2, cudaStream_t stream) {
-  // per-head counts of finished splits start at zero (all-zero bits)
-  cudaError_t e = launch_fill_f32(reinterpret_cast<float*>(a.done), a.B, 0.0f, stream);
-  if (e != cudaSuccess) return e;
   return d == 128 ? launch_split<128>(tmK, tmV, a, out, lse2, stream)
                   : launch_split<64>(tmK, tmV, a, out, lse2, stream);
 }

@@ -447,11 +447,10 @@ kvz_status kvz_select_heads(const float* S_head, int64_t B, int64_t n_c, double 
 
 size_t kvz_decode_workspace_size(int64_t B, int G, int64_t n_c, int d) {
   if (B < 1 || B > 65535 || G < 1 || G > kvz::kDecGMax || n_c < 1 || (d != 64 && d != 128)) return 0;
-  int cps = 0, splits = 0;
-  kvz::decode_plan(B, n_c, &cps, &splits);
-  const size_t parts = static_cast<size_t>(B) * splits * G;
-  return ((parts * 8 + 255) & ~size_t(255)) + ((parts * d * 4 + 255) & ~size_t(255)) +
-         ((static_cast<size_t>(B) * 4 + 255) & ~size_t(255));
+  const size_t items = static_cast<size_t>(kvz::decode_items(B));
+  return ((items * sizeof(kvz::DecItem) + 255) & ~size_t(255)) + ((items * G * 8 + 255) & ~size_t(255)) +
+         ((items * G * d * 4 + 255) & ~size_t(255)) + ((static_cast<size_t>(B) * 4 + 255) & ~size_t(255)) +
+         ((items * 4 + 255) & ~size_t(255));
 }
 
 kvz_status kvz_decode(const void* q, const void* K_out, const void* V_out, int64_t n_rows, const int32_t* counts,
@@ -481,11 +480,18 @@ kvz_status kvz_decode(const void* q, const void* K_out, const void* V_out, int64
   a.q = static_cast<const uint16_t*>(q);
   a.counts = counts;
   a.offsets = offsets;
-  kvz::decode_plan(B, n_c, &a.cps, &a.splits);
-  const size_t parts = static_cast<size_t>(B) * a.splits * G;
-  a.part_ml = static_cast<float2*>(workspace);
-  a.part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((parts * 8 + 255) & ~size_t(255)));
-  a.done = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(a.part_o) + ((parts * d * 4 + 255) & ~size_t(255)));
+  a.n_items = kvz::decode_items(B);
+  const size_t items = static_cast<size_t>(a.n_items);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  a.items = reinterpret_cast<kvz::DecItem*>(w);
+  w += (items * sizeof(kvz::DecItem) + 255) & ~size_t(255);
+  a.part_ml = reinterpret_cast<float2*>(w);
+  w += (items * G * 8 + 255) & ~size_t(255);
+  a.part_o = reinterpret_cast<float*>(w);
+  w += (items * G * d * 4 + 255) & ~size_t(255);
+  a.done = reinterpret_cast<unsigned*>(w);
+  w += (static_cast<size_t>(B) * 4 + 255) & ~size_t(255);
+  a.gdone = reinterpret_cast<unsigned*>(w);
   a.status = d_status;
   return kvz::launch_decode(d, tmK, tmV, a, out, lse2, stream) == cudaSuccess ? KVZ_OK : KVZ_ERR_CUDA;
 }

@@ -64,6 +64,16 @@ cudaError_t launch_fill_f32(float* x, int64_t n, float v, cudaStream_t stream);
 
 // Decode attention over the pruned cache (split-KV partials + combine).
 constexpr int kDecGMax = 8;                 // grouped queries per KV head
+// One CTA of the decode kernel: split sp of head b, tiles t0 .. t0+n-1 of
+// the head's 64-key tiles; its partial is written at the item's index, the
+// head's nsp partials at indices (index - sp) .. (index - sp + nsp - 1).
+struct __align__(16) DecItem {
+  int b, sp, t0, n;                         // n == 0: nothing to do
+  int count, nsp;                           // the head's kept rows and splits
+  long long off;                            // the head's first row in K_out / V_out
+};
+static_assert(sizeof(DecItem) == 32, "two 16-byte loads");
+
 struct DecArgs {
   int B, G;
   int64_t n_c;                              // upper bound of counts[b]
@@ -71,14 +81,16 @@ struct DecArgs {
   const uint16_t* q;                        // bf16 [B][G][d]
   const int32_t* counts;
   const int64_t* offsets;
-  int cps;                                  // 64-key tiles per split
-  int splits;                               // splits per head (grid.x)
-  float2* part_ml;                          // [B][splits][G] (running max, sum), base 2
-  float* part_o;                            // [B][splits][G][d]
-  unsigned* done;                           // [B] splits finished per head (zeroed by the launcher)
+  int n_items;                              // decode CTAs (grid.x): kDecWave + B bounds the splits
+  DecItem* items;                           // [n_items], written by the plan kernel
+  float2* part_ml;                          // [n_items][G] (running max, sum), base 2
+  float* part_o;                            // [n_items][G][d]
+  unsigned* done;                           // [B] split groups merged per head (zeroed by the plan kernel)
+  unsigned* gdone;                          // [n_items] splits finished per group, at the group's first item
   int32_t* status;
 };
-void decode_plan(int64_t B, int64_t n_c, int* cps, int* splits);
+constexpr int kDecWave = 148 * 3;           // about 1.5 waves of two decode CTAs per SM (best of 2, 3, 4, 6 per SM)
+inline int decode_items(int64_t B) { return static_cast<int>(kDecWave + B); }
 cudaError_t launch_decode(int d, const CUtensorMap& tmK, const CUtensorMap& tmV, const DecArgs& a, float* out,
                           float* lse2, cudaStream_t stream);
 

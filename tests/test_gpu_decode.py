@@ -95,3 +95,31 @@ def test_decode_reports_count_above_bound():
     kvz.kvz_decode(q, Ko, Vo, counts, offsets, 100, status=status)     # counts are 250 > 100
     torch.cuda.synchronize()
     assert int(status.item()) == 1
+
+
+def _packed(counts_list, d, seed):
+    """A packed cache with the given per-head counts (rows of head b follow those of head b-1)."""
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    rows = max(1, sum(counts_list))
+    Ko = (torch.randn((rows, d), generator=g, device="cuda") * 1.5).to(torch.bfloat16)
+    Vo = torch.randn((rows, d), generator=g, device="cuda").to(torch.bfloat16)
+    counts = torch.tensor(counts_list, dtype=torch.int32, device="cuda")
+    offsets = torch.zeros(len(counts_list) + 1, dtype=torch.int64, device="cuda")
+    offsets[1:] = torch.cumsum(counts.long(), 0)
+    return Ko, Vo, counts, offsets
+
+
+@pytest.mark.parametrize("counts_list,n_c,G", [
+    ([131072] + [37] * 7, 131072, 8),             # one head holds nearly all rows: its splits reach the cap
+    ([0, 20000, 0, 64, 65, 1, 0, 3000], 20000, 4),  # empty heads between uneven ones, tile-edge counts
+    ([n % 300 for n in range(1000)], 300, 2),     # more heads than CTAs in two waves
+])
+def test_decode_uneven_heads(counts_list, n_c, G):
+    d = 128
+    Ko, Vo, counts, offsets = _packed(counts_list, d, seed=len(counts_list))
+    B = len(counts_list)
+    q = torch.randn((B, G, d), generator=torch.Generator(device="cuda").manual_seed(B), device="cuda")
+    o = _check(q.to(torch.bfloat16), Ko, Vo, counts, offsets, n_c, 0.088)
+    for b, c in enumerate(counts_list):
+        if c == 0:
+            assert np.all(o[b] == 0)
