@@ -145,48 +145,68 @@ __global__ void __launch_bounds__(kGatherThreads)
 // a = max |x| over the row, scale = a / 127 and code = rint(x * (127 / a)),
 // clamped to [-127, 127]; a row of zeros has code 0 and scale 0.  The two
 // divisions and the product are single IEEE float32 operations (no fused or
-// approximate forms), so the codes are reproducible to the bit.  A row is
-// read by vpr threads (16 bytes each); its absmax comes from a shuffle
-// reduction over them.  HBM-bound: 4d bytes read, 2d + 8 written per row.
-constexpr int kQuantThreads = 256;
+// approximate forms), so the codes are reproducible to the bit.
+// HBM-bound: 4d bytes read, 2d + 8 written per row.
+//
+// Two threads per row.  A CTA of 256 threads takes units of 64 slots of one
+// head: threads 0-127 own the unit's K rows, 128-255 its V rows, a pair of
+// adjacent lanes per row, one half of the row each; a shuffle combines the
+// pair's absmax.  The rows of the next units arrive by cp.async (coalesced,
+// 16 bytes per thread) into a three-stage ring while the current unit is
+// quantised.  Each unit's count, offsets and source indices are fetched a
+// unit earlier still and carried in registers, and a CTA steps through its
+// units without integer division, so nothing between the barriers waits on
+// memory or on a 64-bit divide (these two cost 12% of the kernel's time).  A
+// thread reads its half row from shared memory twice (absmax, then codes),
+// writes the codes into a staging tile, and one bulk copy per tensor stores
+// the unit's code rows, which are contiguous in the output.  The 16-byte
+// chunks of a staged row are XOR-swizzled and each thread visits its chunks
+// in a rotated order, chosen by exhaustive search so that at d = 128 no
+// shared-memory access has a bank conflict (at d = 64 some are two-way).
+constexpr int kQ8Rows = 64;                                     // slots per unit
+constexpr int kQ8Threads = 256;
+constexpr int kQ8Stages = 3;                                    // units in the ring: two in flight
 
-// Codes of 8 bf16 values.  v = x * inv is one IEEE product; adding 1.5 * 2^23
-// then rounds v to the nearest integer (ties to even, |v| < 2^22) and leaves
-// that integer in the low bits of the sum's pattern, so the code is its low
-// byte.  |x| <= a gives |v| <= 127 (1 + 2^-24)^2 < 127.5: the code never
-// leaves [-127, 127].
-__device__ __forceinline__ void quant8(const int4& w, float inv, int8_t* dst) {
-  constexpr float kRound = 12582912.0f;                       // 1.5 * 2^23
-  const uint32_t u[4] = {static_cast<uint32_t>(w.x), static_cast<uint32_t>(w.y), static_cast<uint32_t>(w.z),
-                         static_cast<uint32_t>(w.w)};
-  uint32_t c[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    c[2 * i] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(u[i] << 16), inv), kRound));
-    c[2 * i + 1] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(u[i] & 0xFFFF0000u), inv), kRound));
-  }
-  const uint32_t lo = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
-  const uint32_t hi = __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410);
-  *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+template <int D>
+struct Q8 {
+  static constexpr int VPR = D / 8;                             // 16-byte chunks of a bf16 row
+  static constexpr int NCO = D / 16;                            // 16-byte chunks of a code row
+  static constexpr int CPH = VPR / 2;                           // input chunks per half row
+  static constexpr int COH = NCO / 2;                           // code chunks per half row
+  static constexpr int RPT = VPR / 4;                           // rows each thread loads, per tensor
+  static constexpr int LSTRIDE = kQ8Threads / VPR;              // loader row stride
+  static constexpr int ROWB = D * 2;
+  static constexpr int STAGE = 2 * kQ8Rows * ROWB;              // K rows, then V rows
+  static constexpr int OUT = 2 * kQ8Rows * D;                   // K codes, then V codes
+  static constexpr int SMEM = kQ8Stages * STAGE + OUT;
+  // chunk c of staged row r sits at chunk c ^ swz(r)
+  __device__ static int swz(int r) { return r & (VPR - 1); }
+  // step c of the absmax pass reads input chunk h*CPH + p1(c, r, h); step k
+  // of the code pass writes code chunk h*COH + p2(k, r, h)
+  __device__ static int p1(int c, int r, int h) { return D == 128 ? ((c + 4 * h) & 7) : c; }
+  __device__ static int p2(int k, int r, int h) { return D == 128 ? ((k + r + 2 * h) & 3) : k; }
+};
+
+// Codes of 4 bf16 values (w0 = x1:x0, w1 = x3:x2), x0 in the low byte.
+// v = x * inv is one IEEE product; adding 1.5 * 2^23 rounds v to the nearest
+// integer (ties to even, |v| < 2^22) and leaves that integer in the low bits
+// of the sum's pattern, so the code is its low byte.  |x| <= a gives |v| <=
+// 127 (1 + 2^-24)^2 < 127.5: the code never leaves [-127, 127].
+__device__ __forceinline__ uint32_t code4(uint32_t w0, uint32_t w1, float inv) {
+  constexpr float kRound = 12582912.0f;                         // 1.5 * 2^23
+  const uint32_t c0 = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(w0 << 16), inv), kRound));
+  const uint32_t c1 = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(w0 & 0xFFFF0000u), inv), kRound));
+  const uint32_t c2 = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(w1 << 16), inv), kRound));
+  const uint32_t c3 = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(w1 & 0xFFFF0000u), inv), kRound));
+  return __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
 }
 
-// max |x| of 8 bf16 values: magnitude patterns (sign cleared) order like the
-// magnitudes, so two-lane 16-bit integer maxima find it.
-__device__ __forceinline__ float absmax8(const int4& w) {
-  const uint32_t m = __vmaxu2(__vmaxu2(static_cast<uint32_t>(w.x) & 0x7FFF7FFFu, static_cast<uint32_t>(w.y) & 0x7FFF7FFFu),
-                              __vmaxu2(static_cast<uint32_t>(w.z) & 0x7FFF7FFFu, static_cast<uint32_t>(w.w) & 0x7FFF7FFFu));
-  const uint32_t h = (m >> 16) > (m & 0xFFFFu) ? (m >> 16) : (m & 0xFFFFu);
-  return __uint_as_float(h << 16);
+// Magnitude patterns (sign cleared) of bf16 values order like the
+// magnitudes, so two-lane 16-bit integer maxima find max |x|.
+__device__ __forceinline__ uint32_t absmax_u2(const uint4& w, uint32_t m) {
+  return __vmaxu2(__vmaxu2(m, __vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu)),
+                  __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu));
 }
-
-// Work unit = (head b, block of 64 slots of that head): the head is known
-// without a search, and units past a head's count are skipped.  A CTA walks
-// its units with a two-stage shared-memory ring: the rows of its next unit
-// are in flight (cp.async) while the current one is quantised, and the
-// source indices of the unit after that are fetched a step earlier still, so
-// the bytes in flight do not depend on registers or on the compute phase.
-constexpr int kQuantRows = 64;                                  // slots per unit
-constexpr int kQuantStageBytes = 2 * kQuantRows * 256;          // K and V rows of a unit at d = 128
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
@@ -195,145 +215,167 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Bulk copy shared -> global (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_store(void* gmem_dst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
+               "r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_src))), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// This thread's shared-memory writes, visible to the bulk copy (async proxy).
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-__global__ void __launch_bounds__(kQuantThreads)
-    compact_int8_kernel(const int4* __restrict__ K, const int4* __restrict__ V, int64_t B, int64_t n_c, int vpr,
+template <int D>
+__global__ void __launch_bounds__(kQ8Threads)
+    compact_int8_kernel(const int4* __restrict__ K, const int4* __restrict__ V, int64_t B, int64_t n_c,
                         const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
                         const int64_t* __restrict__ offsets, const int64_t* __restrict__ out_offsets,
                         int8_t* __restrict__ Kq, int8_t* __restrict__ Vq, float* __restrict__ Ks,
                         float* __restrict__ Vs, int32_t* status) {
-  extern __shared__ int4 qstage[];                              // [2][K rows | V rows] of a unit
-  constexpr int kPer = kQuantRows / (kQuantThreads / 16);       // rows per thread (4 at d=128, 2 at d=64)
-  const int rows_per_step = kQuantThreads / vpr;
-  const int per = kQuantRows / rows_per_step;                   // rows of a unit per thread
-  const int64_t bph = (n_c + kQuantRows - 1) / kQuantRows;      // units per head
-  const int64_t nunits = B * bph;
-  const int my_row = threadIdx.x / vpr;
-  const int vec = threadIdx.x % vpr;
-  const int tensor_vec = kQuantRows * vpr;
+  using L = Q8<D>;
+  extern __shared__ __align__(128) uint8_t q8s[];               // [3 stages][K | V rows], [K | V codes]
+  const int t = threadIdx.x;
+  const int64_t bph = (n_c + kQ8Rows - 1) / kQ8Rows;            // units per head
+  const int lc = t % L::VPR;                                    // loader: chunk lc of rows lr0 + j * LSTRIDE
+  const int lr0 = t / L::VPR;
+  const int tensor = t >> 7;                                    // quantiser: half h of row r of K (0) or V (1)
+  const int r = (t & 127) >> 1, h = t & 1;
 
-  // next unit of this CTA at or after u that has slots (nunits when none)
-  auto next_active = [&](int64_t u) -> int64_t {
-    for (; u < nunits; u += gridDim.x) {
-      const int64_t cnt = counts[u / bph];
-      if (cnt < 0 || cnt > n_c) {
-        if ((u % bph) == 0 && threadIdx.x == 0) report_err(status, KVZ_ERR_INVALID_ARG);
+  // A unit is (head hb, 64-slot block blk); this CTA visits units blockIdx.x,
+  // blockIdx.x + gridDim.x, ... in that order, stepping (hb, blk) without a
+  // division.  Each queued unit carries what its processing needs (count,
+  // offsets, this thread's source rows), fetched a unit ahead.
+  struct Unit {
+    int64_t hb, blk, cnt, in0, out0;                             // hb == B: none
+    int32_t own;                                                 // source row of this thread's quantiser row
+  };
+  const int64_t step_hb = gridDim.x / bph, step_blk = gridDim.x % bph;
+  auto advance = [&](Unit& x) {
+    x.blk += step_blk;
+    x.hb += step_hb;
+    if (x.blk >= bph) {
+      x.blk -= bph;
+      ++x.hb;
+    }
+  };
+  // the first unit at or after x (inclusive) that has slots; then its offsets and source rows
+  auto next_active = [&](Unit& x, int32_t (&src)[L::RPT]) {
+    for (; x.hb < B; advance(x)) {
+      x.cnt = counts[x.hb];
+      if (x.cnt < 0 || x.cnt > n_c) {
+        if (x.blk == 0 && t == 0) report_err(status, KVZ_ERR_INVALID_ARG);
         continue;
       }
-      if ((u % bph) * kQuantRows < cnt) return u;
+      if (x.blk * kQ8Rows < x.cnt) break;
     }
-    return nunits;
-  };
-  // source row of each of this thread's slots in unit u (-1: no slot there)
-  auto fetch_src = [&](int64_t u, int32_t (&src)[kPer]) {
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) src[k] = -1;
-    if (u >= nunits) return;
-    const int64_t hb = u / bph, p0 = (u % bph) * kQuantRows, cnt = counts[hb], in0 = offsets[hb];
+    for (int j = 0; j < L::RPT; ++j) src[j] = -1;
+    x.own = -1;
+    if (x.hb >= B) return;
+    x.in0 = offsets[x.hb];
+    x.out0 = (out_offsets != nullptr ? out_offsets[x.hb] : x.in0) + x.blk * kQ8Rows;
+    const int64_t p0 = x.blk * kQ8Rows;
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const int64_t pp = p0 + my_row + k * rows_per_step;
-      if (k < per && pp < cnt) src[k] = idx[in0 + pp];
+    for (int j = 0; j < L::RPT; ++j) {
+      const int64_t pp = p0 + lr0 + j * L::LSTRIDE;
+      if (pp < x.cnt) src[j] = idx[x.in0 + pp];
     }
+    if (p0 + r < x.cnt) x.own = idx[x.in0 + p0 + r];
   };
-  auto issue = [&](int64_t u, int st, const int32_t (&src)[kPer]) {
-    if (u < nunits) {
-      const int64_t hb = u / bph;
-      int4* sk = qstage + st * 2 * tensor_vec;
+  auto issue = [&](const Unit& x, int st, const int32_t (&src)[L::RPT]) {
+    if (x.hb < B) {
+      uint8_t* sk = q8s + st * L::STAGE;
+      const int4* kb = K + x.hb * n_c * L::VPR + lc;
+      const int4* vb = V + x.hb * n_c * L::VPR + lc;
 #pragma unroll
-      for (int k = 0; k < kPer; ++k) {
-        const int64_t j = src[k];
-        if (k < per && j >= 0 && j < n_c) {
-          const int r = my_row + k * rows_per_step;
-          cp_async16(sk + r * vpr + vec, K + (hb * n_c + j) * vpr + vec);
-          cp_async16(sk + tensor_vec + r * vpr + vec, V + (hb * n_c + j) * vpr + vec);
+      for (int j = 0; j < L::RPT; ++j) {
+        const int64_t s = src[j];
+        if (s >= 0 && s < n_c) {
+          const int row = lr0 + j * L::LSTRIDE;
+          const int off = row * L::ROWB + ((lc ^ L::swz(row)) * 16);
+          cp_async16(sk + off, kb + s * L::VPR);
+          cp_async16(sk + kQ8Rows * L::ROWB + off, vb + s * L::VPR);
         }
       }
     }
     cp_async_commit();
   };
 
-  int32_t src_cur[kPer], src_nxt[kPer];
-  int64_t u = next_active(blockIdx.x);
-  fetch_src(u, src_cur);
-  issue(u, 0, src_cur);
-  int64_t un = next_active(u + gridDim.x);
-  fetch_src(un, src_nxt);
+  // ring of three stages: units x0 (quantised now), x1 and x2 (in flight)
+  int32_t src[L::RPT];
+  Unit x0{static_cast<int64_t>(blockIdx.x) / bph, static_cast<int64_t>(blockIdx.x) % bph, 0, 0, 0, -1};
+  next_active(x0, src);
+  issue(x0, 0, src);
+  Unit x1 = x0;
+  advance(x1);
+  next_active(x1, src);
+  issue(x1, 1, src);
+  Unit x2 = x1;
+  advance(x2);
+  next_active(x2, src);
   int st = 0;
-  while (u < nunits) {
-    issue(un, st ^ 1, src_nxt);                                   // the next unit's rows go in flight
-    const int64_t unn = next_active(un + gridDim.x);
-    int32_t src_nn[kPer];
-    fetch_src(unn, src_nn);                                       // and the indices of the one after
-    cp_async_wait1();                                             // this thread's rows of unit u
-    __syncthreads();                                              // everyone's
-    const int64_t hb = u / bph, p0 = (u % bph) * kQuantRows;
-    const int64_t cnt = counts[hb];
-    const int64_t out0 = (out_offsets != nullptr ? out_offsets[hb] : offsets[hb]) + p0;
-    const int4* sk = qstage + st * 2 * tensor_vec;
-    // absmax of each row (K and V) over its vpr lanes
-    float ak[kPer], av[kPer];
-    int4 kv[kPer], vv[kPer];
+  while (x0.hb < B) {
+    issue(x2, st == 0 ? 2 : st - 1, src);                       // stage (st + 2) % 3
+    Unit x3 = x2;
+    advance(x3);
+    next_active(x3, src);                                       // the unit after, and its indices
+    cp_async_wait2();                                           // this thread's copies into stage st
+    __syncthreads();                                            // everyone's
+
+    const int nvalid = static_cast<int>(x0.cnt - x0.blk * kQ8Rows < kQ8Rows ? x0.cnt - x0.blk * kQ8Rows : kQ8Rows);
+    const int64_t out0 = x0.out0;
+    const uint8_t* srow = q8s + st * L::STAGE + tensor * kQ8Rows * L::ROWB + r * L::ROWB;
+    uint8_t* orow = q8s + kQ8Stages * L::STAGE + tensor * kQ8Rows * D + r * D;
+    const bool live = r < nvalid;
+    const bool ok = x0.own >= 0 && x0.own < n_c;
+    uint32_t m2 = 0u;
+    if (live) {
+      if (!ok && h == 0) report_err(status, KVZ_ERR_INVALID_ARG);   // idx out of [0, n_c): zeros
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const int r = my_row + k * rows_per_step;
-      kv[k] = vv[k] = make_int4(0, 0, 0, 0);
-      if (k < per) {
-        kv[k] = sk[r * vpr + vec];
-        vv[k] = sk[tensor_vec + r * vpr + vec];
-      }
-      ak[k] = absmax8(kv[k]);
-      av[k] = absmax8(vv[k]);
+      for (int c = 0; c < L::CPH; ++c)
+        m2 = absmax_u2(*reinterpret_cast<const uint4*>(srow + (((h * L::CPH + L::p1(c, r, h)) ^ L::swz(r)) * 16)),
+                       m2);
+    }
+    m2 = __vmaxu2(m2, __shfl_xor_sync(0xffffffffu, m2, 1));    // the row's other half
+    const uint32_t hm = max(m2 >> 16, m2 & 0xFFFFu);
+    const float a = ok ? __uint_as_float(hm << 16) : 0.0f;
+    if (t == 0) bulk_wait_read0();                              // the code tile: the last store has read it
+    __syncthreads();
+    if (live) {
+      const float inv = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
 #pragma unroll
-      for (int o2 = 1; o2 < 16; o2 <<= 1) {
-        if (o2 < vpr) {
-          ak[k] = fmaxf(ak[k], __shfl_xor_sync(0xffffffffu, ak[k], o2));
-          av[k] = fmaxf(av[k], __shfl_xor_sync(0xffffffffu, av[k], o2));
+      for (int k = 0; k < L::COH; ++k) {
+        const int cc = h * L::COH + L::p2(k, r, h);
+        uint4 code = make_uint4(0u, 0u, 0u, 0u);
+        if (ok) {
+          const uint4 w0 = *reinterpret_cast<const uint4*>(srow + (((2 * cc) ^ L::swz(r)) * 16));
+          const uint4 w1 = *reinterpret_cast<const uint4*>(srow + (((2 * cc + 1) ^ L::swz(r)) * 16));
+          code = make_uint4(code4(w0.x, w0.y, inv), code4(w0.z, w0.w, inv), code4(w1.x, w1.y, inv),
+                            code4(w1.z, w1.w, inv));
         }
+        *reinterpret_cast<uint4*>(orow + cc * 16) = code;
       }
+      if (h == 0) (tensor == 0 ? Ks : Vs)[out0 + r] = __fdiv_rn(a, 127.0f);
     }
-    // the row divisions run in parallel, one per lane of the row's group
-    float a = 0.0f;
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      if (vec == 2 * k) a = ak[k];
-      if (vec == 2 * k + 1) a = av[k];
+    fence_proxy_async_smem();                                   // the code tile, to the bulk copy
+    __syncthreads();                                            // stage st and the tile are complete
+    if (t == 0) {
+      const uint8_t* tile = q8s + kQ8Stages * L::STAGE;
+      bulk_store(Kq + out0 * D, tile, static_cast<uint32_t>(nvalid * D));
+      bulk_store(Vq + out0 * D, tile + kQ8Rows * D, static_cast<uint32_t>(nvalid * D));
+      bulk_commit();
     }
-    const float inv = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
-    const float scl = __fdiv_rn(a, 127.0f);
-    const int group = (threadIdx.x & 31) & ~(vpr - 1);
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const float ik = __shfl_sync(0xffffffffu, inv, group + 2 * k);
-      const float iv = __shfl_sync(0xffffffffu, inv, group + 2 * k + 1);
-      const float sk2 = __shfl_sync(0xffffffffu, scl, group + 2 * k);
-      const float sv2 = __shfl_sync(0xffffffffu, scl, group + 2 * k + 1);
-      const int r = my_row + k * rows_per_step;
-      if (k < per && p0 + r < cnt && src_cur[k] >= 0 && src_cur[k] < n_c) {
-        const int64_t dst = out0 + r;
-        quant8(kv[k], ik, Kq + dst * vpr * 8 + vec * 8);
-        quant8(vv[k], iv, Vq + dst * vpr * 8 + vec * 8);
-        if (vec == 0) {
-          Ks[dst] = sk2;
-          Vs[dst] = sv2;
-        }
-      } else if (k < per && p0 + r < cnt && vec == 0) {
-        report_err(status, KVZ_ERR_INVALID_ARG);                  // idx out of [0, n_c)
-      }
-    }
-    __syncthreads();                                              // stage st is free again
-    u = un;
-    un = unn;
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      src_cur[k] = src_nxt[k];
-      src_nxt[k] = src_nn[k];
-    }
-    st ^= 1;
+    x0 = x1;
+    x1 = x2;
+    x2 = x3;
+    st = st == 2 ? 0 : st + 1;
   }
   cp_async_wait0();
+  if (t == 0) bulk_wait_all();
 }
 
 // Dependencies of in-place compaction.  Slot chunk c (slots [cC, (c+1)C))
@@ -553,21 +595,32 @@ cudaError_t launch_compact_gather(const void* K, const void* V, int64_t B, int64
   return cudaGetLastError();
 }
 
+namespace {
+template <int D>
+cudaError_t launch_int8(const void* K, const void* V, int64_t B, int64_t n_c, const int32_t* idx,
+                        const int32_t* counts, const int64_t* offsets, const int64_t* out_offsets, int8_t* Kq,
+                        int8_t* Vq, float* K_scale, float* V_scale, int32_t* status, cudaStream_t stream) {
+  cudaError_t e = smem_limit_once<compact_int8_kernel<D>>(Q8<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  int64_t blocks = B * ((n_c + kQ8Rows - 1) / kQ8Rows);
+  const int64_t cap = D == 128 ? 148 * 2 : 148 * 3;              // resident CTAs per SM by shared memory (112 / 56 KB)
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  compact_int8_kernel<D><<<static_cast<unsigned>(blocks), kQ8Threads, Q8<D>::SMEM, stream>>>(
+      static_cast<const int4*>(K), static_cast<const int4*>(V), B, n_c, idx, counts, offsets, out_offsets, Kq, Vq,
+      K_scale, V_scale, status);
+  return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t launch_compact_int8(const void* K, const void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
                                 const int32_t* counts, const int64_t* offsets, const int64_t* out_offsets,
                                 int8_t* Kq, int8_t* Vq, float* K_scale, float* V_scale, int32_t* status,
                                 cudaStream_t stream) {
-  const int vpr = d / 8;
-  const int smem = 2 * 2 * kQuantRows * vpr * 16;               // two stages of a unit's K and V rows
-  cudaError_t e = smem_limit_once<compact_int8_kernel>(kQuantStageBytes * 2);
-  if (e != cudaSuccess) return e;
-  int64_t blocks = B * ((n_c + kQuantRows - 1) / kQuantRows);
-  if (blocks > 148 * 3) blocks = 148 * 3;                       // three CTAs per SM (64 KB each at d = 128)
-  if (blocks < 1) blocks = 1;
-  compact_int8_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, smem, stream>>>(
-      static_cast<const int4*>(K), static_cast<const int4*>(V), B, n_c, vpr, idx, counts, offsets, out_offsets, Kq,
-      Vq, K_scale, V_scale, status);
-  return cudaGetLastError();
+  return d == 128 ? launch_int8<128>(K, V, B, n_c, idx, counts, offsets, out_offsets, Kq, Vq, K_scale, V_scale,
+                                     status, stream)
+                  : launch_int8<64>(K, V, B, n_c, idx, counts, offsets, out_offsets, Kq, Vq, K_scale, V_scale,
+                                    status, stream);
 }
 
 size_t compact_workspace_bytes(int64_t B, int64_t n_c) {
