@@ -529,6 +529,14 @@ def main():
         ora_set = set(int(v) for v in oracle_idx)
         line["selection_overlap"] = {"head": 0, "jaccard": len(gpu_set & ora_set) / max(1, len(gpu_set | ora_set)),
                                      "kept": len(ora_set)}
+        # exact ties among the GPU's scores of head 0: at the keep threshold
+        # (where the lower-index rule decides) and overall (equal fp32 values)
+        import numpy as np
+        s0 = c.S[0].cpu().numpy()
+        k0 = o1 - o0
+        thr = np.sort(s0)[::-1][k0 - 1] if k0 > 0 else np.float32(np.inf)
+        line["ties"] = {"head": 0, "at_threshold": int(np.count_nonzero(s0 == thr)) if k0 > 0 else 0,
+                        "duplicate_values": int(s0.size - np.unique(s0).size)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
