@@ -204,6 +204,52 @@ kvz_status kvz_select(const float* S, int64_t B, int64_t n_c, double ratio,
                       int32_t* d_status, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Global selection with the heads of one context split over ranks          */
+/* (KVzip §4.1: the r% budget spans all heads of all layers, so a context    */
+/* whose layers sit on several GPUs needs one exchange per radix digit).     */
+/*                                                                          */
+/* The result equals kvz_select(KVZ_GLOBAL) on the concatenation of every    */
+/* rank's S in rank order (rank r holds B_local heads that come after those */
+/* of ranks 0..r-1): k = floor(ratio * B_total * n_c), ties to the lower     */
+/* flattened index across ranks.  Each rank gets the CSR form of its own     */
+/* heads (counts, offsets from 0, idx ascending per head).                   */
+/*                                                                          */
+/* Sequence on every rank, the caller doing the exchanges in between:       */
+/*   kvz_select_dist_begin      writes this rank's first-digit histogram     */
+/*   for pass 0, 1, 2:                                                       */
+/*     (caller) hist <- sum of hist over ranks (in place, uint32 [2048])     */
+/*     kvz_select_dist_step(pass)  picks the digit; for pass < 2 writes the  */
+/*                                 next local histogram, for pass 2 writes   */
+/*                                 eq_total[0] = keys of this rank equal to  */
+/*                                 the threshold (uint64)                    */
+/*   (caller) eq_ranks[r] <- eq_total of rank r, for every rank (all-gather) */
+/*   kvz_select_dist_finish      writes counts, offsets and idx              */
+/* Layout: S [B_local][n_c] fp32 (as kvz_select); hist: 2048 uint32 of      */
+/* device memory, 16-byte aligned, owned by the caller and left zeroed by   */
+/* the last step; eq_total: one uint64; eq_ranks: world uint64.  All calls  */
+/* take the same workspace (kvz_select_dist_workspace_size bytes, 16-byte   */
+/* aligned), which carries the state from one call to the next.             */
+/* idx_capacity >= min(k, B_local * n_c).  B_total >= B_local, 0 <= rank,  */
+/* B_total * n_c < 2^32.                                                    */
+/* Errors as kvz_select; every rank must make the same calls.               */
+/* ------------------------------------------------------------------------ */
+size_t kvz_select_dist_workspace_size(int64_t B_local, int64_t n_c);
+
+kvz_status kvz_select_dist_begin(const float* S, int64_t B_local, int64_t n_c, int64_t B_total,
+                                 double ratio, uint32_t* hist, void* workspace,
+                                 size_t workspace_bytes, int32_t* d_status, cudaStream_t stream);
+
+kvz_status kvz_select_dist_step(const float* S, int64_t B_local, int64_t n_c, int pass,
+                                uint32_t* hist, uint64_t* eq_total, void* workspace,
+                                size_t workspace_bytes, int32_t* d_status, cudaStream_t stream);
+
+kvz_status kvz_select_dist_finish(const float* S, int64_t B_local, int64_t n_c, int64_t B_total,
+                                  double ratio, const uint64_t* eq_ranks, int rank,
+                                  int32_t* idx, int64_t idx_capacity, int32_t* counts,
+                                  int64_t* offsets, void* workspace, size_t workspace_bytes,
+                                  int32_t* d_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Context-independent head scores and head-level eviction (KVzip §4.2,     */
 /* "context-independent eviction": one static importance per head, the pair  */
 /* scores aggregated by a max along the sequence).                           */

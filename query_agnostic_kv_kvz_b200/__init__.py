@@ -16,11 +16,13 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "KvzError", "KvzLibraryError", "lib", "lib_path", "STATUS",
-    "kvz_version", "kvz_keep_count",
-    "kvz_score_workspace_size", "kvz_score", "kvz_score_lse2", "kvz_score_colmax",
-    "kvz_select_workspace_size", "kvz_select", "kvz_compact_workspace_size", "kvz_compact",
-    "PER_HEAD", "GLOBAL",
+    "KvzError", "KvzLibraryError", "lib", "lib_path", "STATUS", "PER_HEAD", "GLOBAL",
+    "kvz_version", "kvz_keep_count", "kvz_score_workspace_size", "kvz_score", "kvz_score_noalloc",
+    "kvz_score_lse2", "kvz_score_colmax", "kvz_select_workspace_size", "kvz_select",
+    "kvz_select_dist_workspace_size", "kvz_select_dist_begin", "kvz_select_dist_step", "kvz_select_dist_finish",
+    "kvz_compact_workspace_size", "kvz_compact", "kvz_compress_host_workspace_size", "kvz_compress_host",
+    "kvz_score_chunked_workspace_size", "kvz_score_chunked", "kvz_head_score", "kvz_select_heads", "kvz_decode",
+    "kvz_select_protected", "kvz_compact_int8",
 ]
 
 PER_HEAD = 0
@@ -63,6 +65,11 @@ _SIGS = {
     "kvz_keep_count": (_i64, [_i64, _f64]),
     "kvz_select_workspace_size": (_sz, [_i64, _i64, _i32]),
     "kvz_select": (_i32, [_vp, _i64, _i64, _f64, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "kvz_select_dist_workspace_size": (_sz, [_i64, _i64]),
+    "kvz_select_dist_begin": (_i32, [_vp, _i64, _i64, _i64, _f64, _vp, _vp, _sz, _vp, _vp]),
+    "kvz_select_dist_step": (_i32, [_vp, _i64, _i64, _i32, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "kvz_select_dist_finish": (_i32, [_vp, _i64, _i64, _i64, _f64, _vp, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp,
+                                      _vp]),
     "kvz_compact_workspace_size": (_sz, [_i64, _i64]),
     "kvz_compact": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp]),
     "kvz_select_protected": (_i32, [_vp, _i64, _i64, _f64, _i32, _i64, _vp, _i64, _vp, _vp, _vp, _sz, _vp, _vp]),
@@ -250,6 +257,46 @@ def kvz_select(S, ratio: float, mode="per_head", idx=None, counts=None, offsets=
     _check("kvz_select", lib().kvz_select(_ptr(S), B, n_c, float(ratio), m, _ptr(idx), idx.numel(), _ptr(counts),
                                           _ptr(offsets), _ptr(workspace), nbytes, _ptr(status), _stream(stream)))
     return idx, counts, offsets
+
+
+def kvz_select_dist_workspace_size(B_local: int, n_c: int) -> int:
+    return lib().kvz_select_dist_workspace_size(B_local, n_c)
+
+
+def _dist_args(S, workspace):
+    if S.dim() != 2 or S.dtype != torch.float32 or not S.is_contiguous():
+        raise ValueError("S must be a contiguous float32 [B_local, n_c] tensor")
+    return S.shape[0], S.shape[1], workspace.numel() * workspace.element_size()
+
+
+def kvz_select_dist_begin(S, B_total: int, ratio: float, hist, workspace, status=None, stream=None):
+    """First step of the global selection over heads split across ranks:
+    this rank's first-digit histogram into hist (uint32 [2048], as int32)."""
+    _need_cuda(S, hist, workspace, status)
+    B, n_c, nbytes = _dist_args(S, workspace)
+    _check("kvz_select_dist_begin", lib().kvz_select_dist_begin(
+        _ptr(S), B, n_c, int(B_total), float(ratio), _ptr(hist), _ptr(workspace), nbytes, _ptr(status),
+        _stream(stream)))
+
+
+def kvz_select_dist_step(S, pass_: int, hist, eq_total, workspace, status=None, stream=None):
+    """Digit pick from the rank-summed hist; the next local histogram, or
+    (pass 2) this rank's threshold-equal count into eq_total (int64 [1])."""
+    _need_cuda(S, hist, eq_total, workspace, status)
+    B, n_c, nbytes = _dist_args(S, workspace)
+    _check("kvz_select_dist_step", lib().kvz_select_dist_step(
+        _ptr(S), B, n_c, int(pass_), _ptr(hist), _ptr(eq_total), _ptr(workspace), nbytes, _ptr(status),
+        _stream(stream)))
+
+
+def kvz_select_dist_finish(S, B_total: int, ratio: float, eq_ranks, rank: int, idx, counts, offsets, workspace,
+                           status=None, stream=None):
+    """Last step: this rank's kept positions (CSR over its own heads)."""
+    _need_cuda(S, eq_ranks, idx, counts, offsets, workspace, status)
+    B, n_c, nbytes = _dist_args(S, workspace)
+    _check("kvz_select_dist_finish", lib().kvz_select_dist_finish(
+        _ptr(S), B, n_c, int(B_total), float(ratio), _ptr(eq_ranks), int(rank), _ptr(idx), idx.numel(),
+        _ptr(counts), _ptr(offsets), _ptr(workspace), nbytes, _ptr(status), _stream(stream)))
 
 
 def kvz_compact_workspace_size(B: int, n_c: int) -> int:

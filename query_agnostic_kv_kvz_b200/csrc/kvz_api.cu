@@ -380,6 +380,79 @@ kvz_status kvz_select(const float* S, int64_t B, int64_t n_c, double ratio, int 
              : KVZ_ERR_CUDA;
 }
 
+namespace {
+// Host checks shared by the distributed selection calls.
+kvz_status dist_check(const float* S, int64_t B_local, int64_t n_c, const void* ws, size_t ws_bytes,
+                      kvz::SelWorkspace* lay) {
+  if (S == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (B_local < 1 || B_local > 65535 || n_c < 1 || n_c > kMaxRows) return KVZ_ERR_INVALID_ARG;
+  if (B_local * n_c >= (int64_t(1) << 32)) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(S, 4)) return KVZ_ERR_ALIGNMENT;
+  *lay = kvz::select_workspace(B_local, n_c, KVZ_GLOBAL);
+  if (ws == nullptr || ws_bytes < lay->bytes) return KVZ_ERR_WORKSPACE;
+  if (!aligned(ws, 16)) return KVZ_ERR_ALIGNMENT;
+  return KVZ_OK;
+}
+}  // namespace
+
+size_t kvz_select_dist_workspace_size(int64_t B_local, int64_t n_c) {
+  if (B_local < 1 || n_c < 1) return 0;
+  return kvz::select_workspace(B_local, n_c, KVZ_GLOBAL).bytes;
+}
+
+kvz_status kvz_select_dist_begin(const float* S, int64_t B_local, int64_t n_c, int64_t B_total, double ratio,
+                                 uint32_t* hist, void* workspace, size_t workspace_bytes, int32_t* d_status,
+                                 cudaStream_t stream) {
+  kvz::SelWorkspace lay;
+  const kvz_status st = dist_check(S, B_local, n_c, workspace, workspace_bytes, &lay);
+  if (st != KVZ_OK) return st;
+  if (hist == nullptr) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(hist, 16)) return KVZ_ERR_ALIGNMENT;
+  if (B_total < B_local || !(ratio >= 0.0 && ratio <= 1.0)) return KVZ_ERR_INVALID_ARG;
+  if (B_total * n_c >= (int64_t(1) << 32)) return KVZ_ERR_INVALID_ARG;   // histogram bins are 32-bit
+  const int64_t k = kvz_keep_count(B_total * n_c, ratio);
+  return kvz::launch_select_dist_begin(S, B_local, n_c, k, hist, workspace, lay, d_status, stream) == cudaSuccess
+             ? KVZ_OK
+             : KVZ_ERR_CUDA;
+}
+
+kvz_status kvz_select_dist_step(const float* S, int64_t B_local, int64_t n_c, int pass, uint32_t* hist,
+                                uint64_t* eq_total, void* workspace, size_t workspace_bytes, int32_t* d_status,
+                                cudaStream_t stream) {
+  kvz::SelWorkspace lay;
+  const kvz_status st = dist_check(S, B_local, n_c, workspace, workspace_bytes, &lay);
+  if (st != KVZ_OK) return st;
+  if (pass < 0 || pass > 2 || hist == nullptr || (pass == 2 && eq_total == nullptr)) return KVZ_ERR_INVALID_ARG;
+  if (!aligned(hist, 16) || (eq_total != nullptr && !aligned(eq_total, 8))) return KVZ_ERR_ALIGNMENT;
+  return kvz::launch_select_dist_step(S, B_local, n_c, pass, hist,
+                                      reinterpret_cast<unsigned long long*>(eq_total), workspace, lay, d_status,
+                                      stream) == cudaSuccess
+             ? KVZ_OK
+             : KVZ_ERR_CUDA;
+}
+
+kvz_status kvz_select_dist_finish(const float* S, int64_t B_local, int64_t n_c, int64_t B_total, double ratio,
+                                  const uint64_t* eq_ranks, int rank, int32_t* idx, int64_t idx_capacity,
+                                  int32_t* counts, int64_t* offsets, void* workspace, size_t workspace_bytes,
+                                  int32_t* d_status, cudaStream_t stream) {
+  kvz::SelWorkspace lay;
+  const kvz_status st = dist_check(S, B_local, n_c, workspace, workspace_bytes, &lay);
+  if (st != KVZ_OK) return st;
+  if (eq_ranks == nullptr || counts == nullptr || offsets == nullptr || rank < 0) return KVZ_ERR_INVALID_ARG;
+  if (B_total < B_local || !(ratio >= 0.0 && ratio <= 1.0)) return KVZ_ERR_INVALID_ARG;
+  if (B_total * n_c >= (int64_t(1) << 32)) return KVZ_ERR_INVALID_ARG;   // histogram bins are 32-bit
+  if (!aligned(eq_ranks, 8) || !aligned(counts, 4) || !aligned(offsets, 8) || (idx && !aligned(idx, 4)))
+    return KVZ_ERR_ALIGNMENT;
+  const int64_t k = kvz_keep_count(B_total * n_c, ratio);
+  const int64_t need = k < B_local * n_c ? k : B_local * n_c;
+  if (idx_capacity < need || (need > 0 && idx == nullptr)) return KVZ_ERR_INVALID_ARG;
+  (void)d_status;
+  return kvz::launch_select_dist_finish(S, B_local, n_c, reinterpret_cast<const unsigned long long*>(eq_ranks),
+                                        rank, idx, counts, offsets, workspace, lay, stream) == cudaSuccess
+             ? KVZ_OK
+             : KVZ_ERR_CUDA;
+}
+
 kvz_status kvz_select_protected(const float* S, int64_t B, int64_t n_c, double ratio, int mode, int64_t n_protect,
                                 int32_t* idx, int64_t idx_capacity, int32_t* counts, int64_t* offsets,
                                 void* workspace, size_t workspace_bytes, int32_t* d_status, cudaStream_t stream) {

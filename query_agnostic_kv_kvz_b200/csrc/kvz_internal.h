@@ -109,6 +109,14 @@ SelWorkspace select_workspace(int64_t B, int64_t n_c, int mode);
 cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int64_t n_protect, int mode, int64_t k,
                           int32_t* idx, int32_t* counts, int64_t* offsets, void* ws, const SelWorkspace& lay,
                           int32_t* status, cudaStream_t stream);
+cudaError_t launch_select_dist_begin(const float* S, int64_t B, int64_t n_c, int64_t k, uint32_t* hist, void* ws,
+                                     const SelWorkspace& lay, int32_t* status, cudaStream_t stream);
+cudaError_t launch_select_dist_step(const float* S, int64_t B, int64_t n_c, int pass, uint32_t* hist,
+                                    unsigned long long* eq_total, void* ws, const SelWorkspace& lay,
+                                    int32_t* status, cudaStream_t stream);
+cudaError_t launch_select_dist_finish(const float* S, int64_t B, int64_t n_c, const unsigned long long* eq_ranks,
+                                      int rank, int32_t* idx, int32_t* counts, int64_t* offsets, void* ws,
+                                      const SelWorkspace& lay, cudaStream_t stream);
 
 // Compaction.
 cudaError_t launch_compact_gather(const void* K, const void* V, int64_t B, int64_t n_c, int d,

@@ -203,7 +203,8 @@ __global__ void __launch_bounds__(1024) sel_scan(int64_t B, int nchunk, int mode
                                                  const uint32_t* cg, const uint32_t* ce,
                                                  unsigned long long* eqb, uint32_t* cbase,
                                                  unsigned long long* head_eq, unsigned long long* head_base,
-                                                 int32_t* counts, int64_t* offsets) {
+                                                 int32_t* counts, int64_t* offsets,
+                                                 const unsigned long long* eq_ranks, int rank) {
   __shared__ unsigned long long wbuf[32];
   __shared__ unsigned long long carry;
   // 1. equal keys before each chunk, within its head
@@ -217,8 +218,14 @@ __global__ void __launch_bounds__(1024) sel_scan(int64_t B, int nchunk, int mode
     head_eq[b] = run;
   }
   __syncthreads();
-  // 2. equal keys in earlier heads (global mode: one segment spans all heads)
-  if (threadIdx.x == 0) carry = 0ull;
+  // 2. equal keys in earlier heads (global mode: one segment spans all heads,
+  //    and with the heads split over ranks, those of lower ranks come first)
+  if (threadIdx.x == 0) {
+    unsigned long long lower = 0ull;
+    if (eq_ranks != nullptr)
+      for (int r = 0; r < rank; ++r) lower += eq_ranks[r];
+    carry = lower;
+  }
   __syncthreads();
   for (int64_t t0 = 0; t0 < B; t0 += blockDim.x) {
     const int64_t b = t0 + threadIdx.x;
@@ -309,6 +316,15 @@ __global__ void __launch_bounds__(kSelThreads) sel_write(const float* S, int64_t
   for (int it = 0; it < kSelItems; ++it) {
     if (keep_bits & (1u << it)) idx[pos++] = static_cast<int32_t>(c0 + l0 + it);
   }
+}
+
+// Single CTA: the number of keys equal to T over all chunks of all heads.
+__global__ void __launch_bounds__(1024) sel_eq_total(const uint32_t* ce, int64_t nx, unsigned long long* out) {
+  __shared__ unsigned long long wbuf[32];
+  unsigned long long v = 0ull;
+  for (int64_t i = threadIdx.x; i < nx; i += blockDim.x) v += ce[i];
+  const unsigned long long incl = block_inclusive_sum<unsigned long long>(v, wbuf);
+  if (threadIdx.x == blockDim.x - 1) *out = incl;
 }
 
 // Per-head mode, one CTA per head: the same radix select and stable write as
@@ -490,8 +506,69 @@ cudaError_t launch_select(const float* S, int64_t B, int64_t n_c, int64_t n_prot
     sel_pick<<<nseg, 1024, 0, stream>>>(pass, st, hist);
   }
   sel_count<<<grid, kSelThreads, 0, stream>>>(S, n_c, n_protect, mode, nchunk, st, cg, ce);
-  sel_scan<<<1, 1024, 0, stream>>>(B, nchunk, mode, st, cg, ce, eqb, cbase, head_eq, head_base, counts, offsets);
+  sel_scan<<<1, 1024, 0, stream>>>(B, nchunk, mode, st, cg, ce, eqb, cbase, head_eq, head_base, counts, offsets,
+                                   nullptr, 0);
   sel_write<<<grid, kSelThreads, 0, stream>>>(S, n_c, n_protect, mode, nchunk, st, eqb, cbase, offsets, idx);
+  return cudaGetLastError();
+}
+
+// Global selection with the heads of one context split over ranks (rank r
+// holds a contiguous range of heads, lower ranks first).  The kernels are
+// those of launch_select in global mode; between the steps the caller sums
+// `hist` over ranks (three times) and gathers every rank's equal-key total.
+namespace {
+struct DistPtrs {
+  SelState* st;
+  uint32_t *cg, *ce, *cbase;
+  unsigned long long *eqb, *head_eq, *head_base;
+};
+DistPtrs dist_ptrs(void* ws, const SelWorkspace& lay) {
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  return DistPtrs{reinterpret_cast<SelState*>(base + lay.off_state),
+                  reinterpret_cast<uint32_t*>(base + lay.off_cg),
+                  reinterpret_cast<uint32_t*>(base + lay.off_ce),
+                  reinterpret_cast<uint32_t*>(base + lay.off_cbase),
+                  reinterpret_cast<unsigned long long*>(base + lay.off_eqb),
+                  reinterpret_cast<unsigned long long*>(base + lay.off_head_eq),
+                  reinterpret_cast<unsigned long long*>(base + lay.off_head_base)};
+}
+}  // namespace
+
+cudaError_t launch_select_dist_begin(const float* S, int64_t B, int64_t n_c, int64_t k, uint32_t* hist, void* ws,
+                                     const SelWorkspace& lay, int32_t* status, cudaStream_t stream) {
+  const DistPtrs w = dist_ptrs(ws, lay);
+  const int nchunk = static_cast<int>((n_c + kSelChunk - 1) / kSelChunk);
+  const dim3 grid(static_cast<unsigned>(nchunk), static_cast<unsigned>(B));
+  sel_init<<<8, 256, 0, stream>>>(w.st, 1, static_cast<unsigned long long>(k), hist);
+  sel_hist<<<grid, kSelThreads, 0, stream>>>(S, n_c, 0, KVZ_GLOBAL, 0, w.st, hist, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_dist_step(const float* S, int64_t B, int64_t n_c, int pass, uint32_t* hist,
+                                    unsigned long long* eq_total, void* ws, const SelWorkspace& lay,
+                                    int32_t* status, cudaStream_t stream) {
+  const DistPtrs w = dist_ptrs(ws, lay);
+  const int nchunk = static_cast<int>((n_c + kSelChunk - 1) / kSelChunk);
+  const dim3 grid(static_cast<unsigned>(nchunk), static_cast<unsigned>(B));
+  sel_pick<<<1, 1024, 0, stream>>>(pass, w.st, hist);
+  if (pass < 2) {
+    sel_hist<<<grid, kSelThreads, 0, stream>>>(S, n_c, 0, KVZ_GLOBAL, pass + 1, w.st, hist, status);
+  } else {
+    sel_count<<<grid, kSelThreads, 0, stream>>>(S, n_c, 0, KVZ_GLOBAL, nchunk, w.st, w.cg, w.ce);
+    sel_eq_total<<<1, 1024, 0, stream>>>(w.ce, B * nchunk, eq_total);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_dist_finish(const float* S, int64_t B, int64_t n_c, const unsigned long long* eq_ranks,
+                                      int rank, int32_t* idx, int32_t* counts, int64_t* offsets, void* ws,
+                                      const SelWorkspace& lay, cudaStream_t stream) {
+  const DistPtrs w = dist_ptrs(ws, lay);
+  const int nchunk = static_cast<int>((n_c + kSelChunk - 1) / kSelChunk);
+  const dim3 grid(static_cast<unsigned>(nchunk), static_cast<unsigned>(B));
+  sel_scan<<<1, 1024, 0, stream>>>(B, nchunk, KVZ_GLOBAL, w.st, w.cg, w.ce, w.eqb, w.cbase, w.head_eq,
+                                   w.head_base, counts, offsets, eq_ranks, rank);
+  sel_write<<<grid, kSelThreads, 0, stream>>>(S, n_c, 0, KVZ_GLOBAL, nchunk, w.st, w.eqb, w.cbase, offsets, idx);
   return cudaGetLastError();
 }
 

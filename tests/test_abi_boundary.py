@@ -248,3 +248,43 @@ def test_protect_and_int8_rejections(lib):
                                                  vp(Vq), vp(Ks), vp(Vs), None, None)
     assert q8(d_=96) == UNSUPPORTED
     assert q8(kq=Kq + 8) == ALIGN
+
+
+def test_select_dist_rejections(lib):
+    b = Bufs()
+    B, n_c, B_total = 3, 1000, 8
+    S = b.get(B * n_c * 4)
+    hist, eq, eqr = b.get(2048 * 4), b.get(16), b.get(8 * 8)
+    idx, cnt, off = b.get(B * n_c * 4), b.get(B * 4), b.get((B + 1) * 8)
+    ws_n = lib.kvz_select_dist_workspace_size(B, n_c)
+    assert ws_n > 0 and lib.kvz_select_dist_workspace_size(0, n_c) == 0
+    ws = b.get(ws_n)
+
+    def begin(Bt=B_total, ratio=0.3, h=hist, wsb=ws_n, s=S):
+        return lib.kvz_select_dist_begin(vp(s), B, n_c, Bt, ratio, vp(h) if h else None, vp(ws), wsb, None, None)
+
+    def step(p=0, h=hist, e=eq, wsb=ws_n):
+        return lib.kvz_select_dist_step(vp(S), B, n_c, p, vp(h) if h else None, vp(e) if e else None, vp(ws), wsb,
+                                        None, None)
+
+    def finish(Bt=B_total, ratio=0.3, er=eqr, rank=1, cap=B * n_c, wsb=ws_n):
+        return lib.kvz_select_dist_finish(vp(S), B, n_c, Bt, ratio, vp(er) if er else None, rank, vp(idx), cap,
+                                          vp(cnt), vp(off), vp(ws), wsb, None, None)
+
+    assert begin(Bt=B - 1) == INVALID                 # fewer heads in all than on this rank
+    assert begin(ratio=1.01) == INVALID
+    assert begin(h=None) == INVALID
+    assert begin(h=hist + 4) == ALIGN
+    assert begin(wsb=ws_n - 1) == WS
+    assert begin(s=S + 2) == ALIGN
+    assert begin(Bt=(1 << 32) // n_c + 1) == INVALID  # 32-bit histogram bins
+    assert step(p=3) == INVALID
+    assert step(p=-1) == INVALID
+    assert step(p=2, e=None) == INVALID               # the last step writes the equal-key total
+    assert step(h=None) == INVALID
+    assert step(e=eq + 4) == ALIGN
+    assert finish(er=None) == INVALID
+    assert finish(rank=-1) == INVALID
+    assert finish(cap=int(0.3 * B_total * n_c) - 1) == INVALID   # min(k, B*n_c) = 2400 slots needed
+    assert finish(er=eqr + 4) == ALIGN
+    assert finish(wsb=0) == WS

@@ -55,3 +55,135 @@ def test_two_ranks_shard_and_reduce():
     assert (r0[0], r0[1], r1[0], r1[1]) == (0, 128, 128, 256)        # disjoint halves
     assert r0[2] != r1[2]                                             # independent seeds
     assert r0[3:] == r1[3:] == [2.0, 10.0, 128.0]                     # max over ranks
+
+
+# ---------------------------------------------------------------------------
+# Sharded global selection: the host orchestration (three histogram
+# all-reduces, one all-gather of equal-key totals) driven over gloo with a
+# NumPy restatement of the device steps, checked against the oracle's
+# global selection over all heads (a stable sort, not a radix select).
+# ---------------------------------------------------------------------------
+import numpy as np  # noqa: E402
+
+from oracle import kvz_oracle as orc  # noqa: E402
+from query_agnostic_kv_kvz_b200.dist import select_global_sharded  # noqa: E402
+
+_SHIFT = (21, 10, 0)
+_MASK = (0x7FF, 0x7FF, 0x3FF)
+
+
+class NumpySelectSteps:
+    """The three-digit radix select of the library's step calls, on the
+    CPU: digit histograms over keys that match the prefix fixed so far, the
+    pick of the digit that holds the k_rem-th largest key, then the keys
+    above the threshold T plus the first r_t keys equal to it in flattened
+    order, counting those of lower ranks first."""
+
+    def buffers(self, S):
+        return {"hist": torch.zeros(2048, dtype=torch.int32), "eq_total": torch.zeros(1, dtype=torch.int64),
+                "state": {}}
+
+    @staticmethod
+    def _keys(S):
+        u = S.numpy().astype(np.float32).view(np.uint32).copy()
+        u[u == 0x80000000] = 0
+        return u
+
+    def _hist(self, keys, st, p):
+        match = (keys & st["mask"]) == st["prefix"]
+        d = (keys[match] >> _SHIFT[p]) & _MASK[p]
+        return np.bincount(d.astype(np.int64), minlength=2048).astype(np.int32)
+
+    def begin(self, S, B_total, ratio, buf, status):
+        keys = self._keys(S).reshape(-1)
+        k = orc.keep_count(B_total * S.shape[1], ratio)
+        st = buf["state"]
+        st.update(prefix=np.uint32(0), mask=np.uint32(0), k_rem=k, keys=keys)
+        buf["hist"][:] = torch.from_numpy(self._hist(keys, st, 0) if k > 0 else np.zeros(2048, np.int32))
+
+    def step(self, S, p, buf, status):
+        st = buf["state"]
+        keys = st["keys"]
+        if st["k_rem"] > 0 and not st.get("done"):
+            h = buf["hist"].numpy().astype(np.int64)
+            nb = 1024 if p == 2 else 2048
+            above = 0
+            for digit in range(nb - 1, -1, -1):          # highest digit first
+                if above + h[digit] >= st["k_rem"]:
+                    break
+                above += h[digit]
+            st["prefix"] = np.uint32(st["prefix"] | (digit << _SHIFT[p]))
+            st["mask"] = np.uint32(st["mask"] | (_MASK[p] << _SHIFT[p]))
+            st["k_rem"] -= above
+        else:
+            st["done"] = True
+        buf["hist"].zero_()
+        if p < 2:
+            if not st.get("done"):
+                buf["hist"][:] = torch.from_numpy(self._hist(keys, st, p + 1))
+        else:
+            buf["eq_total"][0] = 0 if st.get("done") else int(np.count_nonzero(keys == st["prefix"]))
+
+    def finish(self, S, B_total, ratio, eq_ranks, rank, buf, status):
+        st = buf["state"]
+        B, n_c = S.shape
+        keys = st["keys"].reshape(B, n_c)
+        per_head = []
+        if st.get("done"):
+            per_head = [np.zeros(0, np.int64) for _ in range(B)]
+        else:
+            T, r_t = st["prefix"], st["k_rem"]
+            e = int(eq_ranks[:rank].sum())
+            for b in range(B):
+                kept = []
+                for j in range(n_c):
+                    if keys[b, j] > T:
+                        kept.append(j)
+                    elif keys[b, j] == T:
+                        if e < r_t:
+                            kept.append(j)
+                        e += 1
+                per_head.append(np.array(kept, np.int64))
+        counts = np.array([len(x) for x in per_head], np.int32)
+        offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+        idx = np.concatenate(per_head).astype(np.int32) if counts.sum() else np.zeros(0, np.int32)
+        return torch.from_numpy(idx), torch.from_numpy(counts), torch.from_numpy(offsets)
+
+
+def _tie_scores(B, n_c, seed):
+    """Scores with many exact ties (few distinct values), zeros and +inf."""
+    rng = np.random.default_rng(seed)
+    S = rng.choice(np.float32([0.0, 0.125, 0.25, 0.5, 1.0, 3.0]), size=(B, n_c)).astype(np.float32)
+    S[rng.random((B, n_c)) < 0.3] = rng.random(int((rng.random((B, n_c)) < 0.3).sum()) or 1)[0]
+    S[0, :3] = np.inf
+    return S
+
+
+def _sel_worker(rank, world, port, splits, B, n_c, ratio, seed, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        S = torch.from_numpy(_tie_scores(B, n_c, seed))
+        lo, hi = splits[rank], splits[rank + 1]
+        idx, counts, offsets = select_global_sharded(S[lo:hi].contiguous(), ratio, steps=NumpySelectSteps())
+        # this rank's (head, position) pairs, in global head numbering
+        pairs = [(lo + b, int(j)) for b in range(hi - lo) for j in idx[offsets[b]:offsets[b + 1]].tolist()]
+        out[rank] = pairs
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,splits,ratio", [(2, [0, 3, 8], 0.3), (3, [0, 1, 1, 5], 0.55), (2, [0, 4, 5], 0.0)])
+def test_sharded_global_select_matches_oracle(world, splits, ratio):
+    B, n_c, seed = splits[-1], 300, world * 7 + len(splits)
+    port = _free_port()
+    mgr = tmp.Manager()
+    out = mgr.dict()
+    tmp.spawn(_sel_worker, args=(world, port, splits, B, n_c, ratio, seed, out), nprocs=world, join=True)
+    got = sorted(p for r in range(world) for p in out[r])
+    ridx, rcounts, roffsets = orc.select(_tie_scores(B, n_c, seed), ratio, "global")
+    want = sorted((b, int(j)) for b in range(B) for j in ridx[roffsets[b]:roffsets[b + 1]])
+    assert got == want
+    assert len(want) == orc.keep_count(B * n_c, ratio)
