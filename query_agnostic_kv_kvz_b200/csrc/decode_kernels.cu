@@ -4,10 +4,13 @@
 // new token:  out[b, g] = sum_j softmax_j(scale * <q_g, k_j>) v_j.
 //
 // HBM-bound: each step reads every kept key and value once (4*d bytes per
-// kept row).  Split-KV: a CTA takes a contiguous run of 64-key tiles of one
-// head, brought in by TMA (three-stage ring, 128-byte swizzle, read back with
-// ldmatrix), keeps a running (max, sum, output) per query and writes it as a
-// partial; the CTA that finishes a head's last split merges its partials.
+// kept row).  Split-KV over a work list that a one-CTA plan kernel builds
+// from the counts, with the same number of 64-key tiles in every split of
+// every head.  A CTA takes one split, brings its tiles in by TMA (three-stage
+// ring, 128-byte swizzle, read back with ldmatrix), keeps a running (max,
+// sum, output) per query and writes it as a partial; the partials of a head
+// merge in a two-level tree (the last CTA of each group of 16 splits, then
+// the last group merger).
 #include <cuda.h>
 #include <cuda_runtime.h>
 

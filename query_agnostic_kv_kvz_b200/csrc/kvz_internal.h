@@ -62,7 +62,8 @@ cudaError_t launch_colmax(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc
                           cudaStream_t stream);
 cudaError_t launch_fill_f32(float* x, int64_t n, float v, cudaStream_t stream);
 
-// Decode attention over the pruned cache (split-KV partials + combine).
+// Decode attention over the pruned cache (a device-built work list of equal
+// splits; split-KV partials merged by a two-level tree).
 constexpr int kDecGMax = 8;                 // grouped queries per KV head
 // One CTA of the decode kernel: split sp of head b, tiles t0 .. t0+n-1 of
 // the head's 64-key tiles; its partial is written at the item's index, the
