@@ -209,11 +209,12 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        torch.cuda.set_device(local)
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    dev = torch.device("cuda", local if world > 1 else 0)
-    torch.cuda.set_device(dev)
+        if args.impl == "reference":                      # the host oracle: no GPU, a CPU process group
+            dist.init_process_group("gloo", timeout=timedelta(seconds=120))
+        else:
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timedelta(seconds=120))
 
     from query_agnostic_kv_kvz_b200 import synth
     w = synth.WORKLOADS[args.workload]
@@ -238,7 +239,9 @@ def main():
                 dist.destroy_process_group()
             return
         x = synth.layer_inputs(w, seed=rank, device="cpu")
-        steps, warm = max(1, args.steps if args.steps < 3 else 3), 0
+        steps, warm = max(1, args.steps if args.steps < 3 else 3), max(0, min(args.warmup, 3))
+        for s in range(warm):                              # untimed, like the GPU arm's warm-up steps
+            oracle_head_time(x, w, s % w.B)
         times = []
         threads = 1
         for s in range(steps):
@@ -259,6 +262,8 @@ def main():
             dist.destroy_process_group()
         return
 
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
     import query_agnostic_kv_kvz_b200 as kvz
     from query_agnostic_kv_kvz_b200.dist import max_over_ranks, rank_seed
     kvz.lib()
