@@ -187,3 +187,15 @@ def test_sharded_global_select_matches_oracle(world, splits, ratio):
     want = sorted((b, int(j)) for b in range(B) for j in ridx[roffsets[b]:roffsets[b + 1]])
     assert got == want
     assert len(want) == orc.keep_count(B * n_c, ratio)
+
+
+def test_sharded_global_select_without_a_process_group():
+    # one process, no process group: the driver's exchanges reduce to
+    # identities and the result is the oracle's global selection
+    B, n_c, ratio = 4, 257, 0.4
+    S = _tie_scores(B, n_c, seed=11)
+    idx, counts, offsets = select_global_sharded(torch.from_numpy(S), ratio, steps=NumpySelectSteps())
+    ridx, rcounts, roffsets = orc.select(S, ratio, "global")
+    assert counts.tolist() == rcounts.tolist()
+    assert offsets.tolist() == roffsets.tolist()
+    assert idx.tolist() == ridx.tolist()
