@@ -142,6 +142,34 @@ def test_rows_normalise_and_lse_matches_textbook():
             assert abs(np.exp(z - lse).sum() - 1.0) <= 1e-12
 
 
+@pytest.mark.parametrize("seed,G,n_c,n_in,d,sc", [(40, 2, 5, 4, 3, 0.7), (41, 1, 9, 6, 8, 1.0 / math.sqrt(8)),
+                                                  (42, 3, 1, 3, 2, 1.3)])
+def test_row_logits_and_lse_match_brute_force_and_score(seed, G, n_c, n_in, d, sc):
+    # The per-row helpers check every lse2 the kernels write, so they are
+    # pinned to a 50-digit evaluation of the definition (logits scale*<q,k_u>
+    # over the causal key range u < n_c + i + 1, and the log of the softmax
+    # denominator) and, through the softmax they define, to score() itself:
+    # max over (g, i) of exp(z[:n_c] - lse) must be the oracle's S.
+    rng = np.random.default_rng(seed)
+    Q, K_ctx, K_in = _rand_head(rng, G, n_c, n_in, d, scale_keys=2.0)
+    mpmath.mp.dps = 50
+    keys = [list(map(mpmath.mpf, k)) for k in np.concatenate([K_ctx, K_in])]
+    msc = mpmath.mpf(sc)
+    S_rows = np.zeros(n_c)
+    for g in range(G):
+        for i in range(n_in):
+            q = list(map(mpmath.mpf, Q[g, i]))
+            z_mp = [msc * mpmath.fsum(a * b for a, b in zip(q, keys[u])) for u in range(n_c + i + 1)]
+            lse_mp = mpmath.log(mpmath.fsum(mpmath.e ** z for z in z_mp))
+            z = orc.row_logits(Q[g, i], K_ctx, K_in, i, sc)
+            assert z.shape == (n_c + i + 1,)
+            np.testing.assert_allclose(z, [float(v) for v in z_mp], rtol=1e-14, atol=1e-15)
+            lse = orc.row_lse(Q[g, i], K_ctx, K_in, i, sc)
+            assert abs(lse - float(lse_mp)) <= 1e-13 * max(1.0, abs(float(lse_mp)))
+            S_rows = np.maximum(S_rows, np.exp(z[:n_c] - lse))
+    np.testing.assert_allclose(S_rows, orc.score(Q, K_ctx, K_in, sc), rtol=1e-13, atol=0)
+
+
 def test_range_permutation_duplication_shift_chunks():
     rng = np.random.default_rng(6)
     G, n_c, n_in, d = 3, 50, 37, 16
