@@ -154,9 +154,11 @@ kvz_status kvz_score_colmax(const void* Q, const void* K_ctx,
 /* - Returns KVZ_ERR_WORKSPACE, launching nothing, when one 256-row block   */
 /*   of every head and group does not fit: B*G*256*4 > KVZ_NOALLOC_SCRATCH_ */
 /*   BYTES (B*G > 8192).  Other argument errors are those of kvz_score.     */
-/* - The first call on each device looks up the array's device address     */
-/*   (cudaGetSymbolAddress) with that device current; make that first call  */
-/*   before any stream capture that would contain a later one.              */
+/* - The first call in each CUDA context (a device's primary context, or a */
+/*   context the caller made current; a device reset makes a new one)      */
+/*   looks up the array's device address there (cudaGetSymbolAddress);     */
+/*   make that first call before any stream capture that would contain a   */
+/*   later one.                                                             */
 /* - Every call on a device uses the same array and leaves its contents     */
 /*   behind.  Nothing in it needs to start at zero (each call writes every  */
 /*   entry before reading it), but calls that overlap on the GPU (two       */

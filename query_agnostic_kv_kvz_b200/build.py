@@ -43,7 +43,7 @@ def _sources():
 
 def _deps():
     return _sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
-        [os.path.join(INCLUDE, "kvz.h")]
+        glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
 def up_to_date() -> bool:

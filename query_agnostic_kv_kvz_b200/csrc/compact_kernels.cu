@@ -46,7 +46,6 @@ static_assert(kInplaceThreads % 32 == 0, "whole warps");
 static_assert(kInplaceDepth >= 2, "a ring holds the chunk being stored and at least one loading");
 static_assert(kInplaceRows % 4 == 0, "a warp-wide access covers 2 (d = 128) or 4 (d = 64) rows");
 static_assert(kInplaceDepth * kInplaceRows / 2 <= 32, "one validity bit per row, lane and stage in 32 bits");
-constexpr uint64_t kWaitNs = 1000ull * 1000ull * 1000ull;   // 1 s: far beyond any legitimate wait
 
 __device__ __forceinline__ void report_err(int32_t* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
@@ -59,6 +58,19 @@ __device__ __forceinline__ int4 ld_stream(const int4* p) {
   asm volatile("ld.global.nc.L1::no_allocate.v4.s32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
+  return v;
+}
+
+// Coherent streaming load for the in-place kernel, which overwrites rows
+// that other warps of the same launch read: a relaxed gpu-scope load stays
+// inside the memory model the kernel's ordering argument rests on (the
+// read-only .nc path is only for data no thread of the launch writes).
+__device__ __forceinline__ int4 ld_coherent(const int4* p) {
+  int4 v;
+  asm volatile("ld.relaxed.gpu.global.L1::no_allocate.v4.s32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
   return v;
 }
 
@@ -428,14 +440,18 @@ __global__ void __launch_bounds__(256)
 // near chunk rho*c, long finished, so warps rarely wait.  A warp's current
 // chunk is its lowest unpublished one and waits only on lower chunks, so
 // the lowest unpublished chunk of a head always belongs to a warp whose
-// waits are satisfied: every wait ends.  No row is written before its
-// reader has loaded it, so the loads may take the read-only path.
+// waits are satisfied: every wait ends.  Rows are loaded coherently (they
+// are written later in the same launch).
+// `wait_ns` bounds every wait; publication of chunk `hold_c` of head
+// `hold_b` is skipped when both are >= 0 (only the test entry point sets
+// them, to make a wait expire; the normal call passes -1).
 template <int VPR>
 __global__ void __launch_bounds__(kInplaceThreads, kInplaceMinCtas)
     compact_inplace_kernel(int4* K, int4* V, int64_t B, int64_t n_c, int64_t warps_per_head,
                            const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
                            const int64_t* __restrict__ offsets, uint32_t* next_chunk, uint32_t* chunk_read,
-                           int64_t chunks_per_head, const uint32_t* lo_slot, int32_t* status) {
+                           int64_t chunks_per_head, const uint32_t* lo_slot, int32_t* status, uint64_t wait_ns,
+                           int64_t hold_b, int64_t hold_c) {
   constexpr int kRowsPerAccess = 32 / VPR;                    // rows one warp-wide access covers
   constexpr int NR = kInplaceRows / kRowsPerAccess;           // rows of a chunk each lane moves
   constexpr int D = kInplaceDepth;
@@ -478,8 +494,8 @@ __global__ void __launch_bounds__(kInplaceThreads, kInplaceMinCtas)
       if (c >= nchunks || p >= count) continue;
       const int64_t j = jn[k];
       if (j >= p && j < n_c) {
-        dk[st][k] = ld_stream(Xk + j * VPR + col);
-        dv[st][k] = ld_stream(Xv + j * VPR + col);
+        dk[st][k] = ld_coherent(Xk + j * VPR + col);
+        dv[st][k] = ld_coherent(Xv + j * VPR + col);
         bits |= 1u << k;
       } else {
         report_err(status, KVZ_ERR_INVALID_ARG);              // ascending idx guarantees p <= j < n_c
@@ -540,7 +556,7 @@ __global__ void __launch_bounds__(kInplaceThreads, kInplaceMinCtas)
         if (ld_relaxed_gpu(&flags[k]) == 32u) continue;
         const uint64_t t0 = now_ns();
         while (ld_relaxed_gpu(&flags[k]) != 32u) {
-          if (now_ns() - t0 > kWaitNs) {
+          if (now_ns() - t0 > wait_ns) {
             ok = 0;
             break;
           }
@@ -561,7 +577,8 @@ __global__ void __launch_bounds__(kInplaceThreads, kInplaceMinCtas)
         Xv[p * VPR + col] = dv[s][k];
         got |= static_cast<uint32_t>(dk[s][k].x) | static_cast<uint32_t>(dv[s][k].x);
       }
-      red_relaxed_gpu_add(&flags[cur], 1u + dep_zero(got));   // this lane's sources of cur are read
+      if (b != hold_b || static_cast<int64_t>(cur) != hold_c)
+        red_relaxed_gpu_add(&flags[cur], 1u + dep_zero(got));   // this lane's sources of cur are read
       const int sn = (s + D - 1) % D;                         // the stage written out last step
       issue(sn, cl[sn]);
       const uint32_t c_next = __shfl_sync(kFull, pend, 0);
@@ -630,7 +647,7 @@ size_t compact_workspace_bytes(int64_t B, int64_t n_c) {
 
 cudaError_t launch_compact_inplace(void* K, void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
                                    const int32_t* counts, const int64_t* offsets, uint32_t* ws, int32_t* status,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, uint64_t wait_ns, int64_t hold_b, int64_t hold_c) {
   const int64_t chunks = (n_c + kInplaceRows - 1) / kInplaceRows;
   // next_chunk[B] | chunk_read[B][chunks] | lo_slot[B][chunks + 1], all zeroed (all-zero bits)
   uint32_t* next_chunk = ws;
@@ -658,7 +675,7 @@ cudaError_t launch_compact_inplace(void* K, void* V, int64_t B, int64_t n_c, int
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
   kern<<<static_cast<unsigned>(grid), kInplaceThreads, 0, stream>>>(
       static_cast<int4*>(K), static_cast<int4*>(V), B, n_c, wph, idx, counts, offsets, next_chunk, chunk_read, chunks,
-      lo_slot, status);
+      lo_slot, status, wait_ns, hold_b, hold_c);
   return cudaGetLastError();
 }
 

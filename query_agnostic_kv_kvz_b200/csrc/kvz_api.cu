@@ -10,6 +10,7 @@
 
 #include "kvz.h"
 #include "kvz_internal.h"
+#include "kvz_testing.h"
 
 namespace {
 
@@ -293,27 +294,73 @@ kvz_status kvz_score_chunked(const void* Q, const void* Q_tail, const void* K_ct
 // ---------------------------------------------------------------------------
 // Allocation-free scoring: the lse2 scratch is this file-scope device array.
 // In host code its name only stands in for the symbol; the device address
-// comes from cudaGetSymbolAddress, once per device.
+// comes from cudaGetSymbolAddress, looked up once per CUDA context.
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) float kvz_noalloc_lse2[KVZ_NOALLOC_SCRATCH_BYTES / sizeof(float)];
 
 namespace {
 
-constexpr int kMaxDevices = 256;
-std::mutex g_noalloc_mu;
-float* g_noalloc_addr[kMaxDevices] = {};
-
-// Device address of the static scratch on the current device.
-kvz_status noalloc_scratch(float** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVZ_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+// Driver calls that name the current context by its process-unique id, so a
+// context created after a device reset, or a non-primary context a caller
+// made current, never reuses an address looked up in another context.
+struct CtxIdFns {
+  PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  PFN_cuCtxGetId_v12000 get_id = nullptr;
+};
+const CtxIdFns& ctx_id_fns() {
+  static CtxIdFns f;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, kvz_noalloc_lse2) != cudaSuccess || p == nullptr) return KVZ_ERR_CUDA;
-    g_noalloc_addr[dev] = static_cast<float*>(p);
-  }
-  *out = g_noalloc_addr[dev];
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  return f;
+}
+
+constexpr int kMaxContexts = 64;
+std::mutex g_noalloc_mu;
+unsigned long long g_noalloc_ctx[kMaxContexts] = {};   // context ids (0 = free slot)
+float* g_noalloc_addr[kMaxContexts] = {};
+int g_noalloc_next = 0;                                 // round-robin replacement when full
+
+// Process-unique id of the calling thread's current context (0 if none).
+unsigned long long current_ctx_id() {
+  const CtxIdFns& f = ctx_id_fns();
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (f.get_current == nullptr || f.get_id == nullptr || f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      f.get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the static scratch in the current context.  With no
+// context current yet, the symbol lookup itself initialises the current
+// device's primary context, and the id is read after it.
+kvz_status noalloc_scratch(float** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  unsigned long long id = current_ctx_id();
+  if (id != 0)
+    for (int i = 0; i < kMaxContexts; ++i)
+      if (g_noalloc_ctx[i] == id) {
+        *out = g_noalloc_addr[i];
+        return KVZ_OK;
+      }
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, kvz_noalloc_lse2) != cudaSuccess || p == nullptr) return KVZ_ERR_CUDA;
+  if (id == 0 && (id = current_ctx_id()) == 0) return KVZ_ERR_CUDA;
+  const int slot = g_noalloc_next;
+  g_noalloc_next = (g_noalloc_next + 1) % kMaxContexts;
+  g_noalloc_ctx[slot] = id;
+  g_noalloc_addr[slot] = static_cast<float*>(p);
+  *out = g_noalloc_addr[slot];
   return KVZ_OK;
 }
 
@@ -624,6 +671,28 @@ kvz_status kvz_compact(const void* K, const void* V, int64_t B, int64_t n_c, int
   }
   return kvz::launch_compact_gather(K, V, B, n_c, d, idx, offsets, out_offsets, K_out, V_out, d_status,
                                     stream) == cudaSuccess
+             ? KVZ_OK
+             : KVZ_ERR_CUDA;
+}
+
+kvz_status kvz_testing_compact_in_place_withhold(void* K, void* V, int64_t B, int64_t n_c, int d,
+                                                 const int32_t* idx, const int32_t* counts,
+                                                 const int64_t* offsets, void* workspace,
+                                                 size_t workspace_bytes, int64_t wait_ns, int64_t hold_head,
+                                                 int64_t hold_chunk, int32_t* d_status, cudaStream_t stream) {
+  if (K == nullptr || V == nullptr || counts == nullptr || offsets == nullptr || idx == nullptr)
+    return KVZ_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return KVZ_ERR_UNSUPPORTED;
+  if (B < 1 || B > 0x7FFFFFFF / 8 || n_c < 1 || n_c > kMaxRows || K == V) return KVZ_ERR_INVALID_ARG;
+  if (wait_ns < 1000 || wait_ns > 1000000000 || hold_head < 0 || hold_head >= B || hold_chunk < 0)
+    return KVZ_ERR_INVALID_ARG;
+  if (!aligned(K, 16) || !aligned(V, 16) || !aligned(idx, 4) || !aligned(counts, 4) || !aligned(offsets, 8))
+    return KVZ_ERR_ALIGNMENT;
+  if (workspace == nullptr || workspace_bytes < kvz::compact_workspace_bytes(B, n_c)) return KVZ_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return KVZ_ERR_ALIGNMENT;
+  return kvz::launch_compact_inplace(K, V, B, n_c, d, idx, counts, offsets, static_cast<uint32_t*>(workspace),
+                                     d_status, stream, static_cast<uint64_t>(wait_ns), hold_head,
+                                     hold_chunk) == cudaSuccess
              ? KVZ_OK
              : KVZ_ERR_CUDA;
 }

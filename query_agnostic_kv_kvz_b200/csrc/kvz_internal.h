@@ -125,9 +125,14 @@ cudaError_t launch_compact_gather(const void* K, const void* V, int64_t B, int64
                                   void* K_out, void* V_out, int32_t* status, cudaStream_t stream);
 // In place: `ws` holds B + B*ceil(n_c/chunk) uint32 (per-head chunk claims and
 // per-chunk "sources read" flags); the launcher zeroes it on `stream`.
+// `wait_ns` bounds each ordering wait (kInplaceWaitNs normally); when hold_b
+// and hold_c are both >= 0, chunk hold_c of head hold_b never publishes that
+// its sources were read, so a chunk waiting on it times out (test use only).
+constexpr uint64_t kInplaceWaitNs = 1000ull * 1000ull * 1000ull;   // 1 s: far beyond any legitimate wait
 cudaError_t launch_compact_inplace(void* K, void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,
                                    const int32_t* counts, const int64_t* offsets, uint32_t* ws, int32_t* status,
-                                   cudaStream_t stream);
+                                   cudaStream_t stream, uint64_t wait_ns = kInplaceWaitNs, int64_t hold_b = -1,
+                                   int64_t hold_c = -1);
 size_t compact_workspace_bytes(int64_t B, int64_t n_c);
 // Out-of-place compaction into int8 codes with one fp32 scale per row.
 cudaError_t launch_compact_int8(const void* K, const void* V, int64_t B, int64_t n_c, int d, const int32_t* idx,

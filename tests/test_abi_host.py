@@ -1,7 +1,8 @@
 """Host-side checks of the C ABI (no GPU): the library builds, loads, exports
-every function include/kvz.h declares, and its host-only helpers agree with
+every function include/*.h declares, and its host-only helpers agree with
 the definitions (keep count, workspace sizing, status strings)."""
 import ctypes
+import glob
 import os
 import re
 
@@ -12,6 +13,7 @@ from oracle import kvz_oracle as orc
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "kvz.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 @pytest.fixture(scope="module")
@@ -24,7 +26,7 @@ def kvz():
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    text = "\n".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(kvz_[a-z0-9_]+)\s*\(", text)))
 
