@@ -3,6 +3,8 @@ score tolerance, and a spawn-based process pool for per-head oracle runs."""
 import math
 import multiprocessing as mp
 import os
+import shutil
+import tempfile
 from concurrent.futures import ProcessPoolExecutor
 
 import numpy as np
@@ -71,3 +73,60 @@ def oracle_scores(Q, K_ctx, K_in, scale, heads=None):
     if len(jobs) == 1 or Q.shape[2] * K_ctx.shape[1] < 4_000_000:
         return np.stack([_score_one(j) for j in jobs])
     return np.stack(list(pool().map(_score_one, jobs)))
+
+
+# ---------------------------------------------------------------------------
+# Whole heads at full size: the oracle's rows split over worker processes.
+# Each job is oracle.score(..., rows=(r0, r1)), the max over that row range
+# (every row still normalised over all the keys it sees); the ranges' maxima
+# merge exactly by np.maximum, which the oracle's own pins cover.
+# ---------------------------------------------------------------------------
+_HEAD_CACHE = {}
+
+
+def _rows_job(args):
+    qp, kcp, kip, scale, r0, r1, row_block = args
+    from threadpoolctl import threadpool_limits
+    key = (qp, kcp, kip)
+    if key not in _HEAD_CACHE:
+        _HEAD_CACHE.clear()
+        _HEAD_CACHE[key] = tuple(orc.bf16_bits_to_f64(np.load(p)) for p in key)
+    Q, Kc, Ki = _HEAD_CACHE[key]
+    with threadpool_limits(1):
+        return orc.score(Q, Kc, Ki, scale, rows=(r0, r1), row_block=row_block)
+
+
+_ROW_POOL = None
+
+
+def row_pool():
+    """Spawned workers for row-split oracle heads: one per core (at most 32),
+    fewer if host memory is short (up to 4 GB each at the 128K shapes)."""
+    global _ROW_POOL
+    if _ROW_POOL is None:
+        n = min(32, os.cpu_count() or 1)
+        try:
+            import psutil
+            n = max(1, min(n, int(psutil.virtual_memory().available / (4 << 30))))
+        except Exception:
+            pass
+        _ROW_POOL = ProcessPoolExecutor(max_workers=n, mp_context=mp.get_context("spawn"))
+    return _ROW_POOL
+
+
+def oracle_head_rows_parallel(Q_head, Kc_head, Ki_head, scale, rows_per_job=256, row_block=64):
+    """Oracle S [n_c] of ONE head from torch bf16 Q [G, n_in, d], K_ctx
+    [n_c, d], K_in [n_in, d], its input rows split over row_pool()."""
+    tmp = tempfile.mkdtemp(prefix="kvz_oracle_", dir="/dev/shm" if os.path.isdir("/dev/shm") else None)
+    try:
+        paths = []
+        for name, t in (("q", Q_head), ("kc", Kc_head), ("ki", Ki_head)):
+            path = os.path.join(tmp, name + ".npy")
+            np.save(path, bits(t))
+            paths.append(path)
+        n_in = Q_head.shape[1]
+        jobs = [(*paths, float(scale), r0, min(n_in, r0 + rows_per_job), row_block)
+                for r0 in range(0, n_in, rows_per_job)]
+        return np.maximum.reduce(list(row_pool().map(_rows_job, jobs)))
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)

@@ -75,7 +75,8 @@ def test_sharded_steps_equal_global_select(splits, n_c, ratio):
         assert torch.equal(off, roff[lo:hi + 1] - roff[lo])
         n = int(off[-1].item())
         assert torch.equal(idx[:n], ridx[int(roff[lo].item()):int(roff[hi].item())])
-    if B * n_c <= 200000:
-        oidx, ocnt, ooff = orc.select(S.cpu().numpy(), ratio, "global")
-        np.testing.assert_array_equal(rcnt.cpu().numpy(), ocnt)
-        np.testing.assert_array_equal(ridx[:int(roff[-1].item())].cpu().numpy(), oidx)
+    # every case, sharded or not, is also the oracle's stable-sort selection
+    oidx, ocnt, ooff = orc.select(S.cpu().numpy(), ratio, "global")
+    np.testing.assert_array_equal(rcnt.cpu().numpy(), ocnt)
+    np.testing.assert_array_equal(roff.cpu().numpy(), ooff)
+    np.testing.assert_array_equal(ridx[:int(roff[-1].item())].cpu().numpy(), oidx)

@@ -3,11 +3,14 @@ oracle where it can run and by properties that hold at any size elsewhere:
 
 * every workload: selection bit-exact against the oracle's stable sort on the
   GPU's own scores (all heads); compaction bit-exact on sampled heads;
+* whole seeded heads: every score of the head against the oracle, both
+  bounds of the tolerance (the oracle's input rows split over worker
+  processes): two heads of the 32K stack, layer 0 head 1 of the 128K config,
+  one head of each longer context of the ragged batch, and every head of
+  two layers of its 1000-key context;
 * pass 1 (lse2) against the oracle on sampled rows of sampled heads;
 * S[j] >= A[r, j] for every key j and every sampled row r (oracle rows);
-* planted dominant keys: S[j*] equals one oracle row value A[r*, j*];
-* the 1000-key context of the ragged batch: every score of every head
-  against the oracle.
+* planted dominant keys: S[j*] equals one oracle row value A[r*, j*].
 """
 import math
 
@@ -15,7 +18,8 @@ import numpy as np
 import pytest
 import torch
 
-from kvz_testutil import ABS_TOL, REL_FLOOR, REL_TOL, assert_scores_close, bits, f32_scale, f64, oracle_scores
+from kvz_testutil import (ABS_TOL, REL_FLOOR, REL_TOL, assert_scores_close, bits, f32_scale, f64,
+                          oracle_head_rows_parallel, oracle_scores)
 from oracle import kvz_oracle as orc
 from query_agnostic_kv_kvz_b200 import synth
 
@@ -134,6 +138,14 @@ def check_sampled_rows(r, w, layer, head, rows, groups):
                     assert (gap[big] / A[big]).max() <= REL_TOL
 
 
+def check_whole_head(r, w, layer, head):
+    """Every score of head (layer, head) against the oracle, two-sided."""
+    x = r["kept"][layer]
+    ref = oracle_head_rows_parallel(x["Q"][head], x["K_ctx"][head], x["K_in"][head], r["scale"])
+    b = layer * w.H + head
+    assert_scores_close(r["S"][b].cpu().numpy(), ref, "%s layer %d head %d" % (w.name, layer, head))
+
+
 def planter(rows_keys, alpha=1.8):
     """Make context key j of head 0 an enlarged copy of query row (g, i)."""
     def plant(x):
@@ -162,6 +174,8 @@ def test_llama8b_stack_32k_global():
     check_planted(r, plant)
     sel = check_selection(r, w)
     check_compaction(r, sel, heads=[0, 7, 100, 255], in_place=False)
+    check_whole_head(r, w, layer=0, head=3)
+    check_whole_head(r, w, layer=31, head=7)
     rows = sampled_rows(r["n_in"], w.n_prompt, rng)
     check_sampled_rows(r, w, layer=0, head=3, rows=rows, groups=[0, 3])
     check_sampled_rows(r, w, layer=31, head=7, rows=rows, groups=[1])
@@ -174,6 +188,7 @@ def test_qwen14b_128k_row_chunks_in_place():
     r = run_path(w, keep_layers=(0, 47), plant=planter(plant))
     check_planted(r, plant)
     sel = check_selection(r, w)
+    check_whole_head(r, w, layer=0, head=1)
     rows = sampled_rows(r["n_in"], w.n_prompt, rng, k=4)
     check_sampled_rows(r, w, layer=0, head=1, rows=rows, groups=[0, 4])
     check_sampled_rows(r, w, layer=47, head=6, rows=rows[:6], groups=[2])
@@ -198,5 +213,7 @@ def test_stress_ragged_context(ctx):
             ref = oracle_scores(x["Q"], x["K_ctx"], x["K_in"], r["scale"])
             assert_scores_close(r["S"][layer * w.H:(layer + 1) * w.H].cpu().numpy(), ref, "ctx0 layer %d" % layer)
     else:
+        head = int(rng.integers(0, w.H))
+        check_whole_head(r, w, layer=0, head=head)
         rows = sampled_rows(r["n_in"], w.n_prompt, rng, k=3)
-        check_sampled_rows(r, w, layer=0, head=int(rng.integers(0, w.H)), rows=rows, groups=[0, 3])
+        check_sampled_rows(r, w, layer=0, head=head, rows=rows, groups=[0, 3])
