@@ -1,17 +1,20 @@
 """Benchmark of the KVzip compression hot path on B200.
 
-One step = score (pass 1 row log-sum-exp + pass 2 context-key column max)
--> select (top ratio per head) -> compact (gather of the kept K/V rows) over
-one Llama-3.1-8B-shaped layer: 8 KV heads, G=4, d=128, n_c=8192 context keys,
-32-token repeat prompt, keep ratio 0.3 per head, bf16, seeded synthetic
-inputs resident in HBM.  The metric is context KV pairs scored and evicted
-per second (B*n_c per step).  L2 is flushed before every timed step (the
-inputs, ~117 MB, would otherwise stay in the 126 MB L2).
+One step = score (pass 1 row log-sum-exp + pass 2 context-key column max, in
+passes of 4096 input positions) -> select (top 25% per head) -> compact (the
+kept K/V rows packed in place) over a whole Qwen2.5-14B-shaped context: 48
+layers x 8 KV heads, G=5 grouped queries, d=128, n_c=131072 context keys,
+32-token repeat prompt, bf16, seeded synthetic inputs resident in HBM.  The
+metric is context KV pairs scored and evicted per second (B*n_c per step).
+Each step starts from the same uncompacted K/V: a pristine copy is restored
+before every step, outside the timed region (that 52 GB copy also leaves
+nothing of the inputs in L2).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload NAME] [--layers L] [--decode]
 
 With N > 1 (launched by torch.distributed.run) every rank runs its own
-independent layer (different seed): weak scaling, no data-path collective.
+independent context (different seed): weak scaling, no data-path collective.
 """
 from __future__ import annotations
 
@@ -30,20 +33,22 @@ sys.path.insert(0, ROOT)
 
 METRIC = "context KV pairs scored+evicted/sec at 1 B200; score TFLOP/s % of bf16 peak"
 UNIT = "context KV pairs/s"
-WORKLOAD = "llama8b_layer"
+WORKLOAD = "qwen14b_128k"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LONG_STEP_MS = 1000.0        # steps at least this long are rated against the sustained bf16 peak
+L2_BYTES = 126 << 20
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="kvz", choices=["kvz", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    help="llama8b_layer (default, the headline), tiny, llama8b_stack, qwen14b_128k, stress_ragged, "
+                    help="qwen14b_128k (default, the headline), llama8b_layer, tiny, llama8b_stack, stress_ragged, "
                          "llama8b_170k_chunked, llama8b_stack_heads, llama8b_stack_int8")
     ap.add_argument("--decode", action="store_true",
                     help="also time one decode step of attention (G queries per KV head) over the pruned cache "
@@ -67,13 +72,14 @@ def peaks():
         return d
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel's
-    source has not changed since the counters were taken."""
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from a committed ncu
+    summary, if the kernel's source has not changed since the counters were
+    taken (None otherwise)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f).get(kernel)
+            rec = json.load(f)["%s/%s" % (kernel, workload)]
         src = os.path.join(ROOT, rec["source"])
         h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         if h != rec["source_sha256_16"]:
@@ -98,7 +104,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "100",
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "200",
                  "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -121,7 +127,7 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        sm, mx, reasons, power = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -130,6 +136,7 @@ class ClockSampler:
             try:
                 sm.append(float(parts[1]))
                 mx = float(parts[2])
+                power.append(float(parts[3]))
             except ValueError:
                 continue
             for n, v in zip(names, parts[5:9]):
@@ -137,9 +144,9 @@ class ClockSampler:
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
-        sm_sorted = sorted(sm)
+        sm_sorted, pw = sorted(sm), sorted(power)
         return {"sm_mhz": sm_sorted[len(sm_sorted) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "power_w_median": pw[len(pw) // 2] if pw else None}
 
 
 def workload_numbers(w):
@@ -174,29 +181,110 @@ def workload_numbers(w):
 
 
 # ---------------------------------------------------------------------------
-# oracle (CPU baseline / reference arm)
+# oracle (CPU baseline / reference arm): bounded samples of one head
 # ---------------------------------------------------------------------------
-def oracle_head_time(x, w, head):
-    """Time the oracle on one head: score, select, compact (the same work the
-    GPU step does for that head).  Returns (seconds, threads)."""
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_head_sample(head_bits, w, n_c, n_in, target_s, max_s, start_frac=0.5, block=64):
+    """Time the oracle, as it stands, on one head of the workload, bounded.
+
+    The head's bf16 inputs are decoded whole; then oracle.score runs on
+    consecutive blocks of `block` input positions (all G groups) from
+    `start_frac` of the input until `target_s` seconds (at most `max_s`) have
+    passed; selection and compaction run on the head's partial scores.  The
+    head's time is the decode + the scored rows' time scaled by the head's
+    visible (row, key) pairs over theirs + select + compact.
+    Returns (pairs_per_second, threads, description, seconds_spent)."""
     import numpy as np
     from oracle import kvz_oracle as orc
 
-    def bits(t):
-        return t[head].detach().cpu().contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
-
-    Q, Kc, Ki, V = bits(x["Q"]), bits(x["K_ctx"]), bits(x["K_in"]), bits(x["V"])
+    Qb, Kcb, Kib, Vb = head_bits
     scale = float(np.float32(1.0 / math.sqrt(w.d)))
     t0 = time.perf_counter()
-    S = orc.score(orc.bf16_bits_to_f64(Q), orc.bf16_bits_to_f64(Kc), orc.bf16_bits_to_f64(Ki), scale)
-    idx, counts, offsets = orc.select(S[None, :].astype(np.float32), w.ratio, w.mode)
-    orc.compact(Kc[None], V[None], idx, counts, offsets)
-    dt = time.perf_counter() - t0
-    try:
-        threads = len(os.sched_getaffinity(0))
-    except Exception:
-        threads = os.cpu_count() or 1
-    return dt, threads, idx
+    Q, Kc, Ki = orc.bf16_bits_to_f64(Qb), orc.bf16_bits_to_f64(Kcb), orc.bf16_bits_to_f64(Kib)
+    t_dec = time.perf_counter() - t0
+    r0 = min(n_in - 1, int(start_frac * n_in)) // block * block
+    r, t_rows, vis_rows = r0, 0.0, 0
+    S = np.zeros(n_c)
+    while t_rows < target_s and r < n_in and t_rows < max_s:
+        r1 = min(n_in, r + block)
+        t1 = time.perf_counter()
+        S = np.maximum(S, orc.score(Q, Kc, Ki, scale, rows=(r, r1)))
+        t_rows += time.perf_counter() - t1
+        vis_rows += w.G * sum(n_c + i + 1 for i in range(r, r1))
+        r = r1
+    t1 = time.perf_counter()
+    mode = "global" if w.mode == "global" else "per_head"
+    idx, counts, offsets = orc.select(S[None, :].astype(np.float32), w.ratio, mode)
+    orc.compact(Kcb[None], Vb[None], idx, counts, offsets)
+    t_sc = time.perf_counter() - t1
+    vis_head = orc.visible_pairs(w.G, n_c, n_in)
+    t_head = t_dec + t_rows * (vis_head / vis_rows) + t_sc
+    desc = ("input positions [%d, %d) of one head (all %d groups): fp64 score of those rows %.1f s, scaled x%.1f "
+            "to the head's %d visible (row, key) pairs; + the head's bf16 decode %.1f s and select + compact %.2f s; "
+            "value = the head's %d context pairs / that extrapolated head time"
+            % (r0, r, w.G, t_rows, vis_head / vis_rows, vis_head, t_dec, t_sc, n_c))
+    return n_c / t_head, _blas_threads(), desc, t_dec + t_rows + t_sc
+
+
+def head_bits_of(x, h):
+    import numpy as np
+    import torch
+
+    def bits(t):
+        return t[h].detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    return bits(x["Q"]), bits(x["K_ctx"]), bits(x["K_in"]), bits(x["V"])
+
+
+def run_reference(args, w, config, rank, world):
+    """The oracle on the host cores, on the same workload: each step is a
+    bounded sample (a block of input positions of one head; heads cycle)."""
+    import torch.distributed as dist
+    from query_agnostic_kv_kvz_b200 import synth
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    n_c, n_in = w.n_c[0], w.n_in(0)
+    x = synth.layer_inputs(w, seed=0, device="cpu")
+    steps, warm = max(1, args.steps), max(0, args.warmup)
+    # a step is sized to a few seconds so that --steps 20 --warmup 5 ends in minutes
+    target = 2.0 if n_c * n_in * w.G > 1e9 else 1.0
+    rates, threads, desc = [], 1, ""
+    for s in range(warm + steps):
+        h = s % w.H
+        frac = ((s * 0.381966) % 1.0) * 0.98            # spread the sampled row blocks over the input
+        rate, threads, desc, _ = oracle_head_sample(head_bits_of(x, h), w, n_c, n_in, target, 4 * target,
+                                                    start_frac=frac)
+        if s >= warm:
+            rates.append(rate)
+    value = sum(rates) / len(rates)
+    ms_step = w.B * len(w.n_c) * n_c / value * 1e3 if len(w.n_c) == 1 else None
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": "each step: one head of layer 0 (heads cycle, row blocks spread over the "
+                                       "input); the last step: " + desc +
+                                       "; ms_per_step extrapolated to the whole step (%d heads)" % w.B},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 # ---------------------------------------------------------------------------
@@ -211,10 +299,10 @@ def main():
     if world > 1:
         from datetime import timedelta
         if args.impl == "reference":                      # the host oracle: no GPU, a CPU process group
-            dist.init_process_group("gloo", timeout=timedelta(seconds=120))
+            dist.init_process_group("gloo", timeout=timedelta(seconds=600))
         else:
             torch.cuda.set_device(local)
-            dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+            dist.init_process_group("nccl", timeout=timedelta(seconds=600))
 
     from query_agnostic_kv_kvz_b200 import synth
     w = synth.WORKLOADS[args.workload]
@@ -225,41 +313,14 @@ def main():
     nums = workload_numbers(w)
     config = {"workload": "%s (L=%d, H=%d, G=%d, d=%d, n_c=%s, n_prompt=%d, keep %.2f %s%s%s)" % (
         w.name, w.L, w.H, w.G, w.d, "/".join(str(n) for n in w.n_c), w.n_prompt, w.ratio, w.mode,
-        ", rows in chunks of %d" % w.row_chunk if w.row_chunk else "", ", in-place compaction" if w.in_place else "")
+        ", rows in passes of %d" % w.row_chunk if w.row_chunk else "", ", in-place compaction" if w.in_place else "")
         + ("; first %d of its %d layers only" % (w.L, n_layers_full) if w.L < n_layers_full else ""),
         "B_heads": w.B, "G": w.G, "d": w.d, "n_c": list(w.n_c), "n_in": [w.n_in(c) for c in range(len(w.n_c))],
         "ratio": w.ratio, "mode": w.mode,
-        "l2": "flushed before every timed step (256 MB write, outside the timed events)",
         "parallelism": "replicas (weak)" if world > 1 else "single GPU"}
 
     if args.impl == "reference":
-        if rank != 0:
-            if world > 1:
-                dist.barrier()
-                dist.destroy_process_group()
-            return
-        x = synth.layer_inputs(w, seed=rank, device="cpu")
-        steps, warm = max(1, args.steps if args.steps < 3 else 3), max(0, min(args.warmup, 3))
-        for s in range(warm):                              # untimed, like the GPU arm's warm-up steps
-            oracle_head_time(x, w, s % w.B)
-        times = []
-        threads = 1
-        for s in range(steps):
-            dt, threads, _ = oracle_head_time(x, w, s % w.B)
-            times.append(dt)
-        per_head = sum(times) / len(times)
-        value = w.n_c[0] / per_head
-        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-                "steps": steps, "warmup": warm, "ms_per_step": per_head * w.B * 1e3, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
-                "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                 "sample": "%d head(s) of the %d-head layer per step (score+select+compact of "
-                                           "one head); ms_per_step extrapolated x%d heads" % (1, w.B, w.B)},
-                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
-        if world > 1:
-            dist.barrier()
-            dist.destroy_process_group()
+        run_reference(args, w, config, rank, world)
         return
 
     dev = torch.device("cuda", local if world > 1 else 0)
@@ -271,15 +332,29 @@ def main():
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     scale = float(1.0 / math.sqrt(w.d))
     ctxs = [Context(w, c, rank_seed(0, rank), dev, kvz) for c in range(len(w.n_c))]
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    input_bytes = sum(c.input_bytes for c in ctxs)
+    # inputs larger than L2 evict themselves (and in-place workloads restore
+    # 2x their K/V between steps); smaller ones get a 256 MB write flush
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if input_bytes < 4 * L2_BYTES else None
+    config["l2"] = ("inputs (%.1f GB) larger than L2%s" % (input_bytes / 1e9, "; K/V restored from a pristine copy "
+                    "before every step, outside the timed events" if w.in_place else "")) if flush is None else \
+        "flushed before every timed step (256 MB write, outside the timed events)"
     launches_per_step = sum(c.launches for c in ctxs)
 
-    def step(ev=None):
-        """One pass of the whole path over the workload; with `ev`, returns the
-        device time (ms) of pass 1, pass 2, selection and compaction."""
+    def prepare():
+        """Untimed: restore in-place workloads' K/V; flush L2 for small inputs."""
+        for c in ctxs:
+            c.restore()
+        if flush is not None:
+            flush.zero_()
+
+    def step(ev=False):
+        """One pass of the whole path over the workload; with `ev`, returns
+        event marks for pass 1, pass 2, selection and compaction."""
         marks = []
+
         def mark(tag):
-            if ev is not None:
+            if ev:
                 e = torch.cuda.Event(enable_timing=True)
                 e.record(stream)
                 marks.append((tag, e))
@@ -335,11 +410,9 @@ def main():
                 acc[tag] += e0.elapsed_time(e1)
         return [acc["p1"] + acc["sc"], acc["p2"], acc["sel"], acc["cmp"]]
 
-    # the headline workload always gets >= 3 warm-up steps; the large ones
-    # (tens of seconds per step) take what the caller asks for
-    n_warm = max(3, args.warmup) if w.name == WORKLOAD else max(1, args.warmup)
+    n_warm = max(3, args.warmup)
     for _ in range(n_warm):
-        flush.zero_()
+        prepare()
         step()
     torch.cuda.synchronize(dev)
     if int(status.item()) != 0:
@@ -348,162 +421,79 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    all_marks = []
+    all_marks, spans = [], []
     with ClockSampler(dev.index) as clk:
-        for s_ in range(args.steps):
-            flush.zero_()
+        for _ in range(args.steps):
+            prepare()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
             all_marks.append(step(ev=True))
+            e1.record(stream)
+            spans.append((e0, e1))
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     parts = [phase_ms(m) for m in all_marks]
-    ms_step = sum(sum(p) for p in parts) / len(parts)
+    ms_step = sum(e0.elapsed_time(e1) for e0, e1 in spans) / len(spans)
     part_ms = [sum(p[i] for p in parts) / len(parts) for i in range(4)]
     if int(status.item()) != 0:
         raise RuntimeError("device status %d during timing" % int(status.item()))
 
-    # ---- end to end through the host-buffer C-ABI call (pinned buffers): every
-    # step copies the inputs in and the results out inside the timed region
+    # ---- end to end through the host-buffer C-ABI call (kvz_compress_host):
+    # every step copies the inputs in from page-locked host memory and the
+    # results out, inside the timed region
     e2e = None
-    if len(ctxs) == 1 and w.L == 1 and not w.in_place and not w.chunk and not w.quant and not w.n_protect:
-        c = ctxs[0]
-        hx = {"Q": c.Q[0].cpu().pin_memory(), "K_ctx": c.K.cpu().pin_memory(), "K_in": c.Kin[0].cpu().pin_memory(),
-              "V": c.V.cpu().pin_memory()}
-        mode = kvz.GLOBAL if w.mode == "global" else kvz.PER_HEAD
-        k = kvz.kvz_keep_count(w.H * c.n_c if mode == kvz.GLOBAL else c.n_c, w.ratio)
-        kept = max(1, k if mode == kvz.GLOBAL else w.H * k)
-        h_out = {"idx": torch.empty(kept, dtype=torch.int32).pin_memory(),
-                 "counts": torch.empty(w.H, dtype=torch.int32).pin_memory(),
-                 "offsets": torch.empty(w.H + 1, dtype=torch.int64).pin_memory(),
-                 "K_out": torch.empty((kept, w.d), dtype=torch.bfloat16).pin_memory(),
-                 "V_out": torch.empty((kept, w.d), dtype=torch.bfloat16).pin_memory()}
-        ws_host = torch.empty(kvz.kvz_compress_host_workspace_size(w.H, w.G, c.n_c, c.n_in, w.d, w.ratio, mode),
-                              dtype=torch.uint8, device=dev)
-        copy_stream = torch.cuda.Stream(dev)
-        h2d = sum(t.numel() * t.element_size() for t in hx.values())
-        d2h = sum(t.numel() * t.element_size() for t in h_out.values())
-
-        def e2e_step():
-            kvz.kvz_compress_host(hx["Q"], hx["K_ctx"], hx["K_in"], hx["V"], w.ratio, mode, scale=scale, out=h_out,
-                                  workspace=ws_host, status=status, stream=stream, copy_stream=copy_stream)
-
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if int(status.item()) != 0:
-            raise RuntimeError("device status %d during e2e" % int(status.item()))
-        e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
+    if not args.no_e2e:
+        e2e = run_e2e(w, ctxs, kvz, dev, stream, status, scale, ms_step)
 
     # ---- decode attention over the pruned cache vs the full cache (one step, all heads)
     dec = None
     if args.decode and not w.quant:
-        c = ctxs[0]
-        B = w.B
-        gq = torch.Generator(device=dev).manual_seed(11)
-        q = torch.randn((B, w.G, w.d), generator=gq, device=dev).to(torch.bfloat16)
-        if w.in_place:
-            Kd, Vd = c.K.view(B * c.n_c, w.d), c.V.view(B * c.n_c, w.d)
-            off_d = torch.arange(B + 1, dtype=torch.int64, device=dev) * c.n_c
-        else:
-            Kd, Vd, off_d = c.K_out, c.V_out, c.offsets
-        full_cnt = torch.full((B,), c.n_c, dtype=torch.int32, device=dev)
-        full_off = torch.arange(B + 1, dtype=torch.int64, device=dev) * c.n_c
-        Kf, Vf = c.K.view(B * c.n_c, w.d), c.V.view(B * c.n_c, w.d)
-        ws_d = torch.empty(kvz.lib().kvz_decode_workspace_size(B, w.G, c.n_c, w.d), dtype=torch.uint8, device=dev)
-        out_d = torch.empty((B, w.G, w.d), dtype=torch.float32, device=dev)
-        lse_d = torch.empty((B, w.G), dtype=torch.float32, device=dev)
-
-        def time_decode(K_, V_, cnt, off, nbytes, iters=20):
-            # a cache over twice the L2 evicts itself between steps (the timing
-            # rules' "inputs larger than L2"); smaller ones get the write flush,
-            # then a read of the same buffer, so that the flush's dirty lines
-            # are written back before the timed call instead of inside it.
-            # One decode call is captured in a CUDA graph and replayed, so that
-            # the host-side cost of a call (binding, tensor maps, two launches)
-            # does not leave the GPU idle inside a short window.
-            big = nbytes > 2 * (126 << 20)
-            for _ in range(3):
-                kvz.kvz_decode(q, K_, V_, cnt, off, c.n_c, scale=scale, out=out_d, lse2=lse_d, workspace=ws_d,
-                               status=status, stream=stream)
-            torch.cuda.synchronize(dev)
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                kvz.kvz_decode(q, K_, V_, cnt, off, c.n_c, scale=scale, out=out_d, lse2=lse_d, workspace=ws_d,
-                               status=status)
-            evs = []
-            for _ in range(iters):            # all enqueued before one sync
-                if not big:
-                    flush.zero_()
-                    flush.view(torch.float32).sum()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                graph.replay()
-                e1.record(stream)
-                evs.append((e0, e1))
-            torch.cuda.synchronize(dev)
-            del graph
-            ts = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
-            return ts[len(ts) // 2]
-
-        kept_rows = nums["kept"]
-        byt = kept_rows * w.d * 2 * 2
-        byt_full = B * c.n_c * w.d * 4
-        t_pruned = time_decode(Kd, Vd, c.counts, off_d, byt)
-        t_full = time_decode(Kf, Vf, full_cnt, full_off, byt_full)
-        if int(status.item()) != 0:
-            raise RuntimeError("device status %d during decode" % int(status.item()))
-        pk0 = peaks()
-        dec = {"ms": t_pruned, "bytes": byt, "gbs": byt / (t_pruned * 1e-3) / 1e9,
-               "frac_hbm": byt / (t_pruned * 1e-3) / 1e9 / pk0["hbm_gbs"],
-               "full_cache_ms": t_full, "full_cache_gbs": B * c.n_c * w.d * 4 / (t_full * 1e-3) / 1e9,
-               "speedup_vs_full_cache": t_full / t_pruned,
-               "what": "one decode step: %d KV heads x %d grouped queries over the pruned cache (%d kept rows) vs "
-                       "the full cache; median of 20 replays of a CUDA graph of the call; caches over 2x L2 "
-                       "unflushed (larger than L2), smaller ones after a 256 MB write flush and a read of that buffer" % (B, w.G, kept_rows)}
+        dec = run_decode(w, ctxs[0], kvz, dev, stream, status, scale, nums)
 
     red = max_over_ranks([ms_step, e2e["ms"] if e2e else 0.0] + part_ms, device=dev)
     ms_step, e2e_ms, part_ms = red[0], red[1], red[2:]
 
     pk = peaks()
+    long_step = ms_step >= LONG_STEP_MS
+    peak_tf = pk["bf16_tflops_sustained"] if long_step else pk["bf16_tflops"]
+    peak_name = "%s bf16 dense, %s" % (pk["source"], "sustained (the kernel runs inside a step of seconds)"
+                                       if long_step else "burst")
     lse_ms, col_ms, sel_ms, cmp_ms = part_ms
     score_ms = lse_ms + col_ms
     fl1, fl2 = nums["flops_pass1"], nums["flops_pass2"]
     tf = lambda flops, ms: flops / (ms * 1e-3) / 1e12
     n_p1 = sum(w.L * (c.score_launches if w.chunk else len(c.chunks)) for c in ctxs)
     chunked = bool(w.chunk)
+    achieved = tf(fl1 + fl2, lse_ms) if chunked else tf(fl1, lse_ms)
     roof = {
         "bound": "tensor",
         "kernel": ("lse_kernel + colmax_kernel (chunked score call, both passes; executed FLOP)" if chunked else
                    "lse_kernel (score pass 1: QK^T + online log-sum-exp)"),
-        "achieved": tf(fl1 + fl2, lse_ms) if chunked else tf(fl1, lse_ms),
-        "peak": pk["bf16_tflops"],
+        "achieved": achieved,
+        "peak": peak_tf,
         "unit": "TFLOP/s",
-        "frac": (tf(fl1 + fl2, lse_ms) if chunked else tf(fl1, lse_ms)) / pk["bf16_tflops"],
-        "traffic": recorded_traffic("lse_kernel") if w.name == WORKLOAD else None,
-        "peak_source": "%s bf16 dense (burst)" % pk["source"],
+        "frac": achieved / peak_tf,
+        "traffic": recorded_traffic("lse_kernel", w.name) if not chunked and w.L == n_layers_full else None,
+        "peak_source": peak_name,
+        "frac_of_burst": achieved / pk["bf16_tflops"],
         "algorithmic_flops_per_launch": fl1 / n_p1,
         "launches_per_step": n_p1,
+        "launch_ms": lse_ms / n_p1,
         "breakdown": {
             "score_pass1_ms": lse_ms, "score_pass2_ms": col_ms, "select_ms": sel_ms, "compact_ms": cmp_ms,
             "score_tflops_executed": tf(fl1 + fl2, score_ms),
-            "score_frac_executed": tf(fl1 + fl2, score_ms) / pk["bf16_tflops"],
+            "score_frac_executed": tf(fl1 + fl2, score_ms) / peak_tf,
             "score_tflops_algorithmic": tf(nums["flops_algorithmic"], score_ms),
-            "score_frac_algorithmic": tf(nums["flops_algorithmic"], score_ms) / pk["bf16_tflops"],
+            "score_frac_algorithmic": tf(nums["flops_algorithmic"], score_ms) / peak_tf,
             "pass2_tflops": tf(fl2, col_ms) if col_ms > 0 else None,
-            "pass2_frac": tf(fl2, col_ms) / pk["bf16_tflops"] if col_ms > 0 else None,
+            "pass2_frac": tf(fl2, col_ms) / peak_tf if col_ms > 0 else None,
             "compact_bytes": nums["compact_bytes"],
             "compact_gbs": nums["compact_bytes"] / (cmp_ms * 1e-3) / 1e9,
             "compact_frac_hbm": nums["compact_bytes"] / (cmp_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
             "select_gbs": nums["select_bytes"] / (sel_ms * 1e-3) / 1e9,
+            "peaks": {"bf16_tflops_burst": pk["bf16_tflops"], "bf16_tflops_sustained": pk["bf16_tflops_sustained"],
+                      "hbm_gbs": pk["hbm_gbs"], "source": pk["source"]},
         },
     }
     value = nums["pairs_per_step"] * world / (ms_step * 1e-3)
@@ -518,26 +508,21 @@ def main():
         line["decode"] = dec
     if e2e is not None:
         line["e2e"] = {"value": nums["pairs_per_step"] * world / (e2e_ms * 1e-3), "unit": UNIT,
-                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and w.name == WORKLOAD:
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_ms,
+                       "how": e2e["how"]}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         c = ctxs[0]
-        x0 = {"Q": c.Q[0], "K_ctx": c.K[: w.H], "K_in": c.Kin[0], "V": c.V[: w.H]}
-        dt, threads, oracle_idx = oracle_head_time(x0, w, 0)
-        line["cpu_baseline"] = {"value": c.n_c / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": "head 0 of the %d-head layer: fp64 score + select + compact "
-                                          "(%.1f s)" % (w.B, dt)}
-        # index-set overlap of the GPU's kept keys with the oracle's selection
-        # from its own fp64 scores (reported, not gated: a top-k over scores
-        # that agree within the tolerance may still differ at the threshold)
-        o0, o1 = int(c.offsets[0].item()), int(c.offsets[1].item())
-        gpu_set = set(c.idx[o0:o1].cpu().tolist())
-        ora_set = set(int(v) for v in oracle_idx)
-        line["selection_overlap"] = {"head": 0, "jaccard": len(gpu_set & ora_set) / max(1, len(gpu_set | ora_set)),
-                                     "kept": len(ora_set)}
+        x0 = {"Q": c.Q[0] if c.Q else None, "K_ctx": c.K0[: w.H] if c.K0 is not None else c.K[: w.H],
+              "K_in": c.Kin[0] if c.Kin else None, "V": c.V0[: w.H] if c.V0 is not None else c.V[: w.H]}
+        if x0["Q"] is not None:
+            rate, threads, desc, spent = oracle_head_sample(head_bits_of(x0, 0), w, c.n_c, c.n_in, 12.0, 30.0)
+            line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                    "sample": "layer 0 head 0, " + desc + " (%.1f s of CPU time)" % spent}
         # exact ties among the GPU's scores of head 0: at the keep threshold
         # (where the lower-index rule decides) and overall (equal fp32 values)
         import numpy as np
         s0 = c.S[0].cpu().numpy()
+        o0, o1 = int(c.offsets[0].item()), int(c.offsets[1].item())
         k0 = o1 - o0
         thr = np.sort(s0)[::-1][k0 - 1] if k0 > 0 else np.float32(np.inf)
         line["ties"] = {"head": 0, "at_threshold": int(np.count_nonzero(s0 == thr)) if k0 > 0 else 0,
@@ -549,15 +534,179 @@ def main():
         dist.destroy_process_group()
 
 
+def run_e2e(w, ctxs, kvz, dev, stream, status, scale, ms_step):
+    """The metric through kvz_compress_host: host buffers in, host buffers
+    out, the copies inside the timed region.  Per-head workloads call it once
+    per layer (the heads of a layer are one context's independent problems);
+    global ones once for the whole context.  Host inputs live in page-locked
+    memory; when the host cannot hold every layer, the distinct layers it can
+    hold are cycled (stated in `how`)."""
+    import torch
+    if w.chunk or w.quant or w.n_protect or w.mode == "heads" or len(ctxs) != 1:
+        return None
+    c = ctxs[0]
+    per_layer = w.mode == "per_head"
+    calls = w.L if per_layer else 1
+    Bc = w.H if per_layer else w.B
+    row = w.d * 2
+    in_bytes = Bc * (w.G * c.n_in + 2 * c.n_c + c.n_in) * row          # Q, K_ctx, V, K_in of one call
+    mode = kvz.PER_HEAD if per_layer else kvz.GLOBAL
+    k = kvz.kvz_keep_count(c.n_c if per_layer else Bc * c.n_c, w.ratio)
+    kept = Bc * k if per_layer else k
+    out_bytes = kept * (4 + 2 * row) + Bc * 4 + (Bc + 1) * 8
+    try:
+        import psutil
+        budget = int(0.40 * psutil.virtual_memory().available)
+    except Exception:
+        budget = 8 << 30
+    n_host = max(1, min(calls, (budget - 2 * out_bytes) // in_bytes))
+    if n_host < calls and not per_layer:
+        return None
+    cudart = torch.cuda.cudart()
+    registered = []
+
+    def pinned(shape, dtype):
+        # page-locked in place (torch's pinned allocator would round each
+        # buffer up to a power of two); a pinned copy if registration fails
+        t = torch.empty(shape, dtype=dtype)
+        if t.numel() > 0:
+            if int(cudart.cudaHostRegister(t.data_ptr(), t.numel() * t.element_size(), 0)) != 0:
+                return t.pin_memory()
+            registered.append(t)
+        return t
+
+    try:
+        hosts = []
+        for hl in range(n_host):
+            if per_layer:
+                src = {"Q": c.Q[hl], "K_ctx": c.pristine_K()[hl * w.H:(hl + 1) * w.H], "K_in": c.Kin[hl],
+                       "V": c.pristine_V()[hl * w.H:(hl + 1) * w.H]}
+            else:
+                src = {"Q": torch.cat(c.Q), "K_ctx": c.pristine_K(), "K_in": torch.cat(c.Kin), "V": c.pristine_V()}
+            h = {n: pinned(tuple(t.shape), torch.bfloat16) for n, t in src.items()}
+            for n, t in src.items():
+                h[n].copy_(t)
+            hosts.append(h)
+        outs = [{"idx": pinned((max(kept, 1),), torch.int32), "counts": pinned((Bc,), torch.int32),
+                 "offsets": pinned((Bc + 1,), torch.int64), "K_out": pinned((max(kept, 1), w.d), torch.bfloat16),
+                 "V_out": pinned((max(kept, 1), w.d), torch.bfloat16)} for _ in range(2)]
+        ws = torch.empty(kvz.kvz_compress_host_workspace_size(Bc, w.G, c.n_c, c.n_in, w.d, w.ratio, mode),
+                         dtype=torch.uint8, device=dev)
+        copy_stream = torch.cuda.Stream(dev)
+
+        def call(i):
+            hx = hosts[i % n_host]
+            kvz.kvz_compress_host(hx["Q"], hx["K_ctx"], hx["K_in"], hx["V"], w.ratio, mode, scale=scale,
+                                  out=outs[i % 2], workspace=ws, status=status, stream=stream,
+                                  copy_stream=copy_stream)
+
+        call(0)                                             # warm-up: one call
+        torch.cuda.synchronize(dev)
+        steps = max(1, min(20, int(math.ceil(20000.0 / max(ms_step, 1e-3)))))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            for i in range(calls):
+                call(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if int(status.item()) != 0:
+            raise RuntimeError("device status %d during e2e" % int(status.item()))
+        ms = e0.elapsed_time(e1) / steps
+        h2d = calls * in_bytes
+        d2h = calls * out_bytes
+        how = ("kvz_compress_host %s (%d heads per call, %d call(s) per step, %d timed step(s)): inputs copied in "
+               "from page-locked host memory by head chunks overlapping the scoring, selection and out-of-place "
+               "compaction on the device, kept rows / indices copied back; %d distinct host layer(s)%s"
+               % ("per layer" if per_layer else "for the whole context", Bc, calls, steps, n_host,
+                  "" if n_host == calls else " cycled (host memory holds %d of %d)" % (n_host, calls)))
+        return {"ms": ms, "h2d": h2d, "d2h": d2h, "how": how}
+    finally:
+        torch.cuda.synchronize(dev)
+        for t in registered:
+            cudart.cudaHostUnregister(t.data_ptr())
+
+
+def run_decode(w, c, kvz, dev, stream, status, scale, nums):
+    import torch
+    B = w.B
+    gq = torch.Generator(device=dev).manual_seed(11)
+    q = torch.randn((B, w.G, w.d), generator=gq, device=dev).to(torch.bfloat16)
+    if w.in_place:
+        Kd, Vd = c.K.view(B * c.n_c, w.d), c.V.view(B * c.n_c, w.d)
+        off_d = torch.arange(B + 1, dtype=torch.int64, device=dev) * c.n_c
+    else:
+        Kd, Vd, off_d = c.K_out, c.V_out, c.offsets
+    full_cnt = torch.full((B,), c.n_c, dtype=torch.int32, device=dev)
+    full_off = torch.arange(B + 1, dtype=torch.int64, device=dev) * c.n_c
+    Kf, Vf = c.pristine_K().view(B * c.n_c, w.d), c.pristine_V().view(B * c.n_c, w.d)
+    ws_d = torch.empty(kvz.lib().kvz_decode_workspace_size(B, w.G, c.n_c, w.d), dtype=torch.uint8, device=dev)
+    out_d = torch.empty((B, w.G, w.d), dtype=torch.float32, device=dev)
+    lse_d = torch.empty((B, w.G), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def time_decode(K_, V_, cnt, off, nbytes, iters=20):
+        # a cache over twice the L2 evicts itself between steps (inputs larger
+        # than L2); smaller ones get the write flush, then a read of the same
+        # buffer, so that the flush's dirty lines are written back before the
+        # timed call instead of inside it.  One decode call is captured in a
+        # CUDA graph and replayed, so that the host-side cost of a call
+        # (binding, tensor maps, two launches) does not leave the GPU idle
+        # inside a short window.
+        big = nbytes > 2 * L2_BYTES
+        for _ in range(3):
+            kvz.kvz_decode(q, K_, V_, cnt, off, c.n_c, scale=scale, out=out_d, lse2=lse_d, workspace=ws_d,
+                           status=status, stream=stream)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            kvz.kvz_decode(q, K_, V_, cnt, off, c.n_c, scale=scale, out=out_d, lse2=lse_d, workspace=ws_d,
+                           status=status)
+        evs = []
+        for _ in range(iters):            # all enqueued before one sync
+            if not big:
+                flush.zero_()
+                flush.view(torch.float32).sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            evs.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        del graph
+        ts = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
+        return ts[len(ts) // 2]
+
+    kept_rows = nums["kept"]
+    byt = kept_rows * w.d * 2 * 2
+    byt_full = B * c.n_c * w.d * 4
+    t_pruned = time_decode(Kd, Vd, c.counts, off_d, byt)
+    t_full = time_decode(Kf, Vf, full_cnt, full_off, byt_full)
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %d during decode" % int(status.item()))
+    pk0 = peaks()
+    return {"ms": t_pruned, "bytes": byt, "gbs": byt / (t_pruned * 1e-3) / 1e9,
+            "frac_hbm": byt / (t_pruned * 1e-3) / 1e9 / pk0["hbm_gbs"],
+            "full_cache_ms": t_full, "full_cache_gbs": byt_full / (t_full * 1e-3) / 1e9,
+            "speedup_vs_full_cache": t_full / t_pruned,
+            "what": "one decode step: %d KV heads x %d grouped queries over the pruned cache (%d kept rows) vs "
+                    "the full cache; median of 20 replays of a CUDA graph of the call; caches over 2x L2 "
+                    "unflushed (larger than L2), smaller ones after a 256 MB write flush and a read of that "
+                    "buffer" % (B, w.G, kept_rows)}
+
+
 class Context:
     """Device-resident inputs and outputs of one context of a workload: all
-    layers' Q / K_in, the whole K/V cache, scores, selection and outputs."""
+    layers' Q / K_in, the whole K/V cache (and, when it is compacted in
+    place, a pristine copy restored before every step), scores, selection
+    and outputs."""
 
     def __init__(self, w, c, seed, dev, kvz):
         import torch
         from query_agnostic_kv_kvz_b200 import synth
         H, G, d, L = w.H, w.G, w.d, w.L
         B = L * H
+        self.w = w
         self.n_c, self.n_in = w.n_c[c], w.n_in(c)
         self.K = torch.empty((B, self.n_c, d), dtype=torch.bfloat16, device=dev)
         self.V = torch.empty((B, self.n_c, d), dtype=torch.bfloat16, device=dev)
@@ -580,6 +729,9 @@ class Context:
             self.Q.append(x["Q"])
             self.Kin.append(x["K_in"])
             del x
+        self.K0 = self.K.clone() if w.in_place else None
+        self.V0 = self.V.clone() if w.in_place else None
+        self.input_bytes = 2 * self.K.numel() * 2 + sum(t.numel() * 2 for t in self.Q + self.Kin)
         chunk = min(w.row_chunk or self.n_in, self.n_in)
         self.chunks = [(i0, min(self.n_in, i0 + chunk)) for i0 in range(0, self.n_in, chunk)]
         self.ld = (chunk + 255) // 256 * 256
@@ -620,6 +772,17 @@ class Context:
             self.launches = L * (2 * self.score_launches + 1) + sel + (3 if w.in_place else 1)
         else:
             self.launches = L * (2 * len(self.chunks) + 1) + sel + (3 if w.in_place else 1)
+
+    def restore(self):
+        if self.K0 is not None:
+            self.K.copy_(self.K0)
+            self.V.copy_(self.V0)
+
+    def pristine_K(self):
+        return self.K0 if self.K0 is not None else self.K
+
+    def pristine_V(self):
+        return self.V0 if self.V0 is not None else self.V
 
 
 if __name__ == "__main__":
