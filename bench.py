@@ -373,7 +373,7 @@ def main():
                 for (i0, i1) in c.chunks:
                     mark("p1")
                     kvz.kvz_score_lse2(c.Q[l], Kl, c.Kin[l], i_begin=i0, i_end=i1, scale=scale, lse2=c.lse2,
-                                       ld=c.ld, status=status, stream=stream)
+                                       ld=c.ld, workspace=c.lse_ws, status=status, stream=stream)
                     mark("p2")
                     kvz.kvz_score_colmax(c.Q[l], Kl, c.lse2, i_begin=i0, i_end=i1, scale=scale, S=Sl,
                                          accumulate=i0 > 0, status=status, stream=stream)
@@ -556,7 +556,7 @@ def run_e2e(w, ctxs, kvz, dev, stream, status, scale, ms_step):
     out_bytes = kept * (4 + 2 * row) + Bc * 4 + (Bc + 1) * 8
     try:
         import psutil
-        budget = int(0.40 * psutil.virtual_memory().available)
+        budget = int(0.60 * psutil.virtual_memory().available)
     except Exception:
         budget = 8 << 30
     n_host = max(1, min(calls, (budget - 2 * out_bytes) // in_bytes))
@@ -736,6 +736,7 @@ class Context:
         self.chunks = [(i0, min(self.n_in, i0 + chunk)) for i0 in range(0, self.n_in, chunk)]
         self.ld = (chunk + 255) // 256 * 256
         self.lse2 = torch.empty((H, G, self.ld), dtype=torch.float32, device=dev)
+        self.lse_ws = torch.empty(kvz.kvz_score_lse2_workspace_size(), dtype=torch.uint8, device=dev)
         self.S = torch.empty((B, self.n_c), dtype=torch.float32, device=dev)
         mode = kvz.GLOBAL if w.mode == "global" else kvz.PER_HEAD
         if w.mode == "heads":

@@ -30,7 +30,10 @@
  *   - Head index b enumerates the B = L*H KV heads of a call layer-major
  *     (b = l*H + h), so a whole model's cache is one call.
  *   - Results are deterministic: identical inputs give bit-identical S, idx,
- *     counts, offsets and compacted rows, independent of scheduling.
+ *     counts, offsets and compacted rows, independent of scheduling (for
+ *     the same call arguments on the same GPU model: pass 1's grid follows
+ *     the call's sizes and the SM count, and fixes which work units of its
+ *     partial last wave are split over key ranges).
  */
 #ifndef KVZ_H_
 #define KVZ_H_
@@ -86,14 +89,16 @@ const char* kvz_status_string(int status);
 /*                                                                          */
 /* Work is done in row chunks of `row_chunk` input positions (0 = all rows  */
 /* in one pass; otherwise a positive multiple of 256).  Chunks merge by an   */
-/* exact max, so the result does not depend on row_chunk; only the          */
-/* workspace size does.  Limits: d in {64,128}; G >= 1; n_c, n_in >= 1;     */
+/* exact max; row_chunk changes the result only in float rounding (where    */
+/* pass 1 splits its partial last wave, see kvz_score_lse2) and sets the    */
+/* workspace size.  Limits: d in {64,128}; G >= 1; n_c, n_in >= 1;          */
 /* B*G <= 2^31-1; n_c, n_in <= 2^31-1; scale finite and > 0.                */
 /* ------------------------------------------------------------------------ */
 
 /* Bytes of workspace kvz_score needs: B*G*P*4 rounded up to 256, where P is
  * the row count of one chunk, min(row_chunk or n_in, n_in), rounded up to a
- * multiple of 256.  Returns 0 for invalid arguments. */
+ * multiple of 256, plus kvz_score_lse2_workspace_size() for pass 1's split
+ * last wave.  Returns 0 for invalid arguments. */
 size_t kvz_score_workspace_size(int64_t B, int G, int64_t n_in, int64_t row_chunk);
 
 /* Full scoring: zero-fills S, then for each row chunk runs pass 1 (row
@@ -111,11 +116,19 @@ kvz_status kvz_score(const void* Q, const void* K_ctx, const void* K_in,
  * Entries for padding rows, i in [i_end, i_begin + roundup(i_end-i_begin,256)),
  * are set to +inf (they then never contribute in pass 2).
  * Requires i_begin % 256 == 0, 0 <= i_begin < i_end <= n_in,
- * ld_lse2 >= roundup(i_end - i_begin, 256) and ld_lse2 % 4 == 0. */
+ * ld_lse2 >= roundup(i_end - i_begin, 256) and ld_lse2 % 4 == 0.
+ * `workspace` (nullable, kvz_score_lse2_workspace_size() bytes, 16-byte
+ * aligned) lets the work units of the grid's partial last wave be split
+ * over key ranges and merged exactly (max, then rescaled sums, in a fixed
+ * order), so the last wave fills the GPU; NULL computes every unit whole.
+ * The two differ only in float rounding, well inside the score tolerance. */
+size_t kvz_score_lse2_workspace_size(void);
+
 kvz_status kvz_score_lse2(const void* Q, const void* K_ctx, const void* K_in,
                           int64_t B, int G, int64_t n_c, int64_t n_in, int d,
                           float scale, int64_t i_begin, int64_t i_end,
                           float* lse2, int64_t ld_lse2,
+                          void* workspace, size_t workspace_bytes,
                           int32_t* d_status, cudaStream_t stream);
 
 /* Pass 2 alone, for the rows whose lse2 pass 1 produced (same i_begin,

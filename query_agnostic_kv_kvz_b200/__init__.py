@@ -18,7 +18,7 @@ import torch
 __all__ = [
     "KvzError", "KvzLibraryError", "lib", "lib_path", "STATUS", "PER_HEAD", "GLOBAL",
     "kvz_version", "kvz_keep_count", "kvz_score_workspace_size", "kvz_score", "kvz_score_noalloc",
-    "kvz_score_lse2", "kvz_score_colmax", "kvz_select_workspace_size", "kvz_select",
+    "kvz_score_lse2", "kvz_score_lse2_workspace_size", "kvz_score_colmax", "kvz_select_workspace_size", "kvz_select",
     "kvz_select_dist_workspace_size", "kvz_select_dist_begin", "kvz_select_dist_step", "kvz_select_dist_finish",
     "kvz_compact_workspace_size", "kvz_compact", "kvz_compress_host_workspace_size", "kvz_compress_host",
     "kvz_score_chunked_workspace_size", "kvz_score_chunked", "kvz_head_score", "kvz_select_heads", "kvz_decode",
@@ -57,8 +57,9 @@ _SIGS = {
     "kvz_status_string": (_c.c_char_p, [_i32]),
     "kvz_score_workspace_size": (_sz, [_i64, _i32, _i64, _i64]),
     "kvz_score": (_i32, [_vp, _vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _i64, _vp, _vp, _sz, _vp, _vp]),
-    "kvz_score_lse2": (_i32, [_vp, _vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _i64, _i64, _vp, _i64, _vp,
-                              _vp]),
+    "kvz_score_lse2_workspace_size": (_sz, []),
+    "kvz_score_lse2": (_i32, [_vp, _vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _i64, _i64, _vp, _i64, _vp, _sz,
+                              _vp, _vp]),
     "kvz_score_colmax": (_i32, [_vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _i64, _i64, _vp, _i64, _vp,
                                 _i32, _vp, _vp]),
     "kvz_score_noalloc": (_i32, [_vp, _vp, _vp, _i64, _i32, _i64, _i64, _i32, _f32, _vp, _vp, _vp]),
@@ -244,8 +245,11 @@ def kvz_score_noalloc(Q, K_ctx, K_in, scale: Optional[float] = None, S=None, sta
 
 
 def kvz_score_lse2(Q, K_ctx, K_in, i_begin: int = 0, i_end: Optional[int] = None, scale: Optional[float] = None,
-                   lse2=None, ld: Optional[int] = None, status=None, stream=None):
-    """Pass 1: base-2 log-sum-exp of input rows [i_begin, i_end); returns lse2 [B, G, ld]."""
+                   lse2=None, ld: Optional[int] = None, workspace=None, status=None, stream=None):
+    """Pass 1: base-2 log-sum-exp of input rows [i_begin, i_end); returns lse2 [B, G, ld].
+    ``workspace`` (uint8, kvz_score_lse2_workspace_size() bytes) lets the
+    grid's last wave be split over key ranges; it is allocated when not
+    given."""
     fn = "kvz_score_lse2"
     if K_in is None:
         raise ValueError("%s: K_in is required" % fn)
@@ -264,16 +268,24 @@ def kvz_score_lse2(Q, K_ctx, K_in, i_begin: int = 0, i_end: Optional[int] = None
     ld = rows_pad if ld is None else int(ld)
     if ld < rows_pad or ld % 4 != 0:
         raise ValueError("%s: ld must be >= %d and a multiple of 4" % (fn, rows_pad))
+    _req(fn, "workspace", workspace, torch.uint8)
     _status(fn, status)
-    dev = _device(fn, Q, K_ctx, K_in, lse2, status)
+    dev = _device(fn, Q, K_ctx, K_in, lse2, workspace, status)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     with torch.cuda.device(dev):
         if lse2 is None:
             lse2 = torch.empty((B, G, ld), dtype=torch.float32, device=dev)
+        if workspace is None:
+            workspace = torch.empty(kvz_score_lse2_workspace_size(), dtype=torch.uint8, device=dev)
         _check(fn, lib().kvz_score_lse2(_ptr(Q), _ptr(K_ctx), _ptr(K_in), B, G, n_c, n_in, d, scale, i_begin, i_end,
-                                        _ptr(lse2), ld, _ptr(status), _stream(stream)))
+                                        _ptr(lse2), ld, _ptr(workspace), _bytes(workspace), _ptr(status),
+                                        _stream(stream)))
     return lse2
+
+
+def kvz_score_lse2_workspace_size() -> int:
+    return lib().kvz_score_lse2_workspace_size()
 
 
 def kvz_score_colmax(Q, K_ctx, lse2, i_begin: int = 0, i_end: Optional[int] = None,

@@ -107,9 +107,11 @@ kvz_status check_score_common(const void* Q, const void* K_ctx, int64_t B, int G
   return KVZ_OK;
 }
 
+// `part`: kvz::kLsePartBytes of scratch for the split tail of pass 1's
+// grid, or null (no split).
 kvz_status run_lse(const void* Q, const void* K_ctx, const void* K_in, int64_t B, int G, int64_t n_c,
                    int64_t n_in, int d, float scale, int64_t i_begin, int64_t i_end, float* lse2, int64_t ld,
-                   int32_t* status, cudaStream_t stream, CtxGeom geom) {
+                   int32_t* status, cudaStream_t stream, CtxGeom geom, void* part) {
   CUtensorMap tmQ, tmKc, tmKi;
   if (!make_map(&tmQ, Q, d, n_in, B * G) ||
       !make_ctx_map(&tmKc, K_ctx, d, n_c, geom.T, B / geom.T, geom.block_stride, geom.head_stride) ||
@@ -128,6 +130,7 @@ kvz_status run_lse(const void* Q, const void* K_ctx, const void* K_in, int64_t B
   a.ld = ld;
   a.lse2 = lse2;
   a.status = status;
+  a.part = static_cast<float2*>(part);
   return kvz::launch_lse(d, tmQ, tmKc, tmKi, a, stream) == cudaSuccess ? KVZ_OK : KVZ_ERR_CUDA;
 }
 
@@ -175,24 +178,32 @@ const char* kvz_status_string(int status) {
   }
 }
 
+// Bytes of one chunk's lse2 in a scoring workspace (the split-tail scratch
+// of pass 1 follows it).
+int64_t lse_area_bytes(int64_t B, int G, int64_t rows) { return roundup(B * G * roundup(rows, 256) * 4, 256); }
+
 size_t kvz_score_workspace_size(int64_t B, int G, int64_t n_in, int64_t row_chunk) {
   if (B < 1 || G < 1 || n_in < 1 || row_chunk < 0 || (row_chunk % 256) != 0) return 0;
   const int64_t rows = row_chunk == 0 || row_chunk > n_in ? n_in : row_chunk;
-  const int64_t bytes = B * G * roundup(rows, 256) * 4;
-  return static_cast<size_t>(roundup(bytes, 256));
+  return static_cast<size_t>(lse_area_bytes(B, G, rows)) + kvz::kLsePartBytes;
 }
+
+size_t kvz_score_lse2_workspace_size(void) { return kvz::kLsePartBytes; }
 
 kvz_status kvz_score_lse2(const void* Q, const void* K_ctx, const void* K_in, int64_t B, int G, int64_t n_c,
                           int64_t n_in, int d, float scale, int64_t i_begin, int64_t i_end, float* lse2,
-                          int64_t ld_lse2, int32_t* d_status, cudaStream_t stream) {
+                          int64_t ld_lse2, void* workspace, size_t workspace_bytes, int32_t* d_status,
+                          cudaStream_t stream) {
   kvz_status st = check_score_common(Q, K_ctx, B, G, n_c, n_in, d, scale);
   if (st != KVZ_OK) return st;
   if (K_in == nullptr || lse2 == nullptr) return KVZ_ERR_INVALID_ARG;
   if (!aligned(K_in, 16) || !aligned(lse2, 16) || ld_lse2 % 4 != 0) return KVZ_ERR_ALIGNMENT;
   if (i_begin < 0 || i_begin % 256 != 0 || i_end <= i_begin || i_end > n_in) return KVZ_ERR_INVALID_ARG;
   if (ld_lse2 < roundup(i_end - i_begin, 256)) return KVZ_ERR_INVALID_ARG;
+  if (workspace != nullptr && workspace_bytes < kvz::kLsePartBytes) return KVZ_ERR_WORKSPACE;
+  if (workspace != nullptr && !aligned(workspace, 16)) return KVZ_ERR_ALIGNMENT;
   return run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i_begin, i_end, lse2, ld_lse2, d_status, stream,
-                 plain_geom(n_c));
+                 plain_geom(n_c), workspace);
 }
 
 kvz_status kvz_score_colmax(const void* Q, const void* K_ctx, int64_t B, int G, int64_t n_c, int64_t n_in, int d,
@@ -223,10 +234,12 @@ kvz_status kvz_score(const void* Q, const void* K_ctx, const void* K_in, int64_t
   const int64_t chunk = (row_chunk == 0 || row_chunk > n_in) ? n_in : row_chunk;
   const int64_t ld = roundup(chunk, 256);
   float* lse2 = static_cast<float*>(workspace);
+  void* part = static_cast<uint8_t*>(workspace) + lse_area_bytes(B, G, chunk);
   if (kvz::launch_fill_f32(S, B * n_c, 0.0f, stream) != cudaSuccess) return KVZ_ERR_CUDA;
   for (int64_t i0 = 0; i0 < n_in; i0 += chunk) {
     const int64_t i1 = i0 + chunk < n_in ? i0 + chunk : n_in;
-    st = run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, d_status, stream, plain_geom(n_c));
+    st = run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, d_status, stream, plain_geom(n_c),
+                 part);
     if (st != KVZ_OK) return st;
     st = run_colmax(Q, K_ctx, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, S, d_status, stream, plain_geom(n_c),
                     n_c, n_c);
@@ -240,7 +253,7 @@ size_t kvz_score_chunked_workspace_size(int64_t B, int G, int64_t n_c, int64_t n
   const int64_t T = n_c / m, m_last = n_c % m;
   const int64_t full = T > 0 ? B * T * G * roundup(n_prompt + m, 256) * 4 : 0;
   const int64_t tail = m_last > 0 ? B * G * roundup(n_prompt + m_last, 256) * 4 : 0;
-  return static_cast<size_t>(roundup(full > tail ? full : tail, 256));
+  return static_cast<size_t>(roundup(full > tail ? full : tail, 256)) + kvz::kLsePartBytes;
 }
 
 kvz_status kvz_score_chunked(const void* Q, const void* Q_tail, const void* K_ctx, const void* K_in,
@@ -264,12 +277,15 @@ kvz_status kvz_score_chunked(const void* Q, const void* Q_tail, const void* K_ct
     return KVZ_ERR_WORKSPACE;
   if (!aligned(workspace, 16)) return KVZ_ERR_ALIGNMENT;
   float* lse2 = static_cast<float*>(workspace);
+  void* part = static_cast<uint8_t*>(workspace) +
+               (kvz_score_chunked_workspace_size(B, G, n_c, n_prompt, m) - kvz::kLsePartBytes);
   if (kvz::launch_fill_f32(S, B * n_c, 0.0f, stream) != cudaSuccess) return KVZ_ERR_CUDA;
   if (T > 0) {
     // the full chunks of every head as one batch of B*T problems
     const int64_t n_in = n_prompt + m, ld = roundup(n_in, 256);
     const CtxGeom geom{static_cast<int>(T), m, n_c};
-    kvz_status st = run_lse(Q, K_ctx, K_in, B * T, G, m, n_in, d, scale, 0, n_in, lse2, ld, d_status, stream, geom);
+    kvz_status st =
+        run_lse(Q, K_ctx, K_in, B * T, G, m, n_in, d, scale, 0, n_in, lse2, ld, d_status, stream, geom, part);
     if (st != KVZ_OK) return st;
     st = run_colmax(Q, K_ctx, B * T, G, m, n_in, d, scale, 0, n_in, lse2, ld, S, d_status, stream, geom, n_c, m);
     if (st != KVZ_OK) return st;
@@ -280,7 +296,7 @@ kvz_status kvz_score_chunked(const void* Q, const void* Q_tail, const void* K_ct
     const void* K_last = static_cast<const uint8_t*>(K_ctx) + T * m * d * 2;
     const CtxGeom geom{1, m_last, n_c};
     kvz_status st = run_lse(Q_tail, K_last, K_in_tail, B, G, m_last, n_in, d, scale, 0, n_in, lse2, ld, d_status,
-                            stream, geom);
+                            stream, geom, part);
     if (st != KVZ_OK) return st;
     st = run_colmax(Q_tail, K_last, B, G, m_last, n_in, d, scale, 0, n_in, lse2, ld, S + T * m, d_status, stream,
                     geom, n_c, m_last);
@@ -386,7 +402,8 @@ kvz_status kvz_score_noalloc(const void* Q, const void* K_ctx, const void* K_in,
   if (kvz::launch_fill_f32(S, B * n_c, 0.0f, stream) != cudaSuccess) return KVZ_ERR_CUDA;
   for (int64_t i0 = 0; i0 < n_in; i0 += chunk) {
     const int64_t i1 = i0 + chunk < n_in ? i0 + chunk : n_in;
-    st = run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, d_status, stream, plain_geom(n_c));
+    st = run_lse(Q, K_ctx, K_in, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, d_status, stream, plain_geom(n_c),
+                 nullptr);
     if (st != KVZ_OK) return st;
     st = run_colmax(Q, K_ctx, B, G, n_c, n_in, d, scale, i0, i1, lse2, ld, S, d_status, stream, plain_geom(n_c),
                     n_c, n_c);

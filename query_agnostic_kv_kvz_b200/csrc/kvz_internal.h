@@ -32,6 +32,12 @@ cudaError_t smem_limit_once(int bytes) {
 // Problem p reads context-key block (p % T) of head (p / T): T = 1 for the
 // plain score, T = chunks per head for chunked scoring (the context-key map
 // is 4-D: columns, rows of a block, block, head).
+// Grid: one CTA per (head, group, 256-row block) unit, longest first; the
+// last r units (the partial last wave) may each be split into `nsplit`
+// CTAs over consecutive key-tile ranges.  CTA x < n_full computes unit x
+// whole; CTA n_full + t computes part t % nsplit of unit n_full + t / nsplit
+// and writes its rows' partial (max, sum) to part[t * 256 + row]; a merge
+// kernel then combines the parts of each unit in order.
 struct LseArgs {
   int B, G, T;
   int64_t n_c, n_in;
@@ -39,7 +45,16 @@ struct LseArgs {
   int64_t i_begin, i_end, rows_pad, ld;
   float* lse2;
   int32_t* status;
+  int n_full;               // CTAs that compute a whole unit (set by launch_lse)
+  int nsplit;               // parts per split unit, 1 = none (set by launch_lse)
+  float2* part;             // [split CTAs][256] partial (max, sum); null = no split
+  int head_major;           // unit order: 0 = row block, then (head, group); 1 = head, then row block, then
+                            // group (set by launch_lse)
 };
+// Scratch for split units: at most this many split CTAs, 256 rows of
+// (max, sum) each.
+constexpr int kLseMaxSplitCtas = 256;
+constexpr size_t kLsePartBytes = static_cast<size_t>(kLseMaxSplitCtas) * 256 * 8;
 
 // Pass 2 (context-key column max) arguments; lse2 as pass 1 wrote it.
 struct ColArgs {

@@ -59,6 +59,26 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t* bar, uint32_t parity
   return ok;
 }
 
+// As mbar_try_wait, letting the thread be suspended in hardware for up to
+// `hint_ns` nanoseconds while the phase is incomplete (it resumes as soon as
+// the phase completes), so a waiting warp issues fewer polling instructions.
+__device__ __forceinline__ uint32_t mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok;
+}
+
+// Suspend-time hint of the polling loop in mbar_wait (0: none).
+#ifndef KVZ_TRYWAIT_HINT_NS
+#define KVZ_TRYWAIT_HINT_NS 0
+#endif
+
 // Bounded wait for the phase of `bar` with the given parity to complete.
 // Returns false if the CTA-wide abort flag is raised or the wait exceeds
 // kWaitLimitNs (then it raises the flag and records KVZ_ERR_TIMEOUT).
@@ -68,7 +88,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   const uint64_t t0 = globaltimer_ns();
   uint32_t it = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (KVZ_TRYWAIT_HINT_NS > 0 ? mbar_try_wait_hint(bar, parity, KVZ_TRYWAIT_HINT_NS) : mbar_try_wait(bar, parity))
+      return true;
     if ((++it & 15u) == 0u) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {

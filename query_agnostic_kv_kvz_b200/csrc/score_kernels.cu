@@ -41,6 +41,13 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128);
 #define KVZ_POLY_PER16 2
 #endif
 constexpr int kPolyPer16 = KVZ_POLY_PER16;
+
+// 1: each Q sub-tile's MMAs are issued by its own thread (warp 1: sub-tile
+// 0, warp 3: sub-tile 1), so the two sub-tiles' softmax warpgroups are
+// coupled only through the shared K ring; 0: one thread issues both.
+#ifndef KVZ_LSE_SPLIT_ISSUE
+#define KVZ_LSE_SPLIT_ISSUE 0
+#endif
 static_assert(kPolyPer16 % 2 == 0 && kPolyPer16 >= 0 && kPolyPer16 <= 16, "pairs of exp2");
 
 template <int D>
@@ -59,6 +66,25 @@ struct LseLayout {
 
 
 
+// Row block and (head, group) of pass-1 unit u.  Both orders put a head's
+// later (longer) row blocks first.  Row-block-major is longest-first over
+// the whole grid; head-major keeps the CTAs running at one time on one or
+// two heads, so they share those heads' key tiles in L2 (chosen when the
+// units are nearly equal in length).
+__device__ __forceinline__ void lse_unit(const LseArgs& p, int u, int nblk, int& iblk, int& bg) {
+  if (p.head_major) {
+    const int per_head = nblk * p.G;
+    const int b = u / per_head;
+    const int rem = u - b * per_head;
+    iblk = nblk - 1 - rem / p.G;
+    bg = b * p.G + rem % p.G;
+  } else {
+    const int BG = p.B * p.G;
+    iblk = nblk - 1 - u / BG;
+    bg = u % BG;
+  }
+}
+
 // Descriptor of k-step `k` (16 bf16 of K) of a 128-row tile at `tile`.
 __device__ __forceinline__ uint64_t kstep_desc(const uint8_t* tile, int k) {
   return sdesc_kmajor_sw128(smem_u32(tile + (k >> 2) * kSubBytes64 + (k & 3) * 32));
@@ -66,8 +92,11 @@ __device__ __forceinline__ uint64_t kstep_desc(const uint8_t* tile, int k) {
 
 // ============================================================================
 // Pass 1: lse2 of every input row in [i_begin, i_end).
-// CTA = (head b, group g, 256 input rows = two 128-row sub-tiles).  Blocks
-// are numbered longest-first (rows late in the input see more keys).
+// Unit = (head b, group g, 256 input rows = two 128-row sub-tiles), numbered
+// longest-first (rows late in the input see more keys).  A CTA computes a
+// whole unit, or (units of the partial last wave) one of `nsplit`
+// consecutive ranges of the unit's key tiles, writing its rows' partial
+// (max, sum) for lse_merge_kernel.
 // ============================================================================
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -92,12 +121,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit (longest first) ----
+  // ---- work unit (longest first) and this CTA's range of its key tiles ----
   const int nblk = static_cast<int>(p.rows_pad / 256);
-  const int BG = p.B * p.G;
-  const int u = blockIdx.x;
-  const int iblk = nblk - 1 - u / BG;
-  const int bg = u % BG;
+  const int x = blockIdx.x;
+  const bool split = x >= p.n_full;
+  const int u = split ? p.n_full + (x - p.n_full) / p.nsplit : x;
+  const int part = split ? (x - p.n_full) % p.nsplit : 0;
+  int iblk, bg;
+  lse_unit(p, u, nblk, iblk, bg);
   const int b = bg / p.G;
   const int64_t i0 = p.i_begin + static_cast<int64_t>(iblk) * 256;
   const int64_t row_hi = p.i_end;               // rows >= row_hi are padding
@@ -106,19 +137,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   int nin[2];
   nin[0] = static_cast<int>(i0 / kTile) + 1;
   nin[1] = static_cast<int>((i0 + kTile) / kTile) + 1;
-  const int NT = NC + nin[nq_valid - 1];
+  const int NT = NC + nin[nq_valid - 1];                 // the unit's key tiles: context, then input
+  const int t_lo = split ? static_cast<int>(static_cast<int64_t>(NT) * part / p.nsplit) : 0;
+  const int NL = (split ? static_cast<int>(static_cast<int64_t>(NT) * (part + 1) / p.nsplit) : NT) - t_lo;
 
+  const int n_issuers = KVZ_LSE_SPLIT_ISSUE ? nq_valid : 1;   // threads that commit to k_empty / drain
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < Lay::KST; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
+      mbar_init(&k_empty[s], n_issuers);
     }
     for (int s = 0; s < 4; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], 8);                // 8 softmax warps read each buffer
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, n_issuers);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -143,9 +177,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < Lay::KB; ++kb)
           tma_load_3d(sQ + q * Lay::TILE_BYTES + kb * kSubBytes64, &tmQ, q_full, kb * 64,
                       static_cast<int>(i0 + q * kTile), bg);
-      for (int t = 0; t < NT; ++t) {
-        const int s = t % Lay::KST;
-        const uint32_t use = static_cast<uint32_t>(t / Lay::KST);
+      for (int j = 0; j < NL; ++j) {                   // ring slots follow the local tile index j
+        const int t = t_lo + j;
+        const int s = j % Lay::KST;
+        const uint32_t use = static_cast<uint32_t>(j / Lay::KST);
         if (!mbar_wait(&k_empty[s], (use & 1u) ^ 1u, abort_flag, p.status)) break;
         mbar_arrive_expect_tx(&k_full[s], Lay::TILE_BYTES);
         for (int kb = 0; kb < Lay::KB; ++kb) {
@@ -156,22 +191,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(sK + s * Lay::TILE_BYTES + kb * kSubBytes64, &tmKi, &k_full[s], kb * 64,
                         (t - NC) * kTile, b);
         }
-        issued = t + 1;
+        issued = j + 1;
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
+  } else if (warp == 1 || (KVZ_LSE_SPLIT_ISSUE && warp == 3)) {
+    // ------------------------------------------------ MMA issuer(s)
+    const int q_lo = KVZ_LSE_SPLIT_ISSUE && warp == 3 ? 1 : 0;
+    const int q_hi = KVZ_LSE_SPLIT_ISSUE ? q_lo + 1 : 2;
+    if (lane == 0 && q_lo < nq_valid) {
       uint32_t cnt[2] = {0u, 0u};
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       tc_fence_after();
-      for (int t = 0; ok && t < NT; ++t) {
-        const int s = t % Lay::KST;
-        const uint32_t use = static_cast<uint32_t>(t / Lay::KST);
+      for (int j = 0; ok && j < NL; ++j) {
+        const int t = t_lo + j;
+        const int s = j % Lay::KST;
+        const uint32_t use = static_cast<uint32_t>(j / Lay::KST);
         if (!mbar_wait(&k_full[s], use & 1u, abort_flag, p.status)) break;
         tc_fence_after();
-        for (int q = 0; q < nq_valid; ++q) {
+        for (int q = q_lo; q < q_hi && q < nq_valid; ++q) {
           if (t >= NC && t - NC >= nin[q]) continue;
           const uint32_t buf = cnt[q] & 1u;
           const uint32_t bu = cnt[q] >> 1;
@@ -211,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ctx_tail = static_cast<int>(p.n_c - static_cast<int64_t>(NC - 1) * kTile) - h * 64;
     const int diag_lim = rl - h * 64;                 // diagonal tile: column c visible iff c <= diag_lim
     uint32_t cnt = 0;
-    for (int t = 0; t < NT; ++t) {
+    for (int t = t_lo; t < t_lo + NL; ++t) {
       if (t >= NC && t - NC >= nin[q]) continue;
       const uint32_t buf = cnt & 1u;
       const uint32_t bu = cnt >> 1;
@@ -288,13 +326,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t i = i0 + q * kTile + rl;
     const float m1 = sMerge[(q * kTile + rl) * 2 + 0];
     const float l1 = sMerge[(q * kTile + rl) * 2 + 1];
-    float lse2 = INFINITY;
-    if (q < nq_valid && ok && l1 >= 0.0f && i < row_hi) {
-      const float mm = fmaxf(m, m1);                 // finite: every row sees a key
-      const float ll = (m == -INFINITY ? 0.0f : l * exp2f(m - mm)) + (m1 == -INFINITY ? 0.0f : l1 * exp2f(m1 - mm));
-      lse2 = mm + log2f(ll);
+    const bool good = ok && l1 >= 0.0f;
+    const float mm = fmaxf(m, m1);
+    const float ll = (m == -INFINITY ? 0.0f : l * exp2f(m - mm)) + (m1 == -INFINITY ? 0.0f : l1 * exp2f(m1 - mm));
+    if (split) {
+      // this range's (max, sum) of the row: (-inf, 0) if it saw no key of
+      // the row, sum -1 if the CTA gave up
+      p.part[static_cast<int64_t>(x - p.n_full) * 256 + q * kTile + rl] =
+          !good ? make_float2(-INFINITY, -1.0f) : (mm == -INFINITY ? make_float2(-INFINITY, 0.0f)
+                                                                   : make_float2(mm, ll));
+    } else {
+      float lse2 = INFINITY;
+      if (q < nq_valid && good && i < row_hi) lse2 = mm + log2f(ll);   // finite: every row sees a key
+      p.lse2[static_cast<int64_t>(bg) * p.ld + (i - p.i_begin)] = lse2;
     }
-    p.lse2[static_cast<int64_t>(bg) * p.ld + (i - p.i_begin)] = lse2;
   }
   if (*abort_flag) {
     // Unwinding after a timeout: let this CTA's own copies and MMAs finish
@@ -306,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_for(&k_full[s], static_cast<uint32_t>(t_last / Lay::KST) & 1u, 20000000ull);
       }
     }
-    if (warp == 1 && lane == 0) {
+    if ((warp == 1 || (KVZ_LSE_SPLIT_ISSUE && warp == 3 && nq_valid == 2)) && lane == 0) {
       tc_commit(drain);
       mbar_wait_for(drain, 0, 20000000ull);
     }
@@ -319,6 +364,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Merge the key-range parts of each split unit, in part order (so the
+// result does not depend on which part finished first).  Block = one split
+// unit, thread = one of its 256 rows.
+__global__ void __launch_bounds__(256) lse_merge_kernel(LseArgs p) {
+  const int t_unit = blockIdx.x;
+  const int row = threadIdx.x;
+  const int u = p.n_full + t_unit;
+  const int nblk = static_cast<int>(p.rows_pad / 256);
+  int iblk, bg;
+  lse_unit(p, u, nblk, iblk, bg);
+  const int64_t i = p.i_begin + static_cast<int64_t>(iblk) * 256 + row;
+  const float2* pr = p.part + static_cast<int64_t>(t_unit) * p.nsplit * 256 + row;
+  float mm = -INFINITY;
+  bool bad = false;
+  for (int k = 0; k < p.nsplit; ++k) {
+    const float2 v = pr[static_cast<int64_t>(k) * 256];
+    if (v.y < 0.0f) bad = true;
+    else if (v.y > 0.0f) mm = fmaxf(mm, v.x);
+  }
+  float ll = 0.0f;
+  for (int k = 0; k < p.nsplit; ++k) {
+    const float2 v = pr[static_cast<int64_t>(k) * 256];
+    if (v.y > 0.0f) ll += v.y * exp2f(v.x - mm);
+  }
+  const float lse2 = (bad || i >= p.i_end || !(ll > 0.0f)) ? INFINITY : mm + log2f(ll);
+  p.lse2[static_cast<int64_t>(bg) * p.ld + (i - p.i_begin)] = lse2;
+}
+
 __global__ void fill_f32_kernel(float* x, int64_t n, float v) {
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x)
@@ -328,11 +401,39 @@ __global__ void fill_f32_kernel(float* x, int64_t n, float v) {
 }  // namespace
 
 cudaError_t launch_lse(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, const CUtensorMap& tmKi,
-                       const LseArgs& a, cudaStream_t stream) {
+                       const LseArgs& a_in, cudaStream_t stream) {
+  LseArgs a = a_in;
   const int64_t nblk = a.rows_pad / 256;
-  const int64_t grid = static_cast<int64_t>(a.B) * a.G * nblk;
-  if (grid <= 0 || grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  const int64_t units = static_cast<int64_t>(a.B) * a.G * nblk;
+  if (units <= 0 || units > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  a.n_full = static_cast<int>(units);
+  a.nsplit = 1;
+  // Head-major when a call's row blocks differ in key count by at most 1/8
+  // of the context tiles (row passes much shorter than the context).
+  a.head_major = (a.rows_pad / kTile) * 8 <= (a.n_c + kTile - 1) / kTile ? 1 : 0;
+  int64_t grid = units, r = 0;
   cudaError_t e;
+  if (a.part != nullptr) {
+    // One CTA per SM: the units past the last full wave are split over key
+    // ranges so that the last wave fills the SMs.  The tail holds the
+    // shortest units (row block 0 of the call); a part keeps >= 8 tiles.
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    r = sms > 0 ? units % sms : 0;
+    if (r > 0) {
+      // the shortest tail unit: row block 0 of the call in either order
+      const int64_t nt_min = (a.n_c + kTile - 1) / kTile + a.i_begin / kTile + 1;
+      int64_t s = sms / r;
+      if (s > nt_min / 8) s = nt_min / 8;
+      if (s * r > kLseMaxSplitCtas) s = kLseMaxSplitCtas / r;
+      if (s >= 2) {
+        a.n_full = static_cast<int>(units - r);
+        a.nsplit = static_cast<int>(s);
+        grid = a.n_full + r * s;
+      }
+    }
+  }
   if (d == 128) {
     e = smem_limit_once<lse_kernel<128>>(LseLayout<128>::SMEM);
     if (e != cudaSuccess) return e;
@@ -342,7 +443,12 @@ cudaError_t launch_lse(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, c
     if (e != cudaSuccess) return e;
     lse_kernel<64><<<static_cast<unsigned>(grid), kThreads, LseLayout<64>::SMEM, stream>>>(tmQ, tmKc, tmKi, a);
   }
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.nsplit > 1) {
+    lse_merge_kernel<<<static_cast<unsigned>(r), 256, 0, stream>>>(a);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 cudaError_t launch_fill_f32(float* x, int64_t n, float v, cudaStream_t stream) {

@@ -73,15 +73,21 @@ def test_pass_rejections(lib):
     Q, Kc, Ki = b.get(4 * 512 * 128 * 2), b.get(512 * 128 * 2), b.get(512 * 128 * 2)
     lse = b.get(4 * 512 * 4)
     S = b.get(512 * 4)
+    ws = b.get(lib.kvz_score_lse2_workspace_size())
+
+    def lse2(i0=0, i1=512, ld=512, shift=0, ws_bytes=None, ws_ptr=True):
+        return lib.kvz_score_lse2(vp(Q), vp(Kc), vp(Ki), 1, 4, 512, 512, 128, 0.1, i0, i1, vp(lse), ld,
+                                  vp(ws + shift) if ws_ptr else None,
+                                  lib.kvz_score_lse2_workspace_size() if ws_bytes is None else ws_bytes, None, None)
     # i_begin not a multiple of 256, range outside n_in, ld too small
-    assert lib.kvz_score_lse2(vp(Q), vp(Kc), vp(Ki), 1, 4, 512, 512, 128, 0.1, 100, 512, vp(lse), 512, None,
-                              None) == INVALID
-    assert lib.kvz_score_lse2(vp(Q), vp(Kc), vp(Ki), 1, 4, 512, 512, 128, 0.1, 0, 513, vp(lse), 512, None,
-                              None) == INVALID
-    assert lib.kvz_score_lse2(vp(Q), vp(Kc), vp(Ki), 1, 4, 512, 512, 128, 0.1, 0, 512, vp(lse), 256, None,
-                              None) == INVALID
-    assert lib.kvz_score_lse2(vp(Q), vp(Kc), vp(Ki), 1, 4, 512, 512, 128, 0.1, 0, 512, vp(lse), 510, None,
-                              None) == ALIGN
+    assert lse2(i0=100) == INVALID
+    assert lse2(i1=513) == INVALID
+    assert lse2(ld=256) == INVALID
+    assert lse2(ld=510) == ALIGN
+    # the optional workspace: too small, misaligned
+    assert lse2(ws_bytes=1024) == WS
+    assert lse2(shift=8) == ALIGN
+    assert lib.kvz_score_lse2_workspace_size() >= 256 * 256 * 8
     assert lib.kvz_score_colmax(vp(Q), vp(Kc), 1, 4, 512, 512, 128, 0.1, 256, 128, vp(lse), 512, vp(S), 0, None,
                                 None) == INVALID
     assert lib.kvz_score_colmax(vp(Q), vp(Kc), 1, 4, 512, 512, 128, 0.1, 0, 512, None, 512, vp(S), 0, None,
@@ -171,7 +177,8 @@ def test_score_chunked_rejections(lib):
     Ki, Kit = b.get(B * T * (n_prompt + m) * d * 2), b.get(B * (n_prompt + ml) * d * 2)
     S = b.get(B * n_c * 4)
     need = lib.kvz_score_chunked_workspace_size(B, G, n_c, n_prompt, m)
-    assert need == B * T * G * 512 * 4                     # the full chunks' rows, padded to 256, dominate
+    # the full chunks' rows, padded to 256, dominate; plus pass 1's split-tail scratch
+    assert need == B * T * G * 512 * 4 + lib.kvz_score_lse2_workspace_size()
     ws = b.get(need)
 
     def call(q=Q, qt=Qt, d_=d, m_=m, wsb=need, scale=0.1):

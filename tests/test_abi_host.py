@@ -63,10 +63,12 @@ def test_keep_count_rejects_bad_ratio(kvz):
 
 
 def test_score_workspace_size(kvz):
-    # one chunk of rows, padded to 256, fp32, times B*G
-    assert kvz.kvz_score_workspace_size(8, 4, 8224, 0) == 8 * 4 * 8448 * 4
-    assert kvz.kvz_score_workspace_size(384, 5, 131104, 4096) == 384 * 5 * 4096 * 4
-    assert kvz.kvz_score_workspace_size(1, 1, 1, 0) == 256 * 4
+    # one chunk of rows, padded to 256, fp32, times B*G; then pass 1's split-tail scratch
+    part = kvz.kvz_score_lse2_workspace_size()
+    assert part == 256 * 256 * 8
+    assert kvz.kvz_score_workspace_size(8, 4, 8224, 0) == 8 * 4 * 8448 * 4 + part
+    assert kvz.kvz_score_workspace_size(384, 5, 131104, 4096) == 384 * 5 * 4096 * 4 + part
+    assert kvz.kvz_score_workspace_size(1, 1, 1, 0) == 256 * 4 + part
     assert kvz.kvz_score_workspace_size(1, 1, 10, 100) == 0      # chunk not a multiple of 256
     assert kvz.kvz_score_workspace_size(0, 1, 10, 0) == 0
 
