@@ -285,6 +285,70 @@ def test_compact_in_place_structured(pattern):
         np.testing.assert_array_equal(Ko[b, c:], Kh[b, c:])
 
 
+def _pattern_selection(rng, kind, n_c):
+    """Ascending kept positions of one head for a selection pattern."""
+    if kind == "random":
+        keep = rng.random(n_c) < rng.choice([0.02, 0.25, 0.5, 0.9])
+    elif kind == "runs":                   # alternating kept / dropped runs of random lengths
+        keep, pos, on = np.zeros(n_c, bool), 0, bool(rng.integers(2))
+        mean = rng.choice([1.5, 8, 60, 400])
+        while pos < n_c:
+            L = 1 + int(rng.geometric(1.0 / mean))
+            keep[pos:pos + L] = on
+            pos, on = pos + L, not on
+    elif kind == "tail":
+        keep = np.arange(n_c) >= rng.integers(0, n_c)
+    elif kind == "head":
+        keep = np.arange(n_c) < rng.integers(0, n_c + 1)
+    elif kind == "all":
+        keep = np.ones(n_c, bool)
+    else:                                  # none
+        keep = np.zeros(n_c, bool)
+    return np.nonzero(keep)[0].astype(np.int32)
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_compact_in_place_pattern_sweep(seed):
+    """In-place compaction over seeded structured selections (its ordering
+    wait is what keeps a row from being overwritten before it is read):
+    every pattern of every head against the oracle, with every dropped row a
+    sentinel that must never reach the kept prefix."""
+    rng = np.random.default_rng(1000 + seed)
+    B = [1, 3, 7][seed % 3]
+    n_c = [17, 1000, 4097, 20000][seed % 4]
+    d = [64, 128][(seed // 4) % 2]
+    kinds = ["random", "runs", "tail", "head", "all", "none"]
+    sels = [_pattern_selection(rng, kinds[(seed + b) % len(kinds)] if b else "runs", n_c) for b in range(B)]
+    counts_h = np.array([len(x) for x in sels], np.int32)
+    offsets_h = np.zeros(B + 1, np.int64)
+    offsets_h[1:] = np.cumsum(counts_h)
+    idx_h = np.concatenate(sels).astype(np.int32) if offsets_h[-1] else np.zeros(1, np.int32)
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    K = torch.randn((B, n_c, d), generator=g, device="cuda").to(torch.bfloat16)
+    V = torch.randn((B, n_c, d), generator=g, device="cuda").to(torch.bfloat16)
+    for b in range(B):
+        drop = np.setdiff1d(np.arange(n_c), sels[b])
+        if drop.size:
+            dt = torch.from_numpy(drop).cuda()
+            K.view(torch.int16)[b, dt] = 0x7FC1
+            V.view(torch.int16)[b, dt] = 0x7FC1
+    Kh, Vh = bits(K), bits(V)
+    rk, rv = orc.compact(Kh, Vh, idx_h, counts_h, offsets_h)
+    idx, counts, offsets = (torch.from_numpy(idx_h).cuda(), torch.from_numpy(counts_h).cuda(),
+                            torch.from_numpy(offsets_h).cuda())
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvz.kvz_compact(K, V, idx, counts, offsets, in_place=True, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    Ko, Vo = bits(K), bits(V)
+    for b in range(B):
+        c = int(counts_h[b])
+        np.testing.assert_array_equal(Ko[b, :c], rk[offsets_h[b]:offsets_h[b] + c])
+        np.testing.assert_array_equal(Vo[b, :c], rv[offsets_h[b]:offsets_h[b] + c])
+        np.testing.assert_array_equal(Ko[b, c:], Kh[b, c:])
+        assert not np.any(Ko[b, :c] == 0x7FC1) and not np.any(Vo[b, :c] == 0x7FC1)
+
+
 # ---------------------------------------------------------------------------
 # The whole path on the two small workloads
 # ---------------------------------------------------------------------------
