@@ -48,12 +48,6 @@ constexpr int kPolyPer16 = KVZ_POLY_PER16;
 #ifndef KVZ_LSE_SPLIT_ISSUE
 #define KVZ_LSE_SPLIT_ISSUE 0
 #endif
-
-// 1: a tile's exp2s are computed against the running reference while its
-// max is found (see the softmax loop); 0: the max first, then the exp2s.
-#ifndef KVZ_LSE_SPECULATE
-#define KVZ_LSE_SPECULATE 0
-#endif
 static_assert(kPolyPer16 % 2 == 0 && kPolyPer16 >= 0 && kPolyPer16 <= 16, "pairs of exp2");
 
 template <int D>
@@ -264,78 +258,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-#if KVZ_LSE_SPECULATE
-      // The tile's exp2s are taken against the current reference m while
-      // its max is found (both in one block, so the SFU work does not wait
-      // for the max).  A row with no reference yet, or whose tile max exceeds
-      // m + 120 (its exp2s could overflow), takes the tile again against the
-      // tile max, reloaded from tensor memory (the decision is warp-uniform:
-      // tcgen05.ld is a warp collective); otherwise a max above m + 8 rebases
-      // the sum.  The buffer is released once the tile is done.
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(wq * 32) << 16) +
-                             static_cast<uint32_t>((q * 2 + buf) * kTile + h * 64);
-      bool done = false;
-#pragma unroll 1
-      for (int pass = 0; pass < 2; ++pass) {
-        float v[64];
-        tmem_ld64(taddr, v);
-        if (t == NC - 1 && ctx_tail < 64) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c >= ctx_tail) v[c] = -INFINITY;
-        }
-        if (t >= NC && t - NC == nin[q] - 1) {     // diagonal input tile
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c > diag_lim) v[c] = -INFINITY;
-        }
-        float mx[2];
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          float a = v[32 * k];
-#pragma unroll
-          for (int c = 1; c < 31; c += 2) a = fmax3(a, v[32 * k + c], v[32 * k + c + 1]);
-          mx[k] = fmaxf(a, v[32 * k + 31]);
-        }
-        const float2 c22 = make_float2(c2, c2);
-        const float2 nm2 = make_float2(-m, -m);
-        float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0;
-#pragma unroll
-        for (int c = 0; c < 64; c += 16) {
-#pragma unroll
-          for (int k = 0; k < 16 - kPolyPer16; k += 2) {
-            const float2 x = __ffma2_rn(make_float2(v[c + k], v[c + k + 1]), c22, nm2);
-            const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            if (k & 2) s0 = __fadd2_rn(s0, e); else s1 = __fadd2_rn(s1, e);
-          }
-#pragma unroll
-          for (int k = 16 - kPolyPer16; k < 16; k += 2) {
-            const float2 x = __ffma2_rn(make_float2(v[c + k], v[c + k + 1]), c22, nm2);
-            s2 = __fadd2_rn(s2, exp2_poly2(x));
-          }
-        }
-        if (!done) {
-          const float mt = fmaxf(mx[0], mx[1]) * c2;
-          if (m != -INFINITY && !(mt > m + 120.0f)) {
-            l += ((s0.x + s0.y) + (s1.x + s1.y)) + (s2.x + s2.y);
-            if (mt > m + 8.0f) {
-              l *= ex2_approx(m - mt);
-              m = mt;
-            }
-            done = true;
-          } else if (mt == -INFINITY) {
-            done = true;                              // nothing visible here and no reference yet
-          } else {
-            l = m == -INFINITY ? 0.0f : l * ex2_approx(m - mt);
-            m = mt;
-          }
-        }
-        if (__all_sync(0xffffffffu, done)) break;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[q * 2 + buf]);
-#else
       float v[64];
       tmem_ld64(tmem + (static_cast<uint32_t>(wq * 32) << 16) +
                     static_cast<uint32_t>((q * 2 + buf) * kTile + h * 64), v);
@@ -391,7 +313,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l += ((s0.x + s0.y) + (s1.x + s1.y)) + (s2.x + s2.y);
       }
-#endif
       ++cnt;
     }
   }
