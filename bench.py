@@ -703,6 +703,19 @@ def run_decode(w, c, kvz, dev, stream, status, scale, nums):
                     "buffer" % (B, w.G, kept_rows)}
 
 
+def lse_launches(B, G, n_c, i_begin, rows, sms):
+    """Kernels one pass-1 call launches: lse_kernel, plus lse_merge_kernel
+    when the grid's partial last wave is split (launch_lse's rule)."""
+    units = B * G * ((rows + 255) // 256)
+    r = units % sms
+    if r == 0:
+        return 1
+    s = min(sms // r, ((n_c + 127) // 128 + i_begin // 128 + 1) // 8)
+    if s * r > 256:
+        s = 256 // r
+    return 2 if s >= 2 else 1
+
+
 class Context:
     """Device-resident inputs and outputs of one context of a workload: all
     layers' Q / K_in, the whole K/V cache (and, when it is compacted in
@@ -777,10 +790,14 @@ class Context:
         per_head_one = w.mode == "per_head" and (self.n_c <= 49152 or B >= 128)
         # head level: fill + head max, one-segment selection (1 launch up to 49152 heads), csr + idx
         sel = 1 if per_head_one else (5 if w.mode == "heads" else 10)
-        if w.chunk:
-            self.launches = L * (2 * self.score_launches + 1) + sel + (3 if w.in_place else 1)
-        else:
-            self.launches = L * (2 * len(self.chunks) + 1) + sel + (3 if w.in_place else 1)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        if w.chunk:   # per layer: fill, then for the full chunks and the tail: pass 1 (+ merge) and pass 2
+            T, tail = self.n_c // w.chunk, self.n_c % w.chunk
+            per_layer = 1 + (lse_launches(H * T, G, w.chunk, 0, w.n_prompt + w.chunk, sms) + 1 if T else 0) + \
+                (lse_launches(H, G, tail, 0, w.n_prompt + tail, sms) + 1 if tail else 0)
+        else:         # per layer: fill, then per row pass: pass 1 (+ merge) and pass 2
+            per_layer = 1 + sum(lse_launches(H, G, self.n_c, i0, i1 - i0, sms) + 1 for i0, i1 in self.chunks)
+        self.launches = L * per_layer + sel + (3 if w.in_place else 1)
 
     def restore(self):
         if self.K0 is not None:

@@ -139,11 +139,22 @@ def check_sampled_rows(r, w, layer, head, rows, groups):
 
 
 def check_whole_head(r, w, layer, head):
-    """Every score of head (layer, head) against the oracle, two-sided."""
+    """Every score of head (layer, head) against the oracle, two-sided.  In
+    per-head mode also the index-set overlap (Jaccard) of the GPU's kept
+    keys with the oracle's selection from its own fp64 scores: reported,
+    and required to be near 1 (near-ties at the threshold may differ)."""
     x = r["kept"][layer]
     ref = oracle_head_rows_parallel(x["Q"][head], x["K_ctx"][head], x["K_in"][head], r["scale"])
     b = layer * w.H + head
     assert_scores_close(r["S"][b].cpu().numpy(), ref, "%s layer %d head %d" % (w.name, layer, head))
+    if w.mode == "per_head":
+        oi, _, _ = orc.select(ref[None, :].astype(np.float32), w.ratio, "per_head")
+        o0, o1 = int(r["offsets"][b].item()), int(r["offsets"][b + 1].item())
+        gpu = set(r["idx"][o0:o1].cpu().tolist())
+        ora = set(int(v) for v in oi)
+        jac = len(gpu & ora) / max(1, len(gpu | ora))
+        print("selection overlap %s layer %d head %d: Jaccard %.6f over %d kept" % (w.name, layer, head, jac, len(ora)))
+        assert jac >= 0.99, jac
 
 
 def planter(rows_keys, alpha=1.8):
