@@ -562,11 +562,14 @@ def run_e2e(w, ctxs, kvz, dev, stream, status, scale, ms_step):
     k = kvz.kvz_keep_count(c.n_c if per_layer else Bc * c.n_c, w.ratio)
     kept = Bc * k if per_layer else k
     out_bytes = kept * (4 + 2 * row) + Bc * 4 + (Bc + 1) * 8
+    # host memory for the page-locked inputs: 60% of what is available,
+    # shared by the ranks of this node
+    local_ranks = max(1, int(os.environ.get("LOCAL_WORLD_SIZE", os.environ.get("WORLD_SIZE", "1"))))
     try:
         import psutil
-        budget = int(0.60 * psutil.virtual_memory().available)
+        budget = int(0.60 * psutil.virtual_memory().available) // local_ranks
     except Exception:
-        budget = 8 << 30
+        budget = (8 << 30) // local_ranks
     n_host = max(1, min(calls, (budget - 2 * out_bytes) // in_bytes))
     if n_host < calls and not per_layer:
         return None
