@@ -48,6 +48,16 @@ constexpr int kPolyPer16 = KVZ_POLY_PER16;
 #ifndef KVZ_LSE_SPLIT_ISSUE
 #define KVZ_LSE_SPLIT_ISSUE 0
 #endif
+
+// 1: no per-tile max.  A row's reference is the floor of its first tile's
+// max (an integer, so rebasing by powers of two keeps it exact); each tile's
+// exp2s are taken against it directly, the sum is renormalised to [1, 2)
+// with an exact power of two once it reaches 2^24, and only a tile whose
+// terms overflow is reloaded and redone against its own max.  0: the tile
+// max first, the reference moved when it grows by more than 8.
+#ifndef KVZ_LSE_NOMAX
+#define KVZ_LSE_NOMAX 0
+#endif
 static_assert(kPolyPer16 % 2 == 0 && kPolyPer16 >= 0 && kPolyPer16 <= 16, "pairs of exp2");
 
 template <int D>
@@ -83,6 +93,50 @@ __device__ __forceinline__ void lse_unit(const LseArgs& p, int u, int nblk, int&
     iblk = nblk - 1 - u / BG;
     bg = u % BG;
   }
+}
+
+// Max of a thread's 64 logits of a tile (two independent chains of 3-input
+// max).
+__device__ __forceinline__ float tile_max64(const float (&v)[64]) {
+  float mx[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    float a = v[32 * k];
+#pragma unroll
+    for (int c = 1; c < 31; c += 2) a = fmax3(a, v[32 * k + c], v[32 * k + c + 1]);
+    mx[k] = fmaxf(a, v[32 * k + 31]);
+  }
+  return fmaxf(mx[0], mx[1]);
+}
+
+// Sum over a thread's 64 logits of 2^(c2 * s - m): 16 - kPolyPer16 of every
+// 16 exp2 on the SFU, the rest on the FMA pipe as a polynomial, so neither
+// unit limits the pass on its own.
+__device__ __forceinline__ float exp2_sum64(const float (&v)[64], float c2, float m) {
+  const float2 c22 = make_float2(c2, c2);
+  const float2 nm2 = make_float2(-m, -m);
+  float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0;
+#pragma unroll
+  for (int c = 0; c < 64; c += 16) {
+#pragma unroll
+    for (int k = 0; k < 16 - kPolyPer16; k += 2) {
+      const float2 x = __ffma2_rn(make_float2(v[c + k], v[c + k + 1]), c22, nm2);
+      const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      if (k & 2) s0 = __fadd2_rn(s0, e); else s1 = __fadd2_rn(s1, e);
+    }
+#pragma unroll
+    for (int k = 16 - kPolyPer16; k < 16; k += 2) {
+      const float2 x = __ffma2_rn(make_float2(v[c + k], v[c + k + 1]), c22, nm2);
+      s2 = __fadd2_rn(s2, exp2_poly2(x));
+    }
+  }
+  return ((s0.x + s0.y) + (s1.x + s1.y)) + (s2.x + s2.y);
+}
+
+// 2^n for an integer-valued n <= 0, exactly (0 below the normal range).
+__device__ __forceinline__ float exp2_int_nonpos(float n) {
+  const int e = static_cast<int>(n) + 127;
+  return e > 0 ? __int_as_float(e << 23) : 0.0f;
 }
 
 // Descriptor of k-step `k` (16 bf16 of K) of a 128-row tile at `tile`.
@@ -258,32 +312,74 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(wq * 32) << 16) +
+                             static_cast<uint32_t>((q * 2 + buf) * kTile + h * 64);
+      const bool tail_tile = t == NC - 1 && ctx_tail < 64;
+      const bool diag_tile = t >= NC && t - NC == nin[q] - 1;
       float v[64];
-      tmem_ld64(tmem + (static_cast<uint32_t>(wq * 32) << 16) +
-                    static_cast<uint32_t>((q * 2 + buf) * kTile + h * 64), v);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[q * 2 + buf]);
-      if (t == NC - 1 && ctx_tail < 64) {
+      tmem_ld64(taddr, v);
+#if KVZ_LSE_NOMAX
+      if (tail_tile) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
           if (c >= ctx_tail) v[c] = -INFINITY;
       }
-      if (t >= NC && t - NC == nin[q] - 1) {       // diagonal input tile
+      if (diag_tile) {                             // diagonal input tile
 #pragma unroll
         for (int c = 0; c < 64; ++c)
           if (c > diag_lim) v[c] = -INFINITY;
       }
-      // tile max: two independent chains of 3-input max
-      float mx[2];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        float a = v[32 * k];
-#pragma unroll
-        for (int c = 1; c < 31; c += 2) a = fmax3(a, v[32 * k + c], v[32 * k + c + 1]);
-        mx[k] = fmaxf(a, v[32 * k + 31]);
+      if (m == -INFINITY) {                        // no reference yet: this tile's max, floored
+        const float mt = tile_max64(v) * c2;
+        if (mt != -INFINITY) m = floorf(mt);
       }
-      const float mt = fmaxf(mx[0], mx[1]) * c2;
+      float l_new = m == -INFINITY ? l : l + exp2_sum64(v, c2, m);
+      // A term overflowed (a logit ~100 or more above the row's reference):
+      // reload the tile (warp-uniform: tcgen05.ld is a warp collective) and
+      // redo those rows against the tile's own max.
+      if (__any_sync(0xffffffffu, !(l_new <= 0x1p100f))) {
+        tmem_ld64(taddr, v);
+        if (tail_tile) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c >= ctx_tail) v[c] = -INFINITY;
+        }
+        if (diag_tile) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c > diag_lim) v[c] = -INFINITY;
+        }
+        if (!(l_new <= 0x1p100f)) {
+          const float mn = floorf(tile_max64(v) * c2);
+          l = l * exp2_int_nonpos(m - mn);
+          m = mn;
+          l_new = l + exp2_sum64(v, c2, m);
+        }
+      }
+      l = l_new;
+      if (l >= 0x1p24f) {                          // renormalise to [1, 2): exact
+        const int k = ((__float_as_int(l) >> 23) & 0xff) - 127;
+        l = __int_as_float(__float_as_int(l) - (k << 23));
+        m += static_cast<float>(k);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[q * 2 + buf]);
+#else
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[q * 2 + buf]);
+      if (tail_tile) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c >= ctx_tail) v[c] = -INFINITY;
+      }
+      if (diag_tile) {                             // diagonal input tile
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c > diag_lim) v[c] = -INFINITY;
+      }
+      const float mt = tile_max64(v) * c2;
       // Move the reference max only when it grows by more than 2^8; the
       // sum is exact for any reference, and values stay below 2^8.  A half
       // that is fully masked (mt = -inf) changes nothing.
@@ -291,28 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= ex2_approx(m - mt);
         m = mt;
       }
-      if (m != -INFINITY) {
-        // 2^(c2*s - m): 16 - kPolyPer16 of every 16 on the SFU, the rest on
-        // the FMA pipe, so neither unit limits the pass on its own.
-        const float2 c22 = make_float2(c2, c2);
-        const float2 nm2 = make_float2(-m, -m);
-        float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0;
-#pragma unroll
-        for (int c = 0; c < 64; c += 16) {
-#pragma unroll
-          for (int k = 0; k < 16 - kPolyPer16; k += 2) {
-            const float2 x = __ffma2_rn(make_float2(v[c + k], v[c + k + 1]), c22, nm2);
-            const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            if (k & 2) s0 = __fadd2_rn(s0, e); else s1 = __fadd2_rn(s1, e);
-          }
-#pragma unroll
-          for (int k = 16 - kPolyPer16; k < 16; k += 2) {
-            const float2 x = __ffma2_rn(make_float2(v[c + k], v[c + k + 1]), c22, nm2);
-            s2 = __fadd2_rn(s2, exp2_poly2(x));
-          }
-        }
-        l += ((s0.x + s0.y) + (s1.x + s1.y)) + (s2.x + s2.y);
-      }
+      if (m != -INFINITY) l += exp2_sum64(v, c2, m);
+#endif
       ++cnt;
     }
   }
