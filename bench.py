@@ -626,11 +626,13 @@ def run_e2e(w, ctxs, kvz, dev, stream, status, scale, ms_step):
         ms = e0.elapsed_time(e1) / steps
         h2d = calls * in_bytes
         d2h = calls * out_bytes
+        held = ("%d distinct host layer(s)%s" % (n_host, "" if n_host == calls else
+                                                  " cycled (host memory holds %d of %d)" % (n_host, calls))
+                if per_layer else "the whole context's inputs in host memory")
         how = ("kvz_compress_host %s (%d heads per call, %d call(s) per step, %d timed step(s)): inputs copied in "
                "from page-locked host memory by head chunks overlapping the scoring, selection and out-of-place "
-               "compaction on the device, kept rows / indices copied back; %d distinct host layer(s)%s"
-               % ("per layer" if per_layer else "for the whole context", Bc, calls, steps, n_host,
-                  "" if n_host == calls else " cycled (host memory holds %d of %d)" % (n_host, calls)))
+               "compaction on the device, kept rows / indices copied back; %s"
+               % ("per layer" if per_layer else "for the whole context", Bc, calls, steps, held))
         return {"ms": ms, "h2d": h2d, "d2h": d2h, "how": how}
     finally:
         torch.cuda.synchronize(dev)

@@ -48,16 +48,6 @@ constexpr int kPolyPer16 = KVZ_POLY_PER16;
 #ifndef KVZ_LSE_SPLIT_ISSUE
 #define KVZ_LSE_SPLIT_ISSUE 0
 #endif
-
-// 1: no per-tile max.  A row's reference is the floor of its first tile's
-// max (an integer, so rebasing by powers of two keeps it exact); each tile's
-// exp2s are taken against it directly, the sum is renormalised to [1, 2)
-// with an exact power of two once it reaches 2^24, and only a tile whose
-// terms overflow is reloaded and redone against its own max.  0: the tile
-// max first, the reference moved when it grows by more than 8.
-#ifndef KVZ_LSE_NOMAX
-#define KVZ_LSE_NOMAX 0
-#endif
 static_assert(kPolyPer16 % 2 == 0 && kPolyPer16 >= 0 && kPolyPer16 <= 16, "pairs of exp2");
 
 template <int D>
@@ -111,11 +101,14 @@ __device__ __forceinline__ float tile_max64(const float (&v)[64]) {
 
 // Sum over a thread's 64 logits of 2^(c2 * s - m): 16 - kPolyPer16 of every
 // 16 exp2 on the SFU, the rest on the FMA pipe as a polynomial, so neither
-// unit limits the pass on its own.
-__device__ __forceinline__ float exp2_sum64(const float (&v)[64], float c2, float m) {
+// unit limits the pass on its own.  `pmax` gets the largest polynomial
+// input: the polynomial builds 2^n in the exponent bits and is only valid
+// for inputs up to 127 (the SFU returns +inf above its range).
+__device__ __forceinline__ float exp2_sum64(const float (&v)[64], float c2, float m, float& pmax) {
   const float2 c22 = make_float2(c2, c2);
   const float2 nm2 = make_float2(-m, -m);
   float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0;
+  float pm = -INFINITY;
 #pragma unroll
   for (int c = 0; c < 64; c += 16) {
 #pragma unroll
@@ -127,9 +120,11 @@ __device__ __forceinline__ float exp2_sum64(const float (&v)[64], float c2, floa
 #pragma unroll
     for (int k = 16 - kPolyPer16; k < 16; k += 2) {
       const float2 x = __ffma2_rn(make_float2(v[c + k], v[c + k + 1]), c22, nm2);
+      pm = fmax3(pm, x.x, x.y);
       s2 = __fadd2_rn(s2, exp2_poly2(x));
     }
   }
+  pmax = pm;
   return ((s0.x + s0.y) + (s1.x + s1.y)) + (s2.x + s2.y);
 }
 
@@ -290,7 +285,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------ softmax warpgroups
   // Four warpgroups: (sub-tile q, column half h).  A thread owns one query
   // row (its TMEM lane) and 64 of the 128 key columns of every tile; the
-  // two halves' (max, sum) pairs merge exactly at the end.
+  // two halves' (reference, sum) pairs merge exactly at the end.
+  // No per-tile max: a row's reference m is the floor of its first tile's
+  // max (an integer, so rebasing by powers of two keeps it exact); each
+  // tile's exp2s are taken against m directly (the sum is exact for any
+  // reference), the sum is renormalised to [1, 2) by an exact power of two
+  // once it reaches 2^24, and only a tile with a logit about 100 or more
+  // above m (log2 units: its terms overflow, or leave the polynomial's
+  // range) is reloaded and redone against its own max.  The tile's
+  // accumulator buffer is released after the tile.
   const int ew = warp - 4;
   const int q = (ew >> 3) & 1;
   const int h = (ew >> 2) & 1;
@@ -318,7 +321,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool diag_tile = t >= NC && t - NC == nin[q] - 1;
       float v[64];
       tmem_ld64(taddr, v);
-#if KVZ_LSE_NOMAX
       if (tail_tile) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
@@ -333,11 +335,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mt = tile_max64(v) * c2;
         if (mt != -INFINITY) m = floorf(mt);
       }
-      float l_new = m == -INFINITY ? l : l + exp2_sum64(v, c2, m);
-      // A term overflowed (a logit ~100 or more above the row's reference):
-      // reload the tile (warp-uniform: tcgen05.ld is a warp collective) and
-      // redo those rows against the tile's own max.
-      if (__any_sync(0xffffffffu, !(l_new <= 0x1p100f))) {
+      float pmax = -INFINITY;
+      float l_new = m == -INFINITY ? l : l + exp2_sum64(v, c2, m, pmax);
+      // A term overflowed, or a polynomial input left its range (a logit
+      // ~100 or more above the row's reference): reload the tile
+      // (warp-uniform: tcgen05.ld is a warp collective) and redo those rows
+      // against the tile's own max.
+      bool redo = !(l_new <= 0x1p100f) || pmax > 100.0f;
+      if (__any_sync(0xffffffffu, redo)) {
         tmem_ld64(taddr, v);
         if (tail_tile) {
 #pragma unroll
@@ -349,11 +354,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 64; ++c)
             if (c > diag_lim) v[c] = -INFINITY;
         }
-        if (!(l_new <= 0x1p100f)) {
+        if (redo) {
           const float mn = floorf(tile_max64(v) * c2);
           l = l * exp2_int_nonpos(m - mn);
           m = mn;
-          l_new = l + exp2_sum64(v, c2, m);
+          l_new = l + exp2_sum64(v, c2, m, pmax);   // inputs now at most 1
         }
       }
       l = l_new;
@@ -365,30 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[q * 2 + buf]);
-#else
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[q * 2 + buf]);
-      if (tail_tile) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c >= ctx_tail) v[c] = -INFINITY;
-      }
-      if (diag_tile) {                             // diagonal input tile
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c > diag_lim) v[c] = -INFINITY;
-      }
-      const float mt = tile_max64(v) * c2;
-      // Move the reference max only when it grows by more than 2^8; the
-      // sum is exact for any reference, and values stay below 2^8.  A half
-      // that is fully masked (mt = -inf) changes nothing.
-      if (mt > m + 8.0f) {
-        l *= ex2_approx(m - mt);
-        m = mt;
-      }
-      if (m != -INFINITY) l += exp2_sum64(v, c2, m);
-#endif
       ++cnt;
     }
   }

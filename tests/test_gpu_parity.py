@@ -126,6 +126,25 @@ def test_identical_keys_closed_form():
     assert np.abs(S - 1.0 / (n_c + 1)).max() <= 1e-4 / (n_c + 1) + 1e-9
 
 
+@pytest.mark.parametrize("alpha,j", [(6.0, 5000), (12.0, 7950), (25.0, 3000), (12.0, 4110), (40.0, 8000)])
+def test_score_extreme_logit_jumps(alpha, j):
+    """Pass 1 keeps no per-tile max: a row's reference comes from its first
+    tile, and a tile with a logit far above it (terms that overflow, or leave
+    the exp2 polynomial's range) is redone against its own max.  Plant a key
+    alpha * q_r in a late tile, on an SFU column (j % 16 < 14) or a
+    polynomial column (j % 16 >= 14), for logit jumps of roughly 60 to 200
+    in log2 units; every score must still match the oracle."""
+    B, G, n_c, n_prompt, d = 1, 2, 8192, 40, 128
+    x = _inputs(B, G, n_c, n_prompt, d, seed=int(alpha * 100) + j)
+    K = x["K_ctx"].clone()
+    K[0, j] = (alpha * x["Q"][0, 1, 300].float()).to(torch.bfloat16)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    S = kvz.kvz_score(x["Q"], K, x["K_in"], scale=scale)
+    ref = oracle_scores(x["Q"], K, x["K_in"], scale)
+    assert_scores_close(S.cpu().numpy(), ref, "alpha %g key %d" % (alpha, j))
+    assert ref[0, j] > 0.99                    # the planted key dominates its row
+
+
 def test_score_is_deterministic():
     x = _inputs(3, 4, 2000, 32, 128, seed=5)
     S0 = kvz.kvz_score(x["Q"], x["K_ctx"], x["K_in"])
