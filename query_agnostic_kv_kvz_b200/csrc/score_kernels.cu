@@ -8,8 +8,9 @@
 //   A[r, j] = 2^(c2 <q_r, k_j> - lse2_r)  and, exp2 being monotone,
 //   S[j]    = 2^( max_r (c2 <q_r, k_j> - lse2_r) ).
 // Two passes, neither materialising the G*n_in x (n_c+n_in) matrix:
-//   pass 1 (lse_kernel):    one thread per query row, online max / sum over
-//                           key tiles (FlashAttention-style, no P.V);
+//   pass 1 (lse_kernel):    one thread per query row, a running sum of
+//                           exp2 against a per-row reference over key tiles
+//                           (no P.V, no per-tile max);
 //   pass 2 (colmax_kernel): keys in TMEM lanes, one thread per context key,
 //                           running max over query-row columns; no mask
 //                           because every row sees every context key.
