@@ -36,8 +36,9 @@ cudaError_t smem_limit_once(int bytes) {
 // last r units (the partial last wave) may each be split into `nsplit`
 // CTAs over consecutive key-tile ranges.  CTA x < n_full computes unit x
 // whole; CTA n_full + t computes part t % nsplit of unit n_full + t / nsplit
-// and writes its rows' partial (max, sum) to part[t * 256 + row]; a merge
-// kernel then combines the parts of each unit in order.
+// and writes its rows' partial (reference m, sum of 2^(c2 s - m)) to
+// part[t * 256 + row]; a merge kernel then combines the parts of each unit
+// in order.
 struct LseArgs {
   int B, G, T;
   int64_t n_c, n_in;
@@ -47,7 +48,7 @@ struct LseArgs {
   int32_t* status;
   int n_full;               // CTAs that compute a whole unit (set by launch_lse)
   int nsplit;               // parts per split unit, 1 = none (set by launch_lse)
-  float2* part;             // [split CTAs][256] partial (max, sum); null = no split
+  float2* part;             // [split CTAs][256] partial (reference, sum); null = no split
   int head_major;           // unit order: 0 = row block, then (head, group); 1 = head, then row block, then
                             // group (set by launch_lse)
 };
