@@ -42,13 +42,6 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128);
 #define KVZ_POLY_PER16 2
 #endif
 constexpr int kPolyPer16 = KVZ_POLY_PER16;
-// The same count for the odd 16-column groups of a tile half (even groups
-// use kPolyPer16), for shares between the even steps.
-#ifndef KVZ_POLY_PER16_ODD
-#define KVZ_POLY_PER16_ODD KVZ_POLY_PER16
-#endif
-constexpr int kPolyPer16Odd = KVZ_POLY_PER16_ODD;
-static_assert(kPolyPer16Odd % 2 == 0 && kPolyPer16Odd >= 0 && kPolyPer16Odd <= 16, "pairs of exp2");
 
 // 1: each Q sub-tile's MMAs are issued by its own thread (warp 1: sub-tile
 // 0, warp 3: sub-tile 1), so the two sub-tiles' softmax warpgroups are
@@ -119,15 +112,14 @@ __device__ __forceinline__ float exp2_sum64(const float (&v)[64], float c2, floa
   float pm = -INFINITY;
 #pragma unroll
   for (int c = 0; c < 64; c += 16) {
-    const int npoly = (c / 16) % 2 ? kPolyPer16Odd : kPolyPer16;
 #pragma unroll
-    for (int k = 0; k < 16 - npoly; k += 2) {
+    for (int k = 0; k < 16 - kPolyPer16; k += 2) {
       const float2 x = __ffma2_rn(make_float2(v[c + k], v[c + k + 1]), c22, nm2);
       const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
       if (k & 2) s0 = __fadd2_rn(s0, e); else s1 = __fadd2_rn(s1, e);
     }
 #pragma unroll
-    for (int k = 16 - npoly; k < 16; k += 2) {
+    for (int k = 16 - kPolyPer16; k < 16; k += 2) {
       const float2 x = __ffma2_rn(make_float2(v[c + k], v[c + k + 1]), c22, nm2);
       pm = fmax3(pm, x.x, x.y);
       s2 = __fadd2_rn(s2, exp2_poly2(x));
