@@ -258,28 +258,35 @@ def run_reference(args, w, config, rank, world):
             dist.barrier()
             dist.destroy_process_group()
         return
-    n_c, n_in = w.n_c[0], w.n_in(0)
-    x = synth.layer_inputs(w, seed=0, device="cpu")
+    n_ctx = len(w.n_c)
+    xs = [synth.layer_inputs(w, ctx=c, seed=0, device="cpu") for c in range(n_ctx)]
     steps, warm = max(1, args.steps), max(0, args.warmup)
-    # a step is sized to a few seconds so that --steps 20 --warmup 5 ends in minutes
-    target = 2.0 if n_c * n_in * w.G > 1e9 else 1.0
-    rates, threads, desc = [], 1, ""
+    # a step is sized to a few seconds so that --steps 20 --warmup 5 ends in
+    # minutes; steps cycle over the contexts (a ragged batch), then the heads
+    rates = [[] for _ in range(n_ctx)]
+    threads, desc = 1, ""
     for s in range(warm + steps):
-        h = s % w.H
+        c, h = s % n_ctx, (s // n_ctx) % w.H
+        n_c, n_in = w.n_c[c], w.n_in(c)
+        target = 2.0 if n_c * n_in * w.G > 1e9 else 1.0
         frac = ((s * 0.381966) % 1.0) * 0.98            # spread the sampled row blocks over the input
-        rate, threads, desc, _ = oracle_head_sample(head_bits_of(x, h), w, n_c, n_in, target, 4 * target,
+        rate, threads, desc, _ = oracle_head_sample(head_bits_of(xs[c], h), w, n_c, n_in, target, 4 * target,
                                                     start_frac=frac)
         if s >= warm:
-            rates.append(rate)
-    value = sum(rates) / len(rates)
-    ms_step = w.B * len(w.n_c) * n_c / value * 1e3 if len(w.n_c) == 1 else None
+            rates[c].append(rate)
+    # the whole step: every context's B heads at that context's mean sampled rate
+    t_step = sum(w.B * n_c / (sum(r) / len(r)) for n_c, r in zip(w.n_c, rates) if r)
+    pairs = sum(w.B * n_c for n_c, r in zip(w.n_c, rates) if r)
+    value = pairs / t_step
+    ms_step = t_step * 1e3 if all(rates) else None
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": steps, "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": "each step: one head of layer 0 (heads cycle, row blocks spread over the "
-                                       "input); the last step: " + desc +
-                                       "; ms_per_step extrapolated to the whole step (%d heads)" % w.B},
+                             "sample": "each step: one head of layer 0 (%sheads cycle, row blocks spread over the "
+                                       "input); the last step: " % ("contexts, then " if n_ctx > 1 else "") + desc +
+                                       "; value and ms_per_step extrapolated to the whole step (%d heads%s)"
+                                       % (w.B, " x %d contexts" % n_ctx if n_ctx > 1 else "")},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     if world > 1:
