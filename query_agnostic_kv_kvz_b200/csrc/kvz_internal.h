@@ -51,6 +51,7 @@ struct LseArgs {
   float2* part;             // [split CTAs][256] partial (reference, sum); null = no split
   int head_major;           // unit order: 0 = row block, then (head, group); 1 = head, then row block, then
                             // group (set by launch_lse)
+  int wave;                 // CTAs resident at once (the SM count; 0 = unknown) (set by launch_lse)
 };
 // Scratch for split units: at most this many split CTAs, 256 rows of
 // (max, sum) each.

@@ -190,6 +190,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NT = NC + nin[nq_valid - 1];                 // the unit's key tiles: context, then input
   const int t_lo = split ? static_cast<int>(static_cast<int64_t>(NT) * part / p.nsplit) : 0;
   const int NL = (split ? static_cast<int>(static_cast<int64_t>(NT) * (part + 1) / p.nsplit) : NT) - t_lo;
+  // Head-major order: when a head's CTAs span several waves, each wave
+  // walks the head's key tiles in the direction opposite to the wave before
+  // it, so it starts on the tiles that wave read last, which are still in
+  // L2.  Every loop below maps its local index j to tile tile_of(j).
+  bool rev = false;
+  if (p.head_major && p.wave > 0) {
+    const int u0 = b * nblk * p.G;
+    const int x0 = u0 < p.n_full ? u0 : p.n_full + (u0 - p.n_full) * p.nsplit;
+    rev = ((x / p.wave - x0 / p.wave) & 1) != 0;
+  }
+  auto tile_of = [rev, t_lo, NL](int j) { return rev ? t_lo + NL - 1 - j : t_lo + j; };
 
   const int n_issuers = KVZ_LSE_SPLIT_ISSUE ? nq_valid : 1;   // threads that commit to k_empty / drain
   if (threadIdx.x == 0) {
@@ -228,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(sQ + q * Lay::TILE_BYTES + kb * kSubBytes64, &tmQ, q_full, kb * 64,
                       static_cast<int>(i0 + q * kTile), bg);
       for (int j = 0; j < NL; ++j) {                   // ring slots follow the local tile index j
-        const int t = t_lo + j;
+        const int t = tile_of(j);
         const int s = j % Lay::KST;
         const uint32_t use = static_cast<uint32_t>(j / Lay::KST);
         if (!mbar_wait(&k_empty[s], (use & 1u) ^ 1u, abort_flag, p.status)) break;
@@ -254,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       tc_fence_after();
       for (int j = 0; ok && j < NL; ++j) {
-        const int t = t_lo + j;
+        const int t = tile_of(j);
         const int s = j % Lay::KST;
         const uint32_t use = static_cast<uint32_t>(j / Lay::KST);
         if (!mbar_wait(&k_full[s], use & 1u, abort_flag, p.status)) break;
@@ -307,7 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ctx_tail = static_cast<int>(p.n_c - static_cast<int64_t>(NC - 1) * kTile) - h * 64;
     const int diag_lim = rl - h * 64;                 // diagonal tile: column c visible iff c <= diag_lim
     uint32_t cnt = 0;
-    for (int t = t_lo; t < t_lo + NL; ++t) {
+    for (int j = 0; j < NL; ++j) {
+      const int t = tile_of(j);
       if (t >= NC && t - NC >= nin[q]) continue;
       const uint32_t buf = cnt & 1u;
       const uint32_t bu = cnt >> 1;
@@ -471,13 +483,14 @@ cudaError_t launch_lse(int d, const CUtensorMap& tmQ, const CUtensorMap& tmKc, c
   a.head_major = (a.rows_pad / kTile) * 8 <= (a.n_c + kTile - 1) / kTile ? 1 : 0;
   int64_t grid = units, r = 0;
   cudaError_t e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  a.wave = sms;                                     // one CTA per SM
   if (a.part != nullptr) {
-    // One CTA per SM: the units past the last full wave are split over key
-    // ranges so that the last wave fills the SMs.  The tail holds the
-    // shortest units (row block 0 of the call); a part keeps >= 8 tiles.
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    // The units past the last full wave are split over key ranges so that
+    // the last wave fills the SMs.  The tail holds the shortest units (row
+    // block 0 of the call); a part keeps >= 8 tiles.
     r = sms > 0 ? units % sms : 0;
     if (r > 0) {
       // the shortest tail unit: row block 0 of the call in either order

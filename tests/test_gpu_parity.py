@@ -115,6 +115,38 @@ def test_split_last_wave_matches_whole_units():
         assert np.all(np.isposinf(a[:, :, rows:])) and np.all(np.isposinf(b[:, :, rows:]))
 
 
+def test_lse2_head_major_waves_match_oracle_rows():
+    # A row pass much shorter than the context runs head-major: 8 heads x 5
+    # groups x 8 row blocks = 320 units, two full waves of 148 CTAs and a
+    # split tail, so heads 3 and 7 span two waves and their later CTAs walk
+    # the key tiles last to first.  Sampled rows of every (head, group, row
+    # block) against the oracle, with and without the split tail.
+    B, G, n_c, n_prompt, d = 8, 5, 16384, 32, 128
+    i0, i1 = 4096, 6144
+    x = _inputs(B, G, n_c, n_prompt, d, seed=41)
+    n_in = n_c + n_prompt
+    scale = f32_scale(d)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ld = i1 - i0
+    whole = torch.empty((B, G, ld), dtype=torch.float32, device="cuda")
+    kvz.lib().kvz_score_lse2(kvz._ptr(x["Q"]), kvz._ptr(x["K_ctx"]), kvz._ptr(x["K_in"]), B, G, n_c, n_in, d,
+                             scale, i0, i1, kvz._ptr(whole), ld, None, 0, kvz._ptr(st), kvz._stream(None))
+    split = kvz.kvz_score_lse2(x["Q"], x["K_ctx"], x["K_in"], i_begin=i0, i_end=i1, scale=scale, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    a, w = split.cpu().numpy(), whole.cpu().numpy()
+    np.testing.assert_allclose(a[:, :, :ld], w, rtol=0, atol=4e-6 * np.abs(w).max())
+    offs = [0, 97, 128, 255]
+    for b in range(B):
+        Kc, Ki = f64(x["K_ctx"][b]), f64(x["K_in"][b, :i1])
+        for g in range(G):
+            for blk in range(ld // 256):
+                for o in offs[(b + g + blk) % 2::2]:
+                    i = i0 + blk * 256 + o
+                    want = orc.row_lse(f64(x["Q"][b, g, i]), Kc, Ki, i, scale) / math.log(2)
+                    assert abs(float(a[b, g, i - i0]) - want) <= 2e-4, (b, g, i, float(a[b, g, i - i0]), want)
+
+
 def test_identical_keys_closed_form():
     # every causal row is uniform over its visible keys: S[j] = 1/(n_c+1)
     B, G, n_c, n_prompt, d = 2, 4, 1000, 32, 128
