@@ -49,13 +49,6 @@ constexpr int kPolyPer16 = KVZ_POLY_PER16;
 #ifndef KVZ_LSE_SPLIT_ISSUE
 #define KVZ_LSE_SPLIT_ISSUE 0
 #endif
-
-// 1: Q tiles, and in head-major order the key tiles of a head's last wave,
-// are fetched under an evict-first L2 policy (nothing reads them later);
-// 0: every tile under the default policy.
-#ifndef KVZ_LSE_L2_HINT
-#define KVZ_LSE_L2_HINT 1
-#endif
 static_assert(kPolyPer16 % 2 == 0 && kPolyPer16 >= 0 && kPolyPer16 <= 16, "pairs of exp2");
 
 template <int D>
@@ -200,16 +193,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Head-major order: when a head's CTAs span several waves, each wave
   // walks the head's key tiles in the direction opposite to the wave before
   // it, so it starts on the tiles that wave read last, which are still in
-  // L2.  Every loop below maps its local index j to tile tile_of(j).  The
-  // head's last wave fetches its key tiles evict-first (no later CTA reads
-  // them), which leaves L2 to the tiles of a head the next wave continues.
-  bool rev = false, last_wave = false;
+  // L2.  Every loop below maps its local index j to tile tile_of(j).
+  bool rev = false;
   if (p.head_major && p.wave > 0) {
-    const int u0 = b * nblk * p.G, u1 = u0 + nblk * p.G - 1;
+    const int u0 = b * nblk * p.G;
     const int x0 = u0 < p.n_full ? u0 : p.n_full + (u0 - p.n_full) * p.nsplit;
-    const int x1 = u1 < p.n_full ? u1 : p.n_full + (u1 - p.n_full) * p.nsplit + p.nsplit - 1;
     rev = ((x / p.wave - x0 / p.wave) & 1) != 0;
-    last_wave = KVZ_LSE_L2_HINT && x / p.wave == x1 / p.wave;
   }
   auto tile_of = [rev, t_lo, NL](int j) { return rev ? t_lo + NL - 1 - j : t_lo + j; };
 
@@ -244,17 +233,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmKc);
       prefetch_tmap(&tmKi);
-      const uint64_t once = l2_policy_evict_first();  // Q rows: read by this unit only
       mbar_arrive_expect_tx(q_full, nq_valid * Lay::TILE_BYTES);
       for (int q = 0; q < nq_valid; ++q)
-        for (int kb = 0; kb < Lay::KB; ++kb) {
-          if (KVZ_LSE_L2_HINT)
-            tma_load_3d_hint(sQ + q * Lay::TILE_BYTES + kb * kSubBytes64, &tmQ, q_full, kb * 64,
-                             static_cast<int>(i0 + q * kTile), bg, once);
-          else
-            tma_load_3d(sQ + q * Lay::TILE_BYTES + kb * kSubBytes64, &tmQ, q_full, kb * 64,
-                        static_cast<int>(i0 + q * kTile), bg);
-        }
+        for (int kb = 0; kb < Lay::KB; ++kb)
+          tma_load_3d(sQ + q * Lay::TILE_BYTES + kb * kSubBytes64, &tmQ, q_full, kb * 64,
+                      static_cast<int>(i0 + q * kTile), bg);
       for (int j = 0; j < NL; ++j) {                   // ring slots follow the local tile index j
         const int t = tile_of(j);
         const int s = j % Lay::KST;
@@ -262,18 +245,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&k_empty[s], (use & 1u) ^ 1u, abort_flag, p.status)) break;
         mbar_arrive_expect_tx(&k_full[s], Lay::TILE_BYTES);
         for (int kb = 0; kb < Lay::KB; ++kb) {
-          uint8_t* dst = sK + s * Lay::TILE_BYTES + kb * kSubBytes64;
-          if (t < NC) {   // context keys: block (b % T) of head (b / T)
-            if (last_wave)
-              tma_load_4d_hint(dst, &tmKc, &k_full[s], kb * 64, t * kTile, b % p.T, b / p.T, once);
-            else
-              tma_load_4d(dst, &tmKc, &k_full[s], kb * 64, t * kTile, b % p.T, b / p.T);
-          } else {
-            if (last_wave)
-              tma_load_3d_hint(dst, &tmKi, &k_full[s], kb * 64, (t - NC) * kTile, b, once);
-            else
-              tma_load_3d(dst, &tmKi, &k_full[s], kb * 64, (t - NC) * kTile, b);
-          }
+          if (t < NC)   // context keys: block (b % T) of head (b / T)
+            tma_load_4d(sK + s * Lay::TILE_BYTES + kb * kSubBytes64, &tmKc, &k_full[s], kb * 64, t * kTile,
+                        b % p.T, b / p.T);
+          else
+            tma_load_3d(sK + s * Lay::TILE_BYTES + kb * kSubBytes64, &tmKi, &k_full[s], kb * 64,
+                        (t - NC) * kTile, b);
         }
         issued = j + 1;
       }
