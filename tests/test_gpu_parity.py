@@ -115,15 +115,21 @@ def test_split_last_wave_matches_whole_units():
         assert np.all(np.isposinf(a[:, :, rows:])) and np.all(np.isposinf(b[:, :, rows:]))
 
 
-def test_lse2_head_major_waves_match_oracle_rows():
-    # A row pass much shorter than the context runs head-major: 8 heads x 5
-    # groups x 8 row blocks = 320 units, two full waves of 148 CTAs and a
-    # split tail, so heads 3 and 7 span two waves and their later CTAs walk
-    # the key tiles last to first.  Sampled rows of every (head, group, row
-    # block) against the oracle, with and without the split tail.
-    B, G, n_c, n_prompt, d = 8, 5, 16384, 32, 128
-    i0, i1 = 4096, 6144
-    x = _inputs(B, G, n_c, n_prompt, d, seed=41)
+@pytest.mark.parametrize("B,n_c,i0,i1,blocks", [
+    # 8 heads x 5 groups x 8 row blocks = 320 units: two full waves of 148
+    # CTAs and a split tail; heads 3 and 7 span two waves
+    (8, 16384, 4096, 6144, None),
+    # one head, 5 groups x 60 row blocks = 300 units: the head spans two
+    # full waves (forward, then backward) and a tail split 37 ways (forward)
+    (1, 122880, 8192, 23552, [59, 31, 30, 29, 15, 1, 0]),
+])
+def test_lse2_head_major_waves_match_oracle_rows(B, n_c, i0, i1, blocks):
+    # A row pass much shorter than the context runs head-major, and a head
+    # whose CTAs span several waves walks its key tiles in alternating
+    # directions.  Sampled rows of the (head, group, row block) units against
+    # the oracle, with and without the split tail.
+    G, n_prompt, d = 5, 32, 128
+    x = _inputs(B, G, n_c, n_prompt, d, seed=41 + B)
     n_in = n_c + n_prompt
     scale = f32_scale(d)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -140,8 +146,8 @@ def test_lse2_head_major_waves_match_oracle_rows():
     for b in range(B):
         Kc, Ki = f64(x["K_ctx"][b]), f64(x["K_in"][b, :i1])
         for g in range(G):
-            for blk in range(ld // 256):
-                for o in offs[(b + g + blk) % 2::2]:
+            for blk in (range(ld // 256) if blocks is None else blocks):
+                for o in (offs[(b + g + blk) % 2::2] if blocks is None else offs[(g + blk) % 4:][:1]):
                     i = i0 + blk * 256 + o
                     want = orc.row_lse(f64(x["Q"][b, g, i]), Kc, Ki, i, scale) / math.log(2)
                     assert abs(float(a[b, g, i - i0]) - want) <= 2e-4, (b, g, i, float(a[b, g, i - i0]), want)
